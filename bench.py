@@ -1,0 +1,432 @@
+"""Benchmark of the BeaconKV compression step on B200.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl bkv|reference]
+
+One step = one whole compression step (Continual FPS over the newest window,
+tensor-core scoring with max aggregation, top-K, compaction) over every
+(layer, KV head) of the workload, through the C ABI (bkv_compress_step), with
+the inputs resident in HBM.  For N > 1 (launched with torch.distributed.run)
+every rank compresses its own independent cache of the same shape (weak
+scaling; the heads are independent, so no collective is on the data path);
+the timed region is bracketed by a barrier and a device synchronise on every
+rank and the slowest rank's time is reported.
+
+Rank 0 prints one JSON line.  `value` is the number of KV entries (layer, KV
+head, position) scored, selected and compacted per second by all ranks.
+`e2e` is the same metric when each step also copies its inputs from pinned
+host memory and reads the compacted cache back.  `roofline` is the dominant
+kernel's achieved rate against the measured B200 peak; `cpu_baseline` is the
+float64 oracle timed on a bounded sample on this host.  `--impl reference`
+times only that oracle (the baseline arm).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+METRIC = "KV entries scored+selected+compacted/s per compression step"
+UNIT = "entries/s"
+PHASES = ["fps", "row_stats", "aggregate", "select", "compact"]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm_gbs=p["hbm_gbs"], bf16_tflops=p["bf16_tflops"],
+                    bf16_tflops_sustained=p.get("bf16_tflops_sustained", p["bf16_tflops"]),
+                    sm_max_mhz=p.get("sm_max_mhz", 1965.0), source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0,
+                sm_max_mhz=1965.0, source="fallback")
+
+
+# ----------------------------------------------------------------------------
+# algorithmic work per phase (per step, one rank)
+# ----------------------------------------------------------------------------
+def work_model(wl):
+    H = wl.n_layers * wl.n_kv_heads
+    Hq = wl.n_layers * wl.n_q_heads
+    nb = min(wl.M, wl.beacons_in + wl.W) if wl.W else wl.beacons_in
+    n_obs = wl.group * (wl.R + nb)
+    d, L, K = wl.head_dim, wl.L, min(wl.K, wl.L)
+    es = 2 if wl.dtype == "bf16" else 4
+    n_groups = (n_obs + 511) // 512
+    contraction = 2.0 * n_obs * L * d * H
+    return {
+        "fps": {"bound": "alu", "work": float(Hq) * wl.M * (wl.beacons_in + wl.W) * d,
+                "unit": "FMA"},
+        "row_stats": {"bound": "tensor", "work": contraction, "unit": "FLOP"},
+        "aggregate": {"bound": "tensor", "work": contraction, "unit": "FLOP"},
+        "select": {"bound": "hbm", "work": float(H) * (n_groups * 4 * L + 4 * K), "unit": "B"},
+        "compact": {"bound": "hbm", "work": float(H) * 4 * K * d * es, "unit": "B"},
+        # the step: one contraction + the algorithmic bytes of the whole step
+        "step_flop": contraction,
+        "step_bytes": float(H) * (L * d * es + n_obs * d * es + 2 * 4 * L + 2 * 4 * K
+                                  + 4 * K * d * es),
+    }
+
+
+def peak_for(bound, peaks):
+    if bound == "tensor":
+        return peaks["bf16_tflops_sustained"], "TFLOP/s"
+    if bound == "hbm":
+        return peaks["hbm_gbs"], "GB/s"
+    # FP32 FMA pipe: 148 SMs x 128 FMA/clk at the max SM clock
+    return 148 * 128 * peaks["sm_max_mhz"] * 1e6 / 1e12, "TFMA/s"
+
+
+def rate(work, unit, seconds):
+    if unit == "FLOP":
+        return work / seconds / 1e12
+    if unit == "B":
+        return work / seconds / 1e9
+    return work / seconds / 1e12
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.path = None
+        try:
+            bus = torch.cuda.get_device_properties(device_index).pci_bus_id
+        except Exception:
+            bus = None
+        self.sel = ["-i", bus] if bus else []
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="bkv_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", *self.sel, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------
+# the float64 oracle on a bounded sample (CPU baseline / reference arm)
+# ----------------------------------------------------------------------------
+def oracle_sample(wl, seed: int, n_heads: int, L_sample: int):
+    """Run the oracle's whole step on n_heads (layer, KV head)s, one thread
+    each, with each head's keys cut to its first L_sample rows.  Returns
+    (entries, seconds, threads)."""
+    import oracle
+    from kv_cache_compression_bkv_b200 import synth
+
+    wls = wl.replace(L=L_sample, capacity=L_sample, K=min(wl.K, L_sample))
+    jobs = []
+    for i in range(n_heads):
+        l, h = divmod(i, wl.n_kv_heads)
+        l %= wl.n_layers
+        k, v = synth.keys_values(wls, seed, l, h)
+        qs = [synth.head_queries(wls, seed, l, h * wl.group + g) for g in range(wl.group)]
+        recent = np.stack([q[0].to(wls.torch_dtype).double().numpy() for q in qs])
+        beac = np.stack([q[1].to(wls.torch_dtype).double().numpy() for q in qs])
+        win = np.stack([q[2].to(wls.torch_dtype).double().numpy() for q in qs]) if wl.W else None
+        jobs.append((k.to(wls.torch_dtype).double().numpy(), v.to(wls.torch_dtype).double().numpy(),
+                     recent, beac, win))
+    oracle.lib()
+    done = []
+
+    def run(job):
+        k, v, r, b, w = job
+        out = oracle.compress_head(k, v, r, b, wls.beacons_in, w, wls.M, wls.K)
+        done.append(len(out["idx"]))
+
+    threads = [threading.Thread(target=run, args=(j,)) for j in jobs]
+    t0 = time.perf_counter()
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+    dt = time.perf_counter() - t0
+    return n_heads * L_sample, dt, len(threads)
+
+
+def cpu_threads() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, wl, rank, world):
+    if rank != 0:
+        return
+    n_thr = max(1, min(cpu_threads(), 16))
+    # size the per-step sample so that warmup + steps stay within ~2.5 minutes
+    ent, dt, _ = oracle_sample(wl, args.seed, 1, 1024)
+    per_key = dt / 1024.0
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    L_sample = int(max(256, min(wl.L, budget / max(per_key, 1e-9))))
+    L_sample = max(256, L_sample // 256 * 256)
+    for _ in range(args.warmup):
+        oracle_sample(wl, args.seed, n_thr, L_sample)
+    tot_e, tot_t = 0, 0.0
+    for _ in range(args.steps):
+        e, t, _ = oracle_sample(wl, args.seed, n_thr, L_sample)
+        tot_e += e
+        tot_t += t
+    value = tot_e / tot_t
+    sample = (f"per step: {n_thr} (layer, KV head)s of {wl.name} in parallel threads, the whole "
+              f"step (FPS over W={wl.W}, scoring, top-K, compaction) on the first {L_sample} "
+              f"of L={wl.L} keys of each head")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": n_thr, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------
+# the CUDA path
+# ----------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="qwen3_14b")
+    ap.add_argument("--impl", default="bkv", choices=["bkv", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=None)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    from kv_cache_compression_bkv_b200 import synth
+    wl = synth.WORKLOADS[args.workload]
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, wl, rank, world)
+        return
+
+    from kv_cache_compression_bkv_b200 import bkv
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    inp = synth.make_step_inputs(wl, seed=args.seed + rank, pin=True)
+    g = bkv.geometry_of(inp.k, wl.n_q_heads)
+    keep = min(wl.K, wl.L)
+    dstg = bkv.Geometry(g.n_layers, g.n_q_heads, g.n_kv_heads, g.head_dim, keep, g.dtype)
+    names = ("k", "v", "recent", "beacons", "window")
+    host = {n: getattr(inp, n) for n in names}
+    devt = {n: torch.empty_like(host[n], device=dev) for n in names}
+    for n in names:
+        devt[n].copy_(host[n])
+    kd = torch.empty(wl.n_layers, wl.n_kv_heads, keep, wl.head_dim, dtype=inp.k.dtype, device=dev)
+    vd = torch.empty_like(kd)
+    bout = torch.empty_like(devt["beacons"])
+    idx = torch.empty(wl.n_layers, wl.n_kv_heads, keep, dtype=torch.int32, device=dev)
+    ws = torch.empty(bkv.bkv_workspace_size(g, wl.L, wl.R, wl.M, wl.W, wl.K), dtype=torch.uint8,
+                     device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(events=None, t=devt):
+        return bkv.bkv_compress_step(g, t["k"], t["v"], wl.L, wl.K, t["recent"], wl.R,
+                                     t["beacons"], wl.beacons_in, wl.M,
+                                     t["window"] if wl.W else None, wl.W, bout, 0.0, dstg, kd,
+                                     vd, None, idx, ws, stream, events)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st, where = bkv.bkv_read_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} at {where} during warm-up")
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(bkv.STEP_EVENTS)]
+          for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.25)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(ev[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    st, where = bkv.bkv_read_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} at {where} in the timed region")
+    ms_local = t_start.elapsed_time(t_end) / args.steps
+    phase_ms = {p: sum(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(args.steps)) / args.steps
+                for j, p in enumerate(PHASES)}
+    ms = ms_local
+    if dist is not None:
+        tt = torch.tensor([ms_local], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    entries = wl.n_layers * wl.n_kv_heads * wl.L
+    value = world * entries / (ms / 1e3)
+
+    # ---- end to end: pinned host inputs in, compacted cache out, every step
+    e2e_steps = args.e2e_steps or max(3, min(args.steps, 10))
+    out_host = {"kd": torch.empty_like(kd, device="cpu").pin_memory(),
+                "vd": torch.empty_like(vd, device="cpu").pin_memory(),
+                "bout": torch.empty_like(bout, device="cpu").pin_memory(),
+                "idx": torch.empty_like(idx, device="cpu").pin_memory()}
+    h2d = sum(host[n].numel() * host[n].element_size() for n in names if n != "window" or wl.W)
+    d2h = sum(t.numel() * t.element_size() for t in out_host.values())
+    barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        for n in names:
+            devt[n].copy_(host[n], non_blocking=True)
+        step()
+        out_host["kd"].copy_(kd, non_blocking=True)
+        out_host["vd"].copy_(vd, non_blocking=True)
+        out_host["bout"].copy_(bout, non_blocking=True)
+        out_host["idx"].copy_(idx, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if dist is not None:
+        tt = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+
+    if rank != 0:
+        if dist is not None:
+            dist.destroy_process_group()
+        return
+
+    peaks = load_peaks()
+    wm = work_model(wl)
+    phases = {}
+    for p in PHASES:
+        m = wm[p]
+        pk, pu = peak_for(m["bound"], peaks)
+        sec = phase_ms[p] / 1e3
+        ach = rate(m["work"], m["unit"], sec) if sec > 0 else 0.0
+        phases[p] = {"ms": phase_ms[p], "bound": m["bound"], "achieved": ach, "peak": pk,
+                     "unit": pu, "frac": ach / pk if pk else None}
+    dom = max(PHASES, key=lambda p: phase_ms[p])
+    dm = phases[dom]
+    per_launch = wm[dom]["work"]
+    roofline = {"bound": dm["bound"], "achieved": dm["achieved"], "peak": dm["peak"],
+                "unit": dm["unit"], "frac": dm["frac"], "traffic": None, "kernel": dom,
+                "peak_source": peaks["source"] + (" sustained" if dm["bound"] == "tensor" else ""),
+                "work_per_launch": per_launch}
+    t_tensor = wm["step_flop"] / (peaks["bf16_tflops_sustained"] * 1e12)
+    t_hbm = wm["step_bytes"] / (peaks["hbm_gbs"] * 1e9)
+    t_roof = max(t_tensor, t_hbm)
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        n_thr = max(1, min(cpu_threads(), 4))
+        e, t, used = oracle_sample(wl, args.seed, n_thr, wl.L)
+        cpu = {"value": e / t, "unit": UNIT, "cores": used, "kind": "oracle",
+               "sample": f"{n_thr} (layer, KV head)s of {wl.name}, the whole step each "
+                         f"(FPS over W={wl.W}, scoring all L={wl.L} keys, top-K, compaction), "
+                         f"one thread per head, {t:.1f} s wall"}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "n_layers": wl.n_layers, "n_q_heads": wl.n_q_heads,
+                   "n_kv_heads": wl.n_kv_heads, "head_dim": wl.head_dim, "L": wl.L, "R": wl.R,
+                   "M": wl.M, "K": wl.K, "W": wl.W,
+                   "l2": "inputs larger than L2 (K/V cache %.1f GB per step)"
+                         % (2 * inp.k.numel() * inp.k.element_size() / 1e9)},
+        "step_us": ms * 1e3,
+        "pct_roofline": 100.0 * t_roof / (ms / 1e3),
+        "t_roof_us": t_roof * 1e6,
+        "roofline": roofline,
+        "phases": phases,
+        "cpu_baseline": cpu,
+        "e2e": {"value": world * entries / (e2e_ms / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "clocks": clk,
+        "gpu_launches": (5 if wl.W else 4) * args.steps,
+    }
+    print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

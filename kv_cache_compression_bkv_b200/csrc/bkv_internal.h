@@ -1,0 +1,120 @@
+// bkv_internal.h -- geometry shared by the host layer and the kernels of
+// libbkv.so, and the launchers each kernel file exports.  Not installed; the
+// public interface is include/bkv.h.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/bkv.h"
+
+namespace bkv {
+
+constexpr size_t kAlign = 256;  // alignment of every workspace section
+
+__host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// One scoring problem: all (layer, KV head) pairs of a cache, each with its
+// observation set of G * (R + nb) query rows (the R recent queries and the
+// first nb beacons of each of the G query heads of the group).
+struct ScoreGeom {
+  int n_layers, n_q_heads, n_kv_heads, head_dim, group;
+  long long cap;        // rows allocated per (layer, KV head)
+  long long L;          // rows scored
+  int R, nb, M;         // recent rows, valid beacons, beacon slots
+  int n_obs;            // observation rows per KV head
+  int n_obs_pad;        // n_obs rounded up to the row-statistics block (128)
+  int n_groups;         // observation groups of the aggregation pass
+  int rows_per_group;   // rows per group, a multiple of 16, at most 512
+  float scale;          // logit scale
+  __host__ __device__ int n_heads() const { return n_layers * n_kv_heads; }
+};
+
+// Fill the derived fields of a ScoreGeom (n_obs, padding, groups).
+void finish_score_geom(ScoreGeom *g);
+
+// Workspace sections of the scoring passes.
+struct ScoreWorkspace {
+  float *c;      // [n_heads][n_obs_pad]  row normalisers (natural log units)
+  float *ypart;  // [n_groups][n_heads][L] max over a group of (x - c)
+};
+size_t score_workspace_bytes(const ScoreGeom &g);
+ScoreWorkspace carve_score_workspace(const ScoreGeom &g, void *ws);
+
+// ---- score_tc.cu: bf16, head_dim 128, tcgen05 tensor cores
+bkv_status launch_score_rowstats_tc(const ScoreGeom &g, const void *k, const void *recent,
+                                    const void *beacons, float *c, cudaStream_t stream);
+bkv_status launch_score_colmax_tc(const ScoreGeom &g, const void *k, const void *recent,
+                                  const void *beacons, const float *c, float *ypart,
+                                  cudaStream_t stream);
+
+// ---- score_simt.cu: f32, head_dim <= 128 (multiple of 4), CUDA cores
+bkv_status launch_score_rowstats_simt(const ScoreGeom &g, const float *k, const float *recent,
+                                      const float *beacons, float *c, cudaStream_t stream);
+bkv_status launch_score_colmax_simt(const ScoreGeom &g, const float *k, const float *recent,
+                                    const float *beacons, const float *c, float *ypart,
+                                    cudaStream_t stream);
+
+// ---- select_topk.cu
+// Selection input: per row r and position j, the key is
+//   max over p < n_parts of  src[p * part_stride + r * L + j].
+// When s_out is given, exp(key) is also written to s_out[r * L + j] (used when
+// src holds log-domain partial scores).
+struct SelectInput {
+  const float *src;
+  int n_parts;
+  size_t part_stride;
+};
+size_t select_workspace_bytes(int n_rows, long long L);
+bkv_status launch_select_topk(const SelectInput &in, int n_rows, long long L, long long K,
+                              int32_t *idx, float *s_out, void *ws, size_t ws_bytes,
+                              cudaStream_t stream);
+// s[r][j] = exp(max_p src[p][r][j]) for every row and position.
+bkv_status launch_finalize_scores(const SelectInput &in, int n_rows, long long L, float *s,
+                                  cudaStream_t stream);
+// idx[r][i] = i for i < n.
+bkv_status launch_iota_rows(int32_t *idx, int n_rows, long long n, cudaStream_t stream);
+
+// ---- compact.cu
+struct CompactArgs {
+  const uint8_t *k_src, *v_src;
+  uint8_t *k_dst, *v_dst;
+  const int32_t *idx;        // [n_heads][n_keep]; NULL = identity
+  int n_heads;
+  long long n_keep;
+  long long src_cap, dst_cap;  // rows per head
+  int row_bytes;               // multiple of 16
+};
+bkv_status launch_compact(const CompactArgs &a, cudaStream_t stream);
+
+// ---- fps.cu
+struct FpsGeom {
+  int n_layers, n_q_heads, head_dim, dtype;
+  int nb_in, M, W;
+  int n_pick;  // min(M, nb_in + W)
+};
+size_t fps_workspace_bytes(const FpsGeom &g);
+bool fps_supported(const FpsGeom &g);
+bkv_status launch_fps(const FpsGeom &g, const void *beacons_in, const void *window,
+                      void *beacons_out, void *ws, size_t ws_bytes, cudaStream_t stream);
+
+// Raise a kernel's dynamic shared-memory limit once per device (the attribute
+// is per device context).  Returns false if the CUDA call fails.
+template <typename Kernel>
+bool ensure_smem_limit(Kernel kernel, int bytes, int *done_flags /* [64] */) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  if (__atomic_load_n(&done_flags[dev], __ATOMIC_ACQUIRE)) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+      cudaSuccess)
+    return false;
+  __atomic_store_n(&done_flags[dev], 1, __ATOMIC_RELEASE);
+  return true;
+}
+
+// ---- per-file device status accessors (bkv_device_status.cuh)
+int take_status_score_tc(cudaStream_t, int *);
+int take_status_select(cudaStream_t, int *);
+
+}  // namespace bkv

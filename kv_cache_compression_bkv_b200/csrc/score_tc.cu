@@ -1,0 +1,544 @@
+// score_tc.cu -- attention-based scores with max aggregation on the sm_100a
+// tensor cores (BeaconKV, Fig. 5(b)/(c); Table 2 "Max").
+//
+// For one (layer, KV head) with observation rows q_o and keys k_j (bf16,
+// head_dim 128) the scores are
+//     x_oj = scale * q_o . k_j,   c_o = log sum_j exp(x_oj),
+//     y_j  = max_o (x_oj - c_o),  s_j = exp(y_j).
+// c_o needs every key before any y_j is final, so the contraction runs twice:
+//
+//   pass 1 (row statistics)   D[o][j] = Q_blk . K_tile^T, M = 128 observation
+//     rows, N = 256 keys.  TMEM lane = observation row, so each epilogue
+//     thread owns one row and keeps an online (max, sum of exp2) over the
+//     columns it reads; no cross-thread reduction per element.
+//   pass 2 (column max)       D[j][o] = K_tile . Q_grp^T, M = 128 keys, N =
+//     up to 2 x 256 observation rows.  TMEM lane = key, so each epilogue
+//     thread owns one key and reduces max_o (acc - c_o / scale) in registers.
+//
+// Both passes: warp 0 issues TMA loads of the key tiles (128-byte swizzle, no
+// multicast) into a ring of shared-memory stages; warp 1 allocates TMEM and
+// issues tcgen05.mma from one thread, committing to mbarriers; the epilogue
+// warps read the f32 accumulators with tcgen05.ld.  The observation rows are
+// gathered once per CTA from the recent-query and beacon tensors with plain
+// 16-byte loads and written to shared memory in the same swizzled layout.
+// Every wait is bounded (sm100.cuh).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "bkv_internal.h"
+#include "sm100.cuh"
+
+BKV_DEFINE_STATUS_ACCESSOR(take_status_score_tc)
+
+namespace bkv {
+namespace {
+
+using namespace sm100;
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr int kDim = 128;            // head_dim of the tensor-core path
+constexpr int kRowBytes = kDim * 2;  // one bf16 row
+constexpr int kKbBytes = 128;        // one 64-element K block of a row
+
+// Wait-site tags recorded with a timeout.
+enum { kWhereP1Prod = 101, kWhereP1Mma = 102, kWhereP1Epi = 103, kWhereP1Drain = 104,
+       kWhereP2Prod = 201, kWhereP2Mma = 202, kWhereP2Epi = 203, kWhereP2Drain = 204 };
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+__device__ __forceinline__ uint4 ldg_nc_v4(const void *p) {
+  uint4 v;
+  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+// Pointer to observation row o of KV head (layer, kvh): query head g of the
+// group, row i of [recent (R rows); beacons (nb rows)].
+__device__ __forceinline__ const uint16_t *obs_row(const ScoreGeom &g, const uint16_t *recent,
+                                                   const uint16_t *beacons, int layer, int kvh,
+                                                   int o) {
+  const int per = g.R + g.nb;
+  const int gq = o / per;
+  const int i = o - gq * per;
+  const long long qh = static_cast<long long>(layer) * g.n_q_heads +
+                       static_cast<long long>(kvh) * g.group + gq;
+  if (i < g.R) return recent + (qh * g.R + i) * kDim;
+  return beacons + (qh * g.M + (i - g.R)) * kDim;
+}
+
+// Gather observation rows [row0, row0 + nrows) into shared memory as a
+// K-major operand: two K blocks of nrows x 128 B, 128-byte swizzle.  Rows at
+// or past n_obs are zero.
+__device__ __forceinline__ void load_obs_rows_sw128(uint8_t *dst, int nrows, int row0,
+                                                    const ScoreGeom &g, const uint16_t *recent,
+                                                    const uint16_t *beacons, int layer,
+                                                    int kvh) {
+  const int kb_stride = nrows * kKbBytes;
+  for (int id = threadIdx.x; id < nrows * 16; id += blockDim.x) {
+    const int r = id >> 4, c16 = id & 15, kb = c16 >> 3, c = c16 & 7;
+    const int o = row0 + r;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (o < g.n_obs) v = ldg_nc_v4(obs_row(g, recent, beacons, layer, kvh, o) + c16 * 8);
+    *reinterpret_cast<uint4 *>(dst + kb * kb_stride + sw128_offset(r, c)) = v;
+  }
+}
+
+// ------------------------------------------------------------------ pass 1
+constexpr int kP1Rows = 128;
+constexpr int kP1Keys = 256;
+constexpr int kP1Stages = 3;
+constexpr int kP1Threads = 384;  // warp 0 TMA, warp 1 MMA, warps 4..11 epilogue
+constexpr int kP1ABytes = kP1Rows * kRowBytes;     // 32 KB
+constexpr int kP1StageBytes = kP1Keys * kRowBytes; // 64 KB
+constexpr int kP1SmallBytes = 2048;                // barriers, TMEM slot, exchange
+constexpr int kP1SmemBytes = kP1SmallBytes + 1024 + kP1ABytes + kP1Stages * kP1StageBytes;
+
+__global__ void __launch_bounds__(kP1Threads, 1)
+    score_rowstats_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreGeom g,
+                          const uint16_t *__restrict__ recent,
+                          const uint16_t *__restrict__ beacons, float *__restrict__ c_out) {
+  extern __shared__ uint8_t smem_raw[];
+  // small objects first, then the 1024-aligned operand tiles
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem_raw);  // 16 barriers
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem_raw + 128);
+  float *xchg = reinterpret_cast<float *>(smem_raw + 1024);  // [128][2]
+  const uint32_t raw_base = smem_u32(smem_raw);
+  const uint32_t tile_base = (raw_base + kP1SmallBytes + 1023u) & ~1023u;
+  uint8_t *sA = smem_raw + (tile_base - raw_base);
+  uint8_t *sB = sA + kP1ABytes;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int head = blockIdx.y, rb = blockIdx.x;
+  const int layer = head / g.n_kv_heads, kvh = head - layer * g.n_kv_heads;
+  const long long L = g.L;
+  const int n_tiles = static_cast<int>((L + kP1Keys - 1) / kP1Keys);
+
+  const uint32_t full0 = smem_u32(&bars[0]);    // [stages]
+  const uint32_t empty0 = smem_u32(&bars[4]);   // [stages]
+  const uint32_t tfull0 = smem_u32(&bars[8]);   // [2]
+  const uint32_t tempty0 = smem_u32(&bars[10]); // [2]
+  const uint32_t done = smem_u32(&bars[12]);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kP1Stages; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull0 + 8 * a, 1);
+      mbar_init(tempty0 + 8 * a, 8);  // one arrive per epilogue warp
+    }
+    mbar_init(done, 1);
+    fence_barrier_init();
+    prefetch_tensormap(&kmap);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  load_obs_rows_sw128(sA, kP1Rows, rb * kP1Rows, g, recent, beacons, layer, kvh);
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---- TMA producer
+      const int krow0 = static_cast<int>(static_cast<long long>(head) * g.cap);
+      int issued = 0;
+      for (int t = 0; t < n_tiles; ++t) {
+        const int s = t % kP1Stages;
+        const uint32_t ph = (t / kP1Stages) & 1;
+        if (!mbar_wait(empty0 + 8 * s, ph ^ 1, kWhereP1Prod)) break;
+        mbar_arrive_expect_tx(full0 + 8 * s, kP1StageBytes);
+        const uint32_t dst = smem_u32(sB + s * kP1StageBytes);
+        tma_load_2d(dst, &kmap, full0 + 8 * s, 0, krow0 + t * kP1Keys);
+        tma_load_2d(dst + kP1Keys * kKbBytes, &kmap, full0 + 8 * s, 64, krow0 + t * kP1Keys);
+        issued = t + 1;
+      }
+      // wait for the loads still in flight before the CTA may exit
+      for (int t = issued > kP1Stages ? issued - kP1Stages : 0; t < issued; ++t)
+        mbar_wait(full0 + 8 * (t % kP1Stages), (t / kP1Stages) & 1, kWhereP1Drain);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---- MMA issuer
+      constexpr uint32_t idesc = idesc_bf16_f32(kP1Rows, kP1Keys);
+      const uint32_t a_base = smem_u32(sA);
+      for (int t = 0; t < n_tiles; ++t) {
+        const int s = t % kP1Stages, acc = t & 1;
+        if (!mbar_wait(full0 + 8 * s, (t / kP1Stages) & 1, kWhereP1Mma)) break;
+        if (!mbar_wait(tempty0 + 8 * acc, ((t >> 1) & 1) ^ 1, kWhereP1Mma)) break;
+        tc_fence_after();
+        const uint32_t b_base = smem_u32(sB + s * kP1StageBytes);
+        const uint32_t d = tmem + acc * kP1Keys;
+#pragma unroll
+        for (int kb = 0; kb < 2; ++kb) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = smem_desc_k_sw128(a_base + kb * (kP1Rows * kKbBytes) + kk * 32);
+            const uint64_t bd = smem_desc_k_sw128(b_base + kb * (kP1Keys * kKbBytes) + kk * 32);
+            umma_f16(d, ad, bd, idesc, (kb | kk) != 0);
+          }
+        }
+        umma_commit(empty0 + 8 * s);
+        umma_commit(tfull0 + 8 * acc);
+      }
+      umma_commit(done);
+      mbar_wait(done, 0, kWhereP1Drain);
+    }
+  } else if (warp >= 4) {
+    // ---- epilogue: two warpgroups split the 256 columns of each tile
+    const int wg = (warp - 4) >> 2;
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const float kz = g.scale * kLog2e;
+    float m = -INFINITY, ssum = 0.f;
+    bool ok = true;
+    for (int t = 0; t < n_tiles && ok; ++t) {
+      const int acc = t & 1;
+      if (!mbar_wait(tfull0 + 8 * acc, (t >> 1) & 1, kWhereP1Epi)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) +
+                             acc * kP1Keys + wg * 128;
+      const long long key_base = static_cast<long long>(t) * kP1Keys + wg * 128;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        float v[32];
+        tmem_ld_32x32b_x32(taddr + c * 32, v);
+        tmem_ld_wait();
+        const long long k0 = key_base + c * 32;
+        if (k0 + 32 > L) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (k0 + i >= L) v[i] = -INFINITY;
+        }
+        float cm = v[0];
+#pragma unroll
+        for (int i = 1; i < 32; ++i) cm = fmaxf(cm, v[i]);
+        const float mz = cm * kz;
+        if (mz > m) {
+          ssum *= ex2_approx(m - mz);
+          m = mz;
+        }
+        if (m == -INFINITY) continue;  // every column seen so far is masked
+        float cs0 = 0.f, cs1 = 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          cs0 += ex2_approx(fmaf(v[i], kz, -m));
+          cs1 += ex2_approx(fmaf(v[i + 1], kz, -m));
+        }
+        ssum += cs0 + cs1;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
+    }
+    // combine the two column halves of each row
+    if (wg == 1) {
+      xchg[row * 2] = m;
+      xchg[row * 2 + 1] = ok ? ssum : -1.f;
+    }
+    named_barrier_sync(1, 256);
+    if (wg == 0) {
+      const float m1 = xchg[row * 2], s1 = xchg[row * 2 + 1];
+      const int o = rb * kP1Rows + row;
+      if (ok && s1 >= 0.f && o < g.n_obs) {
+        const float M = fmaxf(m, m1);
+        const float S = (m == -INFINITY ? 0.f : ssum * ex2_approx(m - M)) +
+                        (m1 == -INFINITY ? 0.f : s1 * ex2_approx(m1 - M));
+        c_out[static_cast<size_t>(head) * g.n_obs_pad + o] = (M + log2f(S)) * kLn2;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------ pass 2
+constexpr int kP2Keys = 128;
+constexpr int kP2MaxRows = 512;
+constexpr int kP2Threads = 256;  // warp 0 TMA, warp 1 MMA, warps 2..3 loaders, 4..7 epilogue
+constexpr int kP2TileBytes = kP2Keys * kRowBytes;  // 32 KB
+constexpr int kP2SmallBytes = 256 + kP2MaxRows * 4; // barriers + TMEM slot, c / scale
+
+__host__ __device__ constexpr int p2_smem_bytes(int rows_pad, int stages) {
+  return kP2SmallBytes + 1024 + rows_pad * kRowBytes + stages * kP2TileBytes;
+}
+
+__global__ void __launch_bounds__(kP2Threads, 1)
+    score_colmax_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreGeom g,
+                        const uint16_t *__restrict__ recent, const uint16_t *__restrict__ beacons,
+                        const float *__restrict__ c_in, float *__restrict__ ypart, int n_chunks,
+                        int chunk_tiles, int n_stages) {
+  extern __shared__ uint8_t smem_raw[];
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem_raw);  // 16 barriers
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem_raw + 128);
+  float *ct = reinterpret_cast<float *>(smem_raw + 256);   // [512] c_o / scale
+  const uint32_t raw_base = smem_u32(smem_raw);
+  const uint32_t tile_base = (raw_base + kP2SmallBytes + 1023u) & ~1023u;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int bid = blockIdx.x;
+  const int gi = bid % g.n_groups;
+  bid /= g.n_groups;
+  const int ci = bid % n_chunks;
+  const int head = bid / n_chunks;
+  const int layer = head / g.n_kv_heads, kvh = head - layer * g.n_kv_heads;
+  const long long L = g.L;
+  const int n_tiles_all = static_cast<int>((L + kP2Keys - 1) / kP2Keys);
+  const int t0 = ci * chunk_tiles;
+  const int t1 = min(n_tiles_all, t0 + chunk_tiles);
+  const int n_tiles = t1 > t0 ? t1 - t0 : 0;
+
+  const int r0 = gi * g.rows_per_group;
+  const int nrows = min(g.rows_per_group, g.n_obs - r0);
+  const int rows_pad = (nrows + 15) & ~15;
+  const int N0 = min(256, rows_pad);
+  const int N1 = rows_pad - N0;
+  const int n_sub = N1 > 0 ? 2 : 1;
+
+  uint8_t *sQ = smem_raw + (tile_base - raw_base);
+  uint8_t *sK = sQ + rows_pad * kRowBytes;
+
+  const uint32_t full0 = smem_u32(&bars[0]);    // [<=4]
+  const uint32_t empty0 = smem_u32(&bars[4]);   // [<=4]
+  const uint32_t tfull0 = smem_u32(&bars[8]);   // [2]
+  const uint32_t tempty0 = smem_u32(&bars[10]); // [2]
+  const uint32_t done = smem_u32(&bars[12]);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < n_stages; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int u = 0; u < 2; ++u) {
+      mbar_init(tfull0 + 8 * u, 1);
+      mbar_init(tempty0 + 8 * u, 4);  // one arrive per epilogue warp
+    }
+    mbar_init(done, 1);
+    fence_barrier_init();
+    prefetch_tensormap(&kmap);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  const float inv_scale = 1.0f / g.scale;
+  for (int r = threadIdx.x; r < kP2MaxRows; r += blockDim.x)
+    ct[r] = (r < nrows) ? c_in[static_cast<size_t>(head) * g.n_obs_pad + r0 + r] * inv_scale
+                        : INFINITY;
+  load_obs_rows_sw128(sQ, rows_pad, r0, g, recent, beacons, layer, kvh);
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const int krow0 = static_cast<int>(static_cast<long long>(head) * g.cap);
+      int issued = 0;
+      for (int it = 0; it < n_tiles; ++it) {
+        const int t = t0 + it;
+        const int s = it % n_stages;
+        const uint32_t ph = (it / n_stages) & 1;
+        if (!mbar_wait(empty0 + 8 * s, ph ^ 1, kWhereP2Prod)) break;
+        mbar_arrive_expect_tx(full0 + 8 * s, kP2TileBytes);
+        const uint32_t dst = smem_u32(sK + s * kP2TileBytes);
+        tma_load_2d(dst, &kmap, full0 + 8 * s, 0, krow0 + t * kP2Keys);
+        tma_load_2d(dst + kP2Keys * kKbBytes, &kmap, full0 + 8 * s, 64, krow0 + t * kP2Keys);
+        issued = it + 1;
+      }
+      for (int it = issued > n_stages ? issued - n_stages : 0; it < issued; ++it)
+        mbar_wait(full0 + 8 * (it % n_stages), (it / n_stages) & 1, kWhereP2Drain);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc0 = idesc_bf16_f32(kP2Keys, N0);
+      const uint32_t idesc1 = idesc_bf16_f32(kP2Keys, N1 > 0 ? N1 : 16);
+      const uint32_t q_base = smem_u32(sQ);
+      const int q_kb_stride = rows_pad * kKbBytes;
+      bool ok = true;
+      for (int it = 0; it < n_tiles && ok; ++it) {
+        const int s = it % n_stages;
+        if (!mbar_wait(full0 + 8 * s, (it / n_stages) & 1, kWhereP2Mma)) break;
+        const uint32_t a_base = smem_u32(sK + s * kP2TileBytes);
+        for (int u = 0; u < n_sub; ++u) {
+          if (!mbar_wait(tempty0 + 8 * u, (it & 1) ^ 1, kWhereP2Mma)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t d = tmem + u * 256;
+          const uint32_t b_rows = q_base + u * N0 * kKbBytes;
+          const uint32_t idesc = u == 0 ? idesc0 : idesc1;
+#pragma unroll
+          for (int kb = 0; kb < 2; ++kb) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t ad = smem_desc_k_sw128(a_base + kb * (kP2Keys * kKbBytes) + kk * 32);
+              const uint64_t bd = smem_desc_k_sw128(b_rows + kb * q_kb_stride + kk * 32);
+              umma_f16(d, ad, bd, idesc, (kb | kk) != 0);
+            }
+          }
+          umma_commit(tfull0 + 8 * u);
+        }
+        umma_commit(empty0 + 8 * s);
+      }
+      umma_commit(done);
+      mbar_wait(done, 0, kWhereP2Drain);
+    }
+  } else if (warp >= 4) {
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;  // key within the tile
+    float *yout = ypart + (static_cast<size_t>(gi) * g.n_heads() + head) * static_cast<size_t>(L);
+    bool ok = true;
+    for (int it = 0; it < n_tiles && ok; ++it) {
+      float y = -INFINITY;
+      for (int u = 0; u < n_sub; ++u) {
+        if (!mbar_wait(tfull0 + 8 * u, it & 1, kWhereP2Epi)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + u * 256;
+        const float *cu = ct + u * N0;
+        const int Nu = u == 0 ? N0 : N1;
+        int col = 0;
+#pragma unroll 1
+        for (; col + 32 <= Nu; col += 32) {
+          float v[32];
+          tmem_ld_32x32b_x32(taddr + col, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            const float4 c4 = *reinterpret_cast<const float4 *>(cu + col + i);
+            y = fmaxf(y, fmaxf(fmaxf(v[i] - c4.x, v[i + 1] - c4.y),
+                               fmaxf(v[i + 2] - c4.z, v[i + 3] - c4.w)));
+          }
+        }
+        if (col < Nu) {  // Nu is a multiple of 16
+          float v[16];
+          tmem_ld_32x32b_x16(taddr + col, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; i += 4) {
+            const float4 c4 = *reinterpret_cast<const float4 *>(cu + col + i);
+            y = fmaxf(y, fmaxf(fmaxf(v[i] - c4.x, v[i + 1] - c4.y),
+                               fmaxf(v[i + 2] - c4.z, v[i + 3] - c4.w)));
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tempty0 + 8 * u);
+      }
+      if (!ok) break;
+      const long long j = static_cast<long long>(t0 + it) * kP2Keys + row;
+      if (j < L) yout[j] = y * g.scale;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------ host
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// Tensor map of the whole key cache as a 2-D bf16 array
+// [n_layers * n_kv_heads * cap rows][128], boxes of 64 x box_rows, 128 B swizzle.
+bool make_key_map(CUtensorMap *map, const void *k, const ScoreGeom &g, int box_rows) {
+  auto encode = get_encode_fn();
+  if (!encode) return false;
+  const cuuint64_t rows = static_cast<cuuint64_t>(g.n_heads()) * static_cast<cuuint64_t>(g.cap);
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(kDim), rows};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(kRowBytes)};
+  cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(k), dims,
+                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bkv_status launch_score_rowstats_tc(const ScoreGeom &g, const void *k, const void *recent,
+                                    const void *beacons, float *c, cudaStream_t stream) {
+  CUtensorMap map;
+  if (!make_key_map(&map, k, g, kP1Keys)) return BKV_ERR_CUDA;
+  static int attr_done[64];
+  if (!ensure_smem_limit(score_rowstats_kernel, kP1SmemBytes, attr_done)) return BKV_ERR_CUDA;
+  dim3 grid(g.n_obs_pad / kP1Rows, g.n_heads());
+  score_rowstats_kernel<<<grid, kP1Threads, kP1SmemBytes, stream>>>(
+      map, g, static_cast<const uint16_t *>(recent), static_cast<const uint16_t *>(beacons), c);
+  return cudaGetLastError() == cudaSuccess ? BKV_OK : BKV_ERR_CUDA;
+}
+
+bkv_status launch_score_colmax_tc(const ScoreGeom &g, const void *k, const void *recent,
+                                  const void *beacons, const float *c, float *ypart,
+                                  cudaStream_t stream) {
+  CUtensorMap map;
+  if (!make_key_map(&map, k, g, kP2Keys)) return BKV_ERR_CUDA;
+  int max_rows_pad = 0;
+  for (int gi = 0; gi < g.n_groups; ++gi) {
+    const int nrows = std::min(g.rows_per_group, g.n_obs - gi * g.rows_per_group);
+    max_rows_pad = std::max(max_rows_pad, (nrows + 15) & ~15);
+  }
+  constexpr int kSmemLimit = 232448;  // 227 KB opt-in per block on sm_100
+  int stages = 4;
+  while (stages > 2 && p2_smem_bytes(max_rows_pad, stages) > kSmemLimit) --stages;
+  const int smem = p2_smem_bytes(max_rows_pad, stages);
+  if (smem > kSmemLimit) return BKV_ERR_UNSUPPORTED;
+  static int attr_done[64];
+  if (!ensure_smem_limit(score_colmax_kernel, kSmemLimit, attr_done)) return BKV_ERR_CUDA;
+  const int n_tiles = static_cast<int>((g.L + kP2Keys - 1) / kP2Keys);
+  // Split the keys of a head into chunks so that the grid covers the 148 SMs
+  // several times; each chunk reloads the observation rows once.
+  const long long units = static_cast<long long>(g.n_heads()) * g.n_groups;
+  int n_chunks = static_cast<int>(std::max(1LL, (4LL * 148 + units - 1) / units));
+  n_chunks = std::min(n_chunks, std::max(1, n_tiles / 8));
+  const int chunk_tiles = (n_tiles + n_chunks - 1) / n_chunks;
+  n_chunks = (n_tiles + chunk_tiles - 1) / chunk_tiles;
+  const long long grid = units * n_chunks;
+  score_colmax_kernel<<<static_cast<unsigned>(grid), kP2Threads, smem, stream>>>(
+      map, g, static_cast<const uint16_t *>(recent), static_cast<const uint16_t *>(beacons), c,
+      ypart, n_chunks, chunk_tiles, stages);
+  return cudaGetLastError() == cudaSuccess ? BKV_OK : BKV_ERR_CUDA;
+}
+
+}  // namespace bkv

@@ -1,0 +1,195 @@
+"""The C ABI on the host: the library loads, exports every declared entry point,
+and rejects bad arguments before anything is launched (no GPU needed).
+
+Every call below fails a host-side check, so no CUDA call is made; the pointers
+are fake addresses that are never dereferenced.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bkv.h")
+
+bkv = pytest.importorskip("kv_cache_compression_bkv_b200.bkv")
+LIB = bkv.LIB
+
+OK, INVALID, UNSUPPORTED, WORKSPACE = 0, 1, 2, 3
+A = 0x10000          # a 16-byte aligned fake device address
+S = 0                # default stream; never touched by rejected calls
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bkv_\w+)\s*\(", text)))
+
+
+def test_exports_every_declared_function():
+    names = declared_functions()
+    assert "bkv_compress_step" in names and len(names) >= 8
+    for name in names:
+        assert hasattr(LIB, name), name
+    assert set(bkv.EXPORTS) >= set(names) - set(), (set(names) - set(bkv.EXPORTS))
+
+
+def test_status_strings():
+    for code in range(7):
+        assert LIB.bkv_status_string(code)
+    assert LIB.bkv_status_string(99) == b"unknown status"
+
+
+def desc(Ly=2, Hq=8, Hkv=2, d=128, cap=1024, dt=bkv.BKV_BF16):
+    return bkv.CacheDesc(Ly, Hq, Hkv, d, cap, dt)
+
+
+def score(d, k=A, L=1000, recent=A, R=8, beacons=A, nb=16, M=16, scale=0.0, scores=A, ws=A,
+          ws_bytes=1 << 40):
+    return LIB.bkv_score(ctypes.byref(d) if d is not None else None, k, L, recent, R, beacons, nb,
+                         M, scale, scores, ws, ws_bytes, S)
+
+
+def test_workspace_size():
+    d = desc()
+    n = LIB.bkv_workspace_size(ctypes.byref(d), 1000, 8, 16, 64, 300)
+    # at least c, one aggregation partial and the kept indices of every head
+    assert n >= 2 * 2 * (1000 * 4 + 300 * 4)
+    assert LIB.bkv_workspace_size(ctypes.byref(d), 0, 8, 16, 64, 300) == 0
+    assert LIB.bkv_workspace_size(ctypes.byref(desc(Hq=7)), 1000, 8, 16, 64, 300) == 0
+    assert LIB.bkv_workspace_size(None, 1000, 8, 16, 64, 300) == 0
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(d=None), INVALID),
+    (dict(d=desc(Hq=7)), INVALID),            # q heads not a multiple of kv heads
+    (dict(d=desc(cap=0)), INVALID),
+    (dict(d=desc(d=60)), INVALID),            # row not a multiple of 16 bytes
+    (dict(d=desc(dt=5)), INVALID),
+    (dict(L=0), INVALID),
+    (dict(L=1025), INVALID),                  # beyond capacity
+    (dict(nb=17), INVALID),                   # more beacons than slots
+    (dict(R=0, nb=0), INVALID),               # empty observation set
+    (dict(k=0), INVALID),
+    (dict(k=A + 8), INVALID),                 # misaligned
+    (dict(recent=0), INVALID),
+    (dict(beacons=0), INVALID),
+    (dict(scores=0), INVALID),
+    (dict(scale=-1.0), INVALID),
+    (dict(scale=float("nan")), INVALID),
+    (dict(d=desc(d=64)), UNSUPPORTED),        # bf16 tensor-core path is head_dim 128
+    (dict(d=desc(d=256, dt=bkv.BKV_F32)), UNSUPPORTED),
+    (dict(ws=0), WORKSPACE),
+    (dict(ws_bytes=1024), WORKSPACE),
+])
+def test_score_rejects(kw, expect):
+    args = dict(d=desc())
+    args.update(kw)
+    assert score(**args) == expect
+
+
+def test_select_rejects():
+    f = LIB.bkv_select_topk
+    assert f(None, 4, 100, 10, A, None, 0, S) == INVALID
+    assert f(A, 0, 100, 10, A, None, 0, S) == INVALID
+    assert f(A, 4, 0, 10, A, None, 0, S) == INVALID
+    assert f(A, 4, 100, 0, A, None, 0, S) == INVALID
+    assert f(A, 4, 100, 10, None, None, 0, S) == INVALID
+    assert f(A + 4, 4, 100, 10, A, None, 0, S) == INVALID
+    # a row too long for shared memory needs workspace
+    assert f(A, 4, 1 << 20, 10, A, None, 0, S) == WORKSPACE
+
+
+def test_compact_rejects():
+    f = LIB.bkv_compact
+    src, dst = desc(cap=1024), desc(cap=256)
+    big = 1 << 30
+    ok_args = [ctypes.byref(src), A, A + big, A + 2 * big, 256, ctypes.byref(dst), A + 3 * big,
+               A + 4 * big, S]
+
+    def call(**kw):
+        a = list(ok_args)
+        names = ["src", "k_src", "v_src", "idx", "n", "dst", "k_dst", "v_dst", "s"]
+        for key, val in kw.items():
+            a[names.index(key)] = val
+        return f(*a)
+
+    assert call(n=257) == INVALID                       # beyond dst capacity
+    assert call(n=-1) == INVALID
+    assert call(idx=0) == INVALID
+    assert call(k_dst=0) == INVALID                     # pair half missing
+    assert call(k_dst=A + 64) == INVALID                # overlaps k_src
+    assert call(v_dst=A + big + 1024) == INVALID        # overlaps v_src
+    assert call(k_dst=A + 3 * big + 8) == INVALID       # misaligned
+    assert call(dst=ctypes.byref(desc(cap=256, d=64))) == INVALID
+    assert call(dst=ctypes.byref(desc(cap=256, dt=bkv.BKV_F32))) == INVALID
+
+
+def test_update_beacons_rejects():
+    f = LIB.bkv_update_beacons
+    d = desc()
+    n = ctypes.c_int32(-7)
+    big = 1 << 30
+    base = [ctypes.byref(d), A, 16, 16, A + big, 64, A + 2 * big, ctypes.byref(n), None, 0, S]
+
+    def call(**kw):
+        a = list(base)
+        names = ["d", "bin", "nb", "M", "win", "W", "bout", "nout", "ws", "wsb", "s"]
+        for key, val in kw.items():
+            a[names.index(key)] = val
+        return f(*a)
+
+    assert call(M=0) == INVALID
+    assert call(nb=17) == INVALID
+    assert call(nb=0, W=0) == INVALID
+    assert call(win=0) == INVALID
+    assert call(bout=0) == INVALID
+    assert call(bout=A + 64) == INVALID                 # overlaps beacons_in
+    assert call(bout=A + big + 128) == INVALID          # overlaps window
+    assert call(W=100000) == UNSUPPORTED                # distances do not fit shared memory
+    assert n.value == -7                                # outputs untouched
+
+
+def step_args(**kw):
+    a = bkv.StepArgs()
+    big = 1 << 32
+    a.cache = desc(cap=1024)
+    a.k, a.v, a.L, a.K = A, A + big, 1000, 300
+    a.recent_q, a.R = A + 2 * big, 8
+    a.beacons_in, a.n_beacons_in, a.M = A + 3 * big, 16, 16
+    a.window, a.W, a.beacons_out = A + 4 * big, 64, A + 5 * big
+    a.scale = 0.0
+    a.dst_cache = desc(cap=512)
+    a.k_dst, a.v_dst = A + 6 * big, A + 7 * big
+    a.scores_out, a.idx_out = None, None
+    a.workspace, a.workspace_bytes = A + 8 * big, 1 << 31
+    a.stream = None
+    for key, val in kw.items():
+        setattr(a, key, val)
+    return a
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(K=0), INVALID),
+    (dict(dst_cache=desc(cap=299)), INVALID),      # too small for the kept rows
+    (dict(dst_cache=desc(cap=512, d=64)), INVALID),
+    (dict(v=None), INVALID),
+    (dict(k_dst=None), INVALID),
+    (dict(beacons_out=None), INVALID),             # needed when a window is given
+    (dict(k_dst=(1 << 32) + A + 64), INVALID),     # overlaps v
+    (dict(beacons_out=A + 3 * (1 << 32)), INVALID),  # overlaps beacons_in
+    (dict(idx_out=A + 2), INVALID),                # misaligned
+    (dict(workspace_bytes=4096), WORKSPACE),
+    (dict(workspace=None), WORKSPACE),
+    (dict(W=100000), UNSUPPORTED),
+])
+def test_compress_step_rejects(kw, expect):
+    a = step_args(**kw)
+    nb, nl = ctypes.c_int32(-5), ctypes.c_int64(-5)
+    assert LIB.bkv_compress_step(ctypes.byref(a), ctypes.byref(nb), ctypes.byref(nl)) == expect
+    assert nb.value == -5 and nl.value == -5
+
+
+def test_compress_step_null():
+    assert LIB.bkv_compress_step(None, None, None) == INVALID

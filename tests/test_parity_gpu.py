@@ -1,0 +1,228 @@
+"""CUDA path against the float64 oracle, element by element, through the C ABI.
+
+Small cases cover every head of several tiles with ragged tails and the
+degenerate shapes; the full-size workloads run the same launch configuration
+as bench.py and compare seeded samples of heads.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity_helpers import (check_compaction, check_fps, check_scores, check_topk, f64,
+                            picks_from_rows, raw)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dev():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    return torch.device("cuda:0")
+
+
+def _lib():
+    from kv_cache_compression_bkv_b200 import bkv
+    return bkv
+
+
+def _synth():
+    from kv_cache_compression_bkv_b200 import synth
+    return synth
+
+
+def small(**kw):
+    base = dict(name="case", n_layers=1, n_q_heads=4, n_kv_heads=2, head_dim=128, L=1000,
+                R=8, M=16, K=300, W=0, dtype="bf16", n_clusters=4, q_noise=0.5, n_plan=16,
+                plan_span=64, n_outlier_channels=2, n_beacons_in=12)
+    base.update(kw)
+    base.setdefault("capacity", base["L"] + 100)  # poisoned rows past L
+    return _synth().Workload(**base)
+
+
+SCORE_CASES = {
+    "tiny_f32": lambda: _synth().WORKLOADS["tiny"].replace(W=0),
+    "ragged_bf16": lambda: small(n_layers=2),
+    "row_blocks": lambda: small(n_q_heads=16, R=24, M=20, n_beacons_in=20, L=777, K=100),
+    "two_groups": lambda: small(n_q_heads=16, R=40, M=40, n_beacons_in=40, L=513, K=64),
+    "one_key": lambda: small(L=1, K=1, capacity=16),
+    "short": lambda: small(L=129, K=5),
+    "recent_only": lambda: small(n_beacons_in=0, L=300),
+    "beacons_only": lambda: small(R=0, L=300),
+    "exact_tiles": lambda: small(n_q_heads=8, n_kv_heads=1, R=32, M=32, n_beacons_in=32,
+                                 L=4096, K=1024, capacity=4096),
+    "big_norms": lambda: small(big_key_frac=0.05, big_key_norm=40.0, L=2000, K=500),
+}
+
+
+@pytest.mark.parametrize("case", sorted(SCORE_CASES))
+def test_score_select_compact(case, dev):
+    bkv, synth = _lib(), _synth()
+    wl = SCORE_CASES[case]()
+    inp = synth.make_step_inputs(wl, seed=11)
+    g = bkv.geometry_of(inp.k, wl.n_q_heads)
+    k, v = inp.k.to(dev), inp.v.to(dev)
+    rq, bq = inp.recent.to(dev), inp.beacons.to(dev)
+    H = wl.n_heads
+    scores = torch.full((wl.n_layers, wl.n_kv_heads, wl.L), -1.0, device=dev)
+    ws = torch.empty(bkv.bkv_workspace_size(g, wl.L, wl.R, wl.M, 0, wl.K), dtype=torch.uint8,
+                     device=dev)
+    bkv.bkv_score(g, k, wl.L, rq if wl.R else None, wl.R, bq if wl.beacons_in else None,
+                  wl.beacons_in, wl.M, 0.0, scores, ws)
+    keep = min(wl.K, wl.L)
+    idx = torch.full((H, keep), -1, dtype=torch.int32, device=dev)
+    bkv.bkv_select_topk(scores, H, wl.L, wl.K, idx, ws)
+    dst = bkv.Geometry(g.n_layers, g.n_q_heads, g.n_kv_heads, g.head_dim, keep, g.dtype)
+    kd = torch.empty(wl.n_layers, wl.n_kv_heads, keep, wl.head_dim, dtype=inp.k.dtype, device=dev)
+    vd = torch.empty_like(kd)
+    bkv.bkv_compact(g, k, v, idx, keep, dst, kd, vd)
+    torch.cuda.synchronize()
+    assert bkv.bkv_read_device_status()[0] == 0
+    s_all = scores.double().cpu().numpy()
+    idx_all = idx.cpu().numpy()
+    kd_raw, vd_raw = raw(kd), raw(vd)
+    k_raw, v_raw = raw(inp.k), raw(inp.v)
+    for l in range(wl.n_layers):
+        for h in range(wl.n_kv_heads):
+            kk, vv, rr, bb, _ = synth.head_slice(inp, l, h)
+            s_ref, _ = oracle.score_head(f64(kk), f64(rr), f64(bb), wl.beacons_in)
+            check_scores(s_all[l, h], s_ref, f"{case} scores l{l} h{h}")
+            r = l * wl.n_kv_heads + h
+            check_topk(idx_all[r], s_ref, wl.K, f"{case} top-K l{l} h{h}")
+            check_compaction(kd_raw[l, h], k_raw[l, h], idx_all[r], f"{case} K rows")
+            check_compaction(vd_raw[l, h], v_raw[l, h], idx_all[r], f"{case} V rows")
+
+
+FPS_CASES = {
+    "tiny_f32": lambda: _synth().WORKLOADS["tiny"],
+    "bf16_small": lambda: small(W=300, M=24, n_beacons_in=10),
+    "no_beacons": lambda: small(W=40, M=16, n_beacons_in=0),
+    "window_lt_M": lambda: small(W=5, M=16, n_beacons_in=4),
+    "window_only_one": lambda: small(W=1, M=4, n_beacons_in=0, R=1),
+}
+
+
+@pytest.mark.parametrize("case", sorted(FPS_CASES))
+def test_update_beacons(case, dev):
+    bkv, synth = _lib(), _synth()
+    wl = FPS_CASES[case]()
+    inp = synth.make_step_inputs(wl, seed=5)
+    g = bkv.geometry_of(inp.k, wl.n_q_heads)
+    bin_, win = inp.beacons.to(dev), inp.window.to(dev)
+    bout = torch.zeros_like(bin_)
+    n = bkv.bkv_update_beacons(g, bin_ if wl.beacons_in else None, wl.beacons_in, wl.M, win,
+                               wl.W, bout)
+    torch.cuda.synchronize()
+    assert n == min(wl.M, wl.beacons_in + wl.W)
+    out_raw = raw(bout)
+    for l in range(wl.n_layers):
+        for qh in range(wl.n_q_heads):
+            U = torch.cat([inp.beacons[l, qh, :wl.beacons_in], inp.window[l, qh]])
+            picks = picks_from_rows(raw(U), out_raw[l, qh, :n])
+            check_fps(f64(U), picks, wl.M, f"{case} l{l} q{qh}")
+
+
+def _run_step(wl, inp, dev, scores=True):
+    bkv = _lib()
+    g = bkv.geometry_of(inp.k, wl.n_q_heads)
+    keep = min(wl.K, wl.L)
+    dst = bkv.Geometry(g.n_layers, g.n_q_heads, g.n_kv_heads, g.head_dim, keep, g.dtype)
+    t = {n: getattr(inp, n).to(dev) for n in ("k", "v", "recent", "beacons", "window")}
+    out = dict(
+        bout=torch.zeros_like(t["beacons"]),
+        kd=torch.empty(wl.n_layers, wl.n_kv_heads, keep, wl.head_dim, dtype=inp.k.dtype,
+                       device=dev),
+        scores=torch.empty(wl.n_layers, wl.n_kv_heads, wl.L, device=dev) if scores else None,
+        idx=torch.empty(wl.n_layers, wl.n_kv_heads, keep, dtype=torch.int32, device=dev),
+    )
+    out["vd"] = torch.empty_like(out["kd"])
+    ws = torch.empty(bkv.bkv_workspace_size(g, wl.L, wl.R, wl.M, wl.W, wl.K), dtype=torch.uint8,
+                     device=dev)
+    nb, nl = bkv.bkv_compress_step(
+        g, t["k"], t["v"], wl.L, wl.K, t["recent"] if wl.R else None, wl.R,
+        t["beacons"] if wl.beacons_in else None, wl.beacons_in, wl.M,
+        t["window"] if wl.W else None, wl.W, out["bout"], 0.0, dst, out["kd"], out["vd"],
+        out["scores"], out["idx"], ws)
+    torch.cuda.synchronize()
+    assert bkv.bkv_read_device_status()[0] == 0
+    assert nl == keep
+    assert nb == (min(wl.M, wl.beacons_in + wl.W) if wl.W else wl.beacons_in)
+    return out, nb
+
+
+def _check_step_heads(wl, inp, out, nb, heads, what):
+    """Oracle comparison of whole-step outputs for the sampled (layer, KV head)s."""
+    synth = _synth()
+    G = wl.group
+    out_b = raw(out["bout"])
+    s_all = out["scores"].double().cpu().numpy() if out["scores"] is not None else None
+    idx_all = out["idx"].cpu().numpy()
+    kd_raw, vd_raw = raw(out["kd"]), raw(out["vd"])
+    k_raw, v_raw = raw(inp.k), raw(inp.v)
+    n_exact = 0
+    for (l, h) in heads:
+        kk, vv, rr, bb, ww = synth.head_slice(inp, l, h)
+        exact = True
+        if wl.W:
+            for gq in range(G):
+                U = torch.cat([bb[gq, :wl.beacons_in], ww[gq]])
+                picks = picks_from_rows(raw(U), out_b[l, h * G + gq, :nb])
+                exact &= check_fps(f64(U), picks, wl.M, f"{what} FPS l{l} q{h * G + gq}")
+        check_compaction(kd_raw[l, h], k_raw[l, h], idx_all[l, h], f"{what} K rows l{l} h{h}")
+        check_compaction(vd_raw[l, h], v_raw[l, h], idx_all[l, h], f"{what} V rows l{l} h{h}")
+        if not exact:
+            continue  # near-tie in FPS: the oracle scores different beacons
+        n_exact += 1
+        ref = oracle.compress_head(f64(kk), f64(vv), f64(rr), f64(bb), wl.beacons_in,
+                                   f64(ww) if wl.W else None, wl.M, wl.K)
+        if s_all is not None:
+            check_scores(s_all[l, h], ref["scores"], f"{what} scores l{l} h{h}")
+        check_topk(idx_all[l, h], ref["scores"], wl.K, f"{what} top-K l{l} h{h}")
+    return n_exact
+
+
+STEP_CASES = {
+    "tiny_f32": lambda: _synth().WORKLOADS["tiny"],
+    "bf16_fps": lambda: small(n_layers=2, W=200, M=16, n_beacons_in=8, L=1500, K=400,
+                              capacity=1600),
+    "keep_all": lambda: small(L=200, K=512, W=20, capacity=256),
+    "no_window": lambda: small(W=0),
+}
+
+
+@pytest.mark.parametrize("case", sorted(STEP_CASES))
+def test_compress_step_small(case, dev):
+    wl = STEP_CASES[case]()
+    inp = _synth().make_step_inputs(wl, seed=3)
+    out, nb = _run_step(wl, inp, dev)
+    heads = [(l, h) for l in range(wl.n_layers) for h in range(wl.n_kv_heads)]
+    n_exact = _check_step_heads(wl, inp, out, nb, heads, case)
+    assert n_exact == len(heads), "FPS near-ties on a small case"
+
+
+FULL = ["r1_qwen7b", "llama8b", "qwen3_4b_step", "qwen3_14b"]
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_sampled(name, dev):
+    """The benchmark's launch configuration at full size; sampled heads vs the oracle."""
+    synth = _synth()
+    wl = synth.WORKLOADS[name]
+    inp = synth.make_step_inputs(wl, seed=0)
+    out, nb = _run_step(wl, inp, dev)
+    rng = np.random.default_rng(123)
+    heads = sorted({(int(rng.integers(wl.n_layers)), int(rng.integers(wl.n_kv_heads)))
+                    for _ in range(3)} | {(wl.n_layers - 1, wl.n_kv_heads - 1)})
+    n_exact = _check_step_heads(wl, inp, out, nb, heads, name)
+    assert n_exact >= 1, "every sampled head hit an FPS near-tie"
+    # compaction of every head: each kept row is a byte copy of its source row
+    idx = out["idx"].long()
+    k_dev = inp.k.to(dev)
+    gathered = torch.gather(k_dev, 2, idx[..., None].expand(-1, -1, -1, wl.head_dim))
+    assert torch.equal(gathered.view(torch.int16), out["kd"].view(torch.int16))
+    # kept positions are strictly ascending in every head
+    assert bool((idx[..., 1:] > idx[..., :-1]).all())
