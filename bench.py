@@ -309,6 +309,11 @@ def main():
 
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(bkv.STEP_EVENTS)]
           for _ in range(args.steps)]
+    # torch creates an event lazily and refuses elapsed_time() on events it did
+    # not record itself: record each once here; the library re-records them
+    for row in ev:
+        for e in row:
+            e.record(stream)
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local)
