@@ -25,6 +25,7 @@ import argparse
 import json
 import math
 import os
+import shutil
 import statistics
 import subprocess
 import sys
@@ -110,32 +111,38 @@ class ClockSampler:
     def __init__(self, device_index: int):
         self.proc = None
         self.path = None
+        self.err = None
         try:
             bus = torch.cuda.get_device_properties(device_index).pci_bus_id
         except Exception:
             bus = None
-        self.sel = ["-i", bus] if bus else []
+        self.sel = ["-i", str(bus)] if bus else []
 
     def start(self):
         fd, self.path = tempfile.mkstemp(prefix="bkv_clocks_", suffix=".csv")
         os.close(fd)
+        exe = shutil.which("nvidia-smi") or "/usr/bin/nvidia-smi"
         try:
+            self.out = open(self.path, "w")
             self.proc = subprocess.Popen(
-                ["nvidia-smi", *self.sel, f"--query-gpu={self.FIELDS}",
+                [exe, *self.sel, f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-        except Exception:
+                stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception as e:  # noqa: BLE001
             self.proc = None
+            self.err = type(e).__name__ + ": " + str(e)
 
     def stop(self):
         if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+            return {"sm_mhz": None, "sm_max_mhz": None,
+                    "reasons": ["nvidia-smi unavailable (%s)" % self.err]}
         time.sleep(0.15)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
+        self.out.close()
         rows = []
         with open(self.path) as f:
             for line in f:

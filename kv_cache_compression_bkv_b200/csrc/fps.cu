@@ -5,15 +5,28 @@
 // is sampled greedily: seed U[0]; each further pick is the unselected point
 // with the largest distance to the selected set (ties to the lowest index);
 // dist(a, b) = 1 - (u_a . u_b) / (|u_a| |u_b|), clamped to [0, 2], and 1 when a
-// norm is zero.  One CTA per query head keeps the running distances and the
-// inverse norms in shared memory; each pick rereads the points (L2-resident)
-// to take their dot products with the newly picked point in f32.  bf16 inputs
-// make every product exact in f32.
+// norm is zero.
+//
+// The greedy picks are found in exact speculative rounds, so that the points
+// are streamed once per round rather than once per pick:
+//   1. the T+1 best unselected points by (distance desc, index asc) are found
+//      by a radix select over the shared-memory distance array; the first T
+//      are the candidates, the last bounds every other point (distances only
+//      ever decrease);
+//   2. the candidates' Gram block is formed (same arithmetic as step 4);
+//   3. one warp replays the greedy choice among the candidates alone: the best
+//      remaining candidate is the true argmax while it beats that bound, so it
+//      is picked and the other candidates' distances are lowered with the Gram
+//      block; the round stops at the first candidate that does not;
+//   4. one pass over the points lowers every distance by the round's picks
+//      (packed FFMA2 dot products, the point loaded and converted once per
+//      round and reused for every pick).
+// The result is exactly the greedy sequence (no approximation); bf16 products
+// are exact in f32, the sums are f32.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
-#include <mutex>
 
 #include "bkv_internal.h"
 
@@ -22,66 +35,199 @@ namespace {
 
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
-constexpr int kSmemLimit = 232448;
+constexpr int kCand = 32;        // candidates per round (T)
 constexpr int kMaxDim = 128;
+constexpr int kSmemLimit = 232448;
+
+// ---- element access: 8 consecutive elements as f32
+__device__ __forceinline__ void load8(const __nv_bfloat16 *p, float (&u)[8]) {
+  const uint4 w = *reinterpret_cast<const uint4 *>(p);
+  u[0] = __uint_as_float(w.x << 16); u[1] = __uint_as_float(w.x & 0xffff0000u);
+  u[2] = __uint_as_float(w.y << 16); u[3] = __uint_as_float(w.y & 0xffff0000u);
+  u[4] = __uint_as_float(w.z << 16); u[5] = __uint_as_float(w.z & 0xffff0000u);
+  u[6] = __uint_as_float(w.w << 16); u[7] = __uint_as_float(w.w & 0xffff0000u);
+}
+__device__ __forceinline__ void load8(const float *p, float (&u)[8]) {
+  const float4 a = *reinterpret_cast<const float4 *>(p);
+  const float4 b = *reinterpret_cast<const float4 *>(p + 4);
+  u[0] = a.x; u[1] = a.y; u[2] = a.z; u[3] = a.w;
+  u[4] = b.x; u[5] = b.y; u[6] = b.z; u[7] = b.w;
+}
+
+// One 8-element step of a dot product, the same operation sequence wherever a
+// dot product is formed (point pass and Gram block), so both agree bit for bit.
+__device__ __forceinline__ float2 dot8_step(float2 acc, const float (&u)[8], const float *s) {
+  const float4 s0 = *reinterpret_cast<const float4 *>(s);
+  const float4 s1 = *reinterpret_cast<const float4 *>(s + 4);
+  acc = __ffma2_rn(make_float2(u[0], u[1]), make_float2(s0.x, s0.y), acc);
+  acc = __ffma2_rn(make_float2(u[2], u[3]), make_float2(s0.z, s0.w), acc);
+  acc = __ffma2_rn(make_float2(u[4], u[5]), make_float2(s1.x, s1.y), acc);
+  acc = __ffma2_rn(make_float2(u[6], u[7]), make_float2(s1.z, s1.w), acc);
+  return acc;
+}
+
+__device__ __forceinline__ float cos_dist(float2 acc, float inv_a, float inv_b) {
+  const float dot = __fadd_rn(acc.x, acc.y);
+  const float dd = __fmaf_rn(-__fmul_rn(dot, inv_a), inv_b, 1.0f);
+  return fminf(fmaxf(dd, 0.f), 2.f);
+}
+
+// Order key of a distance: larger distance -> larger key; selected points
+// (distance -1) -> 0, below every unselected point.
+__device__ __forceinline__ uint32_t dist_key(float d) {
+  return d < 0.f ? 0u : (__float_as_uint(d) | 0x80000000u);
+}
+
+// (distance desc, index asc): true if (da, ia) comes before (db, ib).
+__device__ __forceinline__ bool before(float da, int ia, float db, int ib) {
+  return da > db || (da == db && ia < ib);
+}
+
+struct Smem {
+  float *dist;       // [n]
+  float *inv;        // [n]
+  float *cvec;       // [kCand][d] candidate vectors (f32)
+  float *pvec;       // [kCand][d] this round's picks (f32)
+  float *gram;       // [kCand][kCand]
+  uint32_t *hist;    // [256]
+  int *cidx;         // [kCand + 1] candidates, then the bound
+  float *cdist;      // [kCand + 1]
+  int *pick;         // [kCand] candidate slots picked this round
+  float *pinv;       // [kCand]
+  int *scal;         // [8]
+};
 
 template <typename T>
-struct Vec;
-
-template <>
-struct Vec<float> {
-  // 4 elements per 16-byte load
-  static constexpr int kPer = 4;
-  __device__ static float dot16(const float *p, const float *s) {
-    const float4 x = *reinterpret_cast<const float4 *>(p);
-    const float4 y = *reinterpret_cast<const float4 *>(s);
-    return fmaf(x.x, y.x, fmaf(x.y, y.y, fmaf(x.z, y.z, x.w * y.w)));
+struct Points {
+  const T *B, *Wp;
+  int nb, d;
+  __device__ const T *operator()(int i) const {
+    return i < nb ? B + static_cast<size_t>(i) * d : Wp + static_cast<size_t>(i - nb) * d;
   }
-  __device__ static float sq16(const float *p) {
-    const float4 x = *reinterpret_cast<const float4 *>(p);
-    return fmaf(x.x, x.x, fmaf(x.y, x.y, fmaf(x.z, x.z, x.w * x.w)));
-  }
-  __device__ static float to_f(float v) { return v; }
 };
 
-__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
-
-template <>
-struct Vec<__nv_bfloat16> {
-  static constexpr int kPer = 8;
-  __device__ static float dot16(const __nv_bfloat16 *p, const float *s) {
-    const uint4 x = *reinterpret_cast<const uint4 *>(p);
-    const float4 s0 = *reinterpret_cast<const float4 *>(s);
-    const float4 s1 = *reinterpret_cast<const float4 *>(s + 4);
-    float a = bf_lo(x.x) * s0.x;
-    a = fmaf(bf_hi(x.x), s0.y, a);
-    a = fmaf(bf_lo(x.y), s0.z, a);
-    a = fmaf(bf_hi(x.y), s0.w, a);
-    a = fmaf(bf_lo(x.z), s1.x, a);
-    a = fmaf(bf_hi(x.z), s1.y, a);
-    a = fmaf(bf_lo(x.w), s1.z, a);
-    a = fmaf(bf_hi(x.w), s1.w, a);
-    return a;
+// Lower every unselected point's distance by the picks pvec[0..np) (or set it,
+// for the seed).  NP >= np accumulators are carried; the extra ones are not used.
+template <int NP, typename T>
+__device__ void point_pass(const Smem &s, const Points<T> &pt, int n, int d, int np,
+                           bool first) {
+  for (int i = threadIdx.x; i < n; i += kThreads) {
+    float di = s.dist[i];
+    if (!first && di < 0.f) continue;
+    const T *p = pt(i);
+    float2 acc[NP];
+#pragma unroll
+    for (int k = 0; k < NP; ++k) acc[k] = make_float2(0.f, 0.f);
+    for (int t = 0; t < d; t += 8) {
+      float u[8];
+      load8(p + t, u);
+#pragma unroll
+      for (int k = 0; k < NP; ++k) acc[k] = dot8_step(acc[k], u, s.pvec + k * kMaxDim + t);
+    }
+    const float inv_i = s.inv[i];
+#pragma unroll
+    for (int k = 0; k < NP; ++k) {
+      if (k < np) {
+        const float dd = cos_dist(acc[k], inv_i, s.pinv[k]);
+        di = (first && k == 0) ? dd : fminf(di, dd);
+      }
+    }
+    s.dist[i] = di;
   }
-  __device__ static float sq16(const __nv_bfloat16 *p) {
-    const uint4 x = *reinterpret_cast<const uint4 *>(p);
-    float a = bf_lo(x.x) * bf_lo(x.x);
-    a = fmaf(bf_hi(x.x), bf_hi(x.x), a);
-    a = fmaf(bf_lo(x.y), bf_lo(x.y), a);
-    a = fmaf(bf_hi(x.y), bf_hi(x.y), a);
-    a = fmaf(bf_lo(x.z), bf_lo(x.z), a);
-    a = fmaf(bf_hi(x.z), bf_hi(x.z), a);
-    a = fmaf(bf_lo(x.w), bf_lo(x.w), a);
-    a = fmaf(bf_hi(x.w), bf_hi(x.w), a);
-    return a;
-  }
-  __device__ static float to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
-};
+}
 
-// (distance, index) order of the argmax: larger distance wins, then lower index.
-__device__ __forceinline__ bool better(float d1, int i1, float d2, int i2) {
-  return d1 > d2 || (d1 == d2 && i1 < i2);
+template <typename T>
+__device__ void point_pass_dispatch(const Smem &s, const Points<T> &pt, int n, int d, int np,
+                                    bool first) {
+  switch ((np + 3) >> 2) {
+    case 1: point_pass<4>(s, pt, n, d, np, first); break;
+    case 2: point_pass<8>(s, pt, n, d, np, first); break;
+    case 3: point_pass<12>(s, pt, n, d, np, first); break;
+    case 4: point_pass<16>(s, pt, n, d, np, first); break;
+    case 5: point_pass<20>(s, pt, n, d, np, first); break;
+    case 6: point_pass<24>(s, pt, n, d, np, first); break;
+    case 7: point_pass<28>(s, pt, n, d, np, first); break;
+    default: point_pass<32>(s, pt, n, d, np, first); break;
+  }
+}
+
+// The `want` best unselected points in (distance desc, index asc) order, into
+// s.cidx / s.cdist (unordered).  Requires `want` <= number of unselected.
+__device__ void select_best(const Smem &s, int n, int want) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  uint32_t prefix = 0, mask = 0;
+  int krem = want;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int b = tid; b < 256; b += kThreads) s.hist[b] = 0;
+    __syncthreads();
+    for (int i = tid; i < n; i += kThreads) {
+      const uint32_t key = dist_key(s.dist[i]);
+      if (key != 0u && (key & mask) == prefix) atomicAdd(&s.hist[(key >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    if (warp == 0) {
+      uint32_t cnt[8], local = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        cnt[j] = s.hist[255 - 8 * lane - j];
+        local += cnt[j];
+      }
+      uint32_t incl = local;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+      }
+      const uint32_t excl = incl - local;
+      if (static_cast<int>(excl) < krem && krem <= static_cast<int>(incl)) {
+        uint32_t acc = excl;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (static_cast<int>(acc + cnt[j]) >= krem) {
+            s.scal[0] = 255 - 8 * lane - j;
+            s.scal[1] = static_cast<int>(acc);
+            break;
+          }
+          acc += cnt[j];
+        }
+      }
+    }
+    __syncthreads();
+    prefix |= static_cast<uint32_t>(s.scal[0]) << shift;
+    mask |= 255u << shift;
+    krem -= s.scal[1];
+    __syncthreads();
+  }
+  // emit: every key above the threshold, and the lowest-index krem keys equal
+  // to it (an ordered scan only over the equal keys)
+  if (tid == 0) { s.scal[2] = 0; s.scal[3] = 0; }
+  __syncthreads();
+  int eq_base = 0;
+  for (int base = 0; base < n; base += kThreads) {
+    const int i = base + tid;
+    const uint32_t key = i < n ? dist_key(s.dist[i]) : 0u;
+    const bool gt = key > prefix;
+    const bool eq = key == prefix && key != 0u;
+    const uint32_t eb = __ballot_sync(0xffffffffu, eq);
+    if (lane == 0) s.hist[warp] = __popc(eb);
+    __syncthreads();
+    int before_me = 0, total = 0;
+    for (int w = 0; w < kWarps; ++w) {
+      const int c = static_cast<int>(s.hist[w]);
+      if (w < warp) before_me += c;
+      total += c;
+    }
+    before_me += __popc(eb & ((1u << lane) - 1u));
+    if (gt || (eq && eq_base + before_me < krem)) {
+      const int pos = atomicAdd(&s.scal[2], 1);
+      if (pos < want) {
+        s.cidx[pos] = i;
+        s.cdist[pos] = s.dist[i];
+      }
+    }
+    eq_base += total;
+    __syncthreads();
+  }
 }
 
 template <typename T>
@@ -91,98 +237,163 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ __align__(16) float sm[];
   const int d = g.head_dim;
   const int n = g.nb_in + g.W;
-  float *sv = sm;                 // [kMaxDim] picked point, f32
-  float *inv = sv + kMaxDim;      // [n] inverse norms (0 for a zero vector)
-  float *dist = inv + n;          // [n] distance to the selected set; -1 = selected
-  __shared__ float red_d[kWarps];
-  __shared__ int red_i[kWarps];
-  __shared__ int pick_sh;
+  const int m = g.n_pick;
+  Smem s;
+  s.cvec = sm;
+  s.pvec = s.cvec + kCand * kMaxDim;
+  s.gram = s.pvec + kCand * kMaxDim;
+  s.pinv = s.gram + kCand * kCand;
+  s.cdist = s.pinv + kCand;
+  s.dist = s.cdist + (kCand + 4);
+  s.inv = s.dist + n;
+  s.hist = reinterpret_cast<uint32_t *>(s.inv + n);
+  s.cidx = reinterpret_cast<int *>(s.hist + 256);
+  s.pick = s.cidx + (kCand + 4);
+  s.scal = s.pick + kCand;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const size_t qh = blockIdx.x;  // layer * n_q_heads + query head
-  const T *B = beacons_in + qh * static_cast<size_t>(g.M) * d;
-  const T *Wp = window + qh * static_cast<size_t>(g.W) * d;
+  Points<T> pt{beacons_in + qh * static_cast<size_t>(g.M) * d,
+               window + qh * static_cast<size_t>(g.W) * d, g.nb_in, d};
   T *out = beacons_out + qh * static_cast<size_t>(g.M) * d;
-  auto point = [&](int i) -> const T * {
-    return i < g.nb_in ? B + static_cast<size_t>(i) * d : Wp + static_cast<size_t>(i - g.nb_in) * d;
-  };
 
+  // inverse norms (0 for a zero vector, which makes its distance 1)
   for (int i = tid; i < n; i += kThreads) {
-    const T *p = point(i);
+    const T *p = pt(i);
     float ss = 0.f;
-    for (int t = 0; t < d; t += Vec<T>::kPer) ss += Vec<T>::sq16(p + t);
-    inv[i] = ss > 0.f ? 1.0f / sqrtf(ss) : 0.f;
+    for (int t = 0; t < d; t += 8) {
+      float u[8];
+      load8(p + t, u);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) ss = fmaf(u[j], u[j], ss);
+    }
+    s.inv[i] = ss > 0.f ? 1.0f / sqrtf(ss) : 0.f;
   }
-  int pick = 0;
-  for (int step = 0; step < g.n_pick; ++step) {
-    const T *pp = point(pick);
-    for (int t = tid; t < d; t += kThreads) {
-      out[static_cast<size_t>(step) * d + t] = pp[t];
-      sv[t] = Vec<T>::to_f(pp[t]);
-    }
-    __syncthreads();  // sv and (first step) inv are ready
-    if (step + 1 == g.n_pick) break;
-    const float inv_s = inv[pick];
-    float best_d = -2.f;
-    int best_i = n;
-    for (int i = tid; i < n; i += kThreads) {
-      float di;
-      if (i == pick || (step > 0 && dist[i] < 0.f)) {
-        di = -1.f;
-      } else {
-        const T *p = point(i);
-        float dot = 0.f;
-        for (int t = 0; t < d; t += Vec<T>::kPer) dot += Vec<T>::dot16(p + t, sv + t);
-        float dd = 1.0f - dot * inv[i] * inv_s;
-        dd = fminf(fmaxf(dd, 0.f), 2.f);
-        di = step > 0 ? fminf(dist[i], dd) : dd;
-      }
-      dist[i] = di;
-      if (better(di, i, best_d, best_i)) {
-        best_d = di;
-        best_i = i;
-      }
-    }
-    for (int off = 16; off > 0; off >>= 1) {
-      const float od = __shfl_xor_sync(0xffffffffu, best_d, off);
-      const int oi = __shfl_xor_sync(0xffffffffu, best_i, off);
-      if (better(od, oi, best_d, best_i)) {
-        best_d = od;
-        best_i = oi;
-      }
-    }
-    if (lane == 0) {
-      red_d[warp] = best_d;
-      red_i[warp] = best_i;
+  // the seed, U[0], is the first pick
+  for (int t = tid; t < d; t += kThreads) {
+    s.pvec[t] = static_cast<float>(pt(0)[t]);
+    out[t] = pt(0)[t];
+  }
+  __syncthreads();
+  if (tid == 0) s.pinv[0] = s.inv[0];
+  __syncthreads();
+  point_pass_dispatch(s, pt, n, d, 1, true);
+  __syncthreads();
+  if (tid == 0) s.dist[0] = -1.f;
+  __syncthreads();
+
+  int picked = 1;
+  while (picked < m) {
+    const int unsel = n - picked;
+    const int nc = min(kCand, unsel);           // candidates this round
+    const bool bounded = unsel > kCand;         // a (kCand+1)-th point exists
+    select_best(s, n, bounded ? kCand + 1 : nc);
+    __syncthreads();
+    // order the selected points: rank by (distance desc, index asc)
+    const int want = bounded ? kCand + 1 : nc;
+    int my_i = 0;
+    float my_d = 0.f;
+    int my_rank = 0;
+    if (tid < want) {
+      my_i = s.cidx[tid];
+      my_d = s.cdist[tid];
+      for (int j = 0; j < want; ++j)
+        if (j != tid && before(s.cdist[j], s.cidx[j], my_d, my_i)) ++my_rank;
     }
     __syncthreads();
+    if (tid < want) {
+      s.cidx[my_rank] = my_i;
+      s.cdist[my_rank] = my_d;
+    }
+    __syncthreads();
+    // candidate vectors, f32
+    for (int e = tid; e < nc * (d / 8); e += kThreads) {
+      const int a = e / (d / 8), t = (e - a * (d / 8)) * 8;
+      float u[8];
+      load8(pt(s.cidx[a]) + t, u);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) s.cvec[a * kMaxDim + t + j] = u[j];
+    }
+    __syncthreads();
+    // Gram block: gram[a][b] = u_a . u_b with a as the point and b as the pick
+    for (int e = tid; e < nc * nc; e += kThreads) {
+      const int a = e / nc, b = e - a * nc;
+      float2 acc = make_float2(0.f, 0.f);
+      for (int t = 0; t < d; t += 8) {
+        float u[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) u[j] = s.cvec[a * kMaxDim + t + j];
+        acc = dot8_step(acc, u, s.cvec + b * kMaxDim + t);
+      }
+      s.gram[a * kCand + b] = __fadd_rn(acc.x, acc.y);
+    }
+    __syncthreads();
+    // replay the greedy choice among the candidates (warp 0; lane a = candidate a)
     if (warp == 0) {
-      best_d = lane < kWarps ? red_d[lane] : -2.f;
-      best_i = lane < kWarps ? red_i[lane] : n;
-      for (int off = 16; off > 0; off >>= 1) {
-        const float od = __shfl_xor_sync(0xffffffffu, best_d, off);
-        const int oi = __shfl_xor_sync(0xffffffffu, best_i, off);
-        if (better(od, oi, best_d, best_i)) {
-          best_d = od;
-          best_i = oi;
+      const bool live = lane < nc;
+      float cd = live ? s.cdist[lane] : -3.f;
+      const int ci = live ? s.cidx[lane] : 0x7fffffff;
+      const float cinv = live ? s.inv[ci] : 0.f;
+      const float bd = bounded ? s.cdist[kCand] : -3.f;
+      const int bi = bounded ? s.cidx[kCand] : 0x7fffffff;
+      bool taken = !live;
+      int np = 0;
+      while (picked + np < m) {
+        float best_d = taken ? -3.f : cd;
+        int best_i = taken ? 0x7fffffff : ci;
+        int best_a = lane;
+        for (int off = 16; off > 0; off >>= 1) {
+          const float od = __shfl_xor_sync(0xffffffffu, best_d, off);
+          const int oi = __shfl_xor_sync(0xffffffffu, best_i, off);
+          const int oa = __shfl_xor_sync(0xffffffffu, best_a, off);
+          if (before(od, oi, best_d, best_i)) {
+            best_d = od;
+            best_i = oi;
+            best_a = oa;
+          }
+        }
+        if (best_d < 0.f) break;                       // no candidate left
+        if (bounded && !before(best_d, best_i, bd, bi)) break;
+        if (lane == 0) s.pick[np] = best_a;
+        ++np;
+        if (lane == best_a) taken = true;
+        if (!taken) {
+          const float2 dotv = make_float2(s.gram[lane * kCand + best_a], 0.f);
+          cd = fminf(cd, cos_dist(dotv, cinv, s.inv[best_i]));
         }
       }
-      if (lane == 0) pick_sh = best_i;
+      if (lane == 0) s.scal[4] = np;
     }
     __syncthreads();
-    pick = pick_sh;
+    const int np = s.scal[4];
+    // this round's picks: outputs, vectors, inverse norms
+    for (int e = tid; e < np * d; e += kThreads) {
+      const int k = e / d, t = e - k * d;
+      const int a = s.pick[k];
+      s.pvec[k * kMaxDim + t] = s.cvec[a * kMaxDim + t];
+      out[static_cast<size_t>(picked + k) * d + t] = pt(s.cidx[a])[t];
+    }
+    if (tid < np) s.pinv[tid] = s.inv[s.cidx[s.pick[tid]]];
+    __syncthreads();
+    if (tid < np) s.dist[s.cidx[s.pick[tid]]] = -1.f;
+    __syncthreads();
+    point_pass_dispatch(s, pt, n, d, np, false);
+    __syncthreads();
+    picked += np;
   }
 }
 
 size_t fps_smem_bytes(const FpsGeom &g) {
-  return (kMaxDim + 2 * static_cast<size_t>(g.nb_in + g.W)) * sizeof(float);
+  const size_t n = static_cast<size_t>(g.nb_in) + g.W;
+  return sizeof(float) * (2 * kCand * kMaxDim + kCand * kCand + kCand + kCand + 4 + 2 * n) +
+         sizeof(uint32_t) * 256 + sizeof(int) * (kCand + 4 + kCand + 8);
 }
 
 template <typename T>
 bkv_status launch_typed(const FpsGeom &g, const void *bin, const void *win, void *bout,
                         cudaStream_t stream) {
   static int attr_done[64];
-  if (!ensure_smem_limit(fps_kernel<T>, kSmemLimit - 1024, attr_done)) return BKV_ERR_CUDA;
+  if (!ensure_smem_limit(fps_kernel<T>, kSmemLimit, attr_done)) return BKV_ERR_CUDA;
   const unsigned grid = static_cast<unsigned>(g.n_layers) * static_cast<unsigned>(g.n_q_heads);
   fps_kernel<T><<<grid, kThreads, fps_smem_bytes(g), stream>>>(
       g, static_cast<const T *>(bin), static_cast<const T *>(win), static_cast<T *>(bout));
@@ -194,7 +405,8 @@ bkv_status launch_typed(const FpsGeom &g, const void *bin, const void *win, void
 size_t fps_workspace_bytes(const FpsGeom &) { return 0; }
 
 bool fps_supported(const FpsGeom &g) {
-  return g.head_dim <= kMaxDim && fps_smem_bytes(g) <= static_cast<size_t>(kSmemLimit - 1024);
+  return g.head_dim <= kMaxDim && g.head_dim % 8 == 0 &&
+         fps_smem_bytes(g) <= static_cast<size_t>(kSmemLimit);
 }
 
 bkv_status launch_fps(const FpsGeom &g, const void *beacons_in, const void *window,
