@@ -175,6 +175,32 @@ typedef struct {
 bkv_status bkv_compress_step(const bkv_step_args *args, int32_t *n_beacons_out,
                              int64_t *new_len);
 
+/* Scoring without a caller workspace.  The paper has no counterpart: this is
+ * an interface addition for callers that cannot allocate device memory where
+ * they score -- for example code running inside another runtime's execute
+ * callback that hands over only the tensors it asked for, or a serving loop
+ * that must not allocate after start-up because a pool allocator has reserved
+ * the device's memory.  Same arguments and results as bkv_score, without the
+ * workspace: the scratch is one array of BKV_SCORE_NOALLOC_SCRATCH_BYTES
+ * (32 MiB) compiled into libbkv.so, which every GPU that loads the library
+ * holds until the process exits.
+ *   - The first call on each device looks up the array's device address with
+ *     that device current (cudaGetSymbolAddress); make that first call before
+ *     any stream capture.
+ *   - A problem whose scratch does not fit the array (at most
+ *     bkv_workspace_size(desc, L, R, n_beacons, 0, 1) bytes are needed) is
+ *     rejected with BKV_ERR_WORKSPACE before anything is launched.
+ *   - Every call uses the same array and leaves its contents behind.  Calls
+ *     whose kernels can overlap on the GPU (other streams, other host threads)
+ *     race on it and produce wrong scores: order them on one stream or with
+ *     events.  Nothing in the array needs to start at zero.
+ *   - It calls no cudaMalloc, cudaFree or other allocating routine. */
+#define BKV_SCORE_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+bkv_status bkv_score_noalloc(const bkv_cache_desc *desc, const void *k,
+                             int64_t L, const void *recent_q, int32_t R,
+                             const void *beacons, int32_t n_beacons, int32_t M,
+                             float scale, float *scores, void *stream);
+
 /* Device-side status.  Kernels never trap: a bounded wait that runs out or a
  * failed consistency check records BKV_ERR_TIMEOUT / BKV_ERR_DEVICE_ASSERT in
  * a status word of the library instead.  This call synchronises `stream`,

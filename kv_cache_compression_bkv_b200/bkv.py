@@ -24,7 +24,8 @@ STATUS = {0: "BKV_OK", 1: "BKV_ERR_INVALID_ARG", 2: "BKV_ERR_UNSUPPORTED",
           6: "BKV_ERR_DEVICE_ASSERT"}
 EXPORTS = ("bkv_workspace_size", "bkv_score", "bkv_select_topk", "bkv_compact",
            "bkv_update_beacons", "bkv_compress_step", "bkv_read_device_status",
-           "bkv_status_string")
+           "bkv_status_string", "bkv_score_noalloc")
+SCORE_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 class BkvError(RuntimeError):
@@ -74,6 +75,7 @@ def _load() -> ctypes.CDLL:
                                ctypes.POINTER(I64)], ctypes.c_int),
         "bkv_read_device_status": ([P, ctypes.POINTER(I32)], ctypes.c_int),
         "bkv_status_string": ([ctypes.c_int], ctypes.c_char_p),
+        "bkv_score_noalloc": ([D, P, I64, P, I32, P, I32, I32, F, P, P], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -146,6 +148,16 @@ def bkv_score(geom: Geometry, k, L: int, recent_q, R: int, beacons, n_beacons: i
                          M, scale, _ptr(scores), _ptr(workspace),
                          0 if workspace is None else workspace.numel() * workspace.element_size(),
                          _stream(stream)), "bkv_score")
+
+
+def bkv_score_noalloc(geom: Geometry, k, L: int, recent_q, R: int, beacons, n_beacons: int,
+                      M: int, scale: float, scores, stream=None) -> None:
+    """bkv_score on the library's built-in scratch array, for callers that
+    cannot allocate device memory where they score (no workspace argument)."""
+    d = geom.desc()
+    _check(LIB.bkv_score_noalloc(ctypes.byref(d), _ptr(k), L, _ptr(recent_q), R, _ptr(beacons),
+                                 n_beacons, M, scale, _ptr(scores), _stream(stream)),
+           "bkv_score_noalloc")
 
 
 def bkv_select_topk(scores, n_rows: int, L: int, K: int, idx, workspace=None,
