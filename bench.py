@@ -113,10 +113,10 @@ class ClockSampler:
         self.path = None
         self.err = None
         try:
-            bus = torch.cuda.get_device_properties(device_index).pci_bus_id
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            self.sel = ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
         except Exception:
-            bus = None
-        self.sel = ["-i", str(bus)] if bus else []
+            self.sel = []
 
     def start(self):
         fd, self.path = tempfile.mkstemp(prefix="bkv_clocks_", suffix=".csv")
@@ -149,9 +149,12 @@ class ClockSampler:
                 parts = [p.strip() for p in line.split(",")]
                 if len(parts) >= 9:
                     rows.append(parts)
-        os.unlink(self.path)
         if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+            with open(self.path) as f:
+                head = f.read(200).strip().replace("\n", " ")
+            os.unlink(self.path)
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples: " + head]}
+        os.unlink(self.path)
         sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
         mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
@@ -254,11 +257,15 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="use only this many layers (small cases for profiler captures)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
     from kv_cache_compression_bkv_b200 import synth
     wl = synth.WORKLOADS[args.workload]
+    if args.layers:
+        wl = wl.replace(n_layers=args.layers)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -29,64 +29,24 @@
 #include <algorithm>
 
 #include "bkv_internal.h"
+#include "fps_common.cuh"
 
 namespace bkv {
 namespace {
+
+using namespace fpsk;
 
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kCand = 32;        // candidates per round (T)
 constexpr int kMaxDim = 128;
+constexpr int kCStride = kMaxDim + 4;  // candidate rows, padded against bank conflicts
 constexpr int kSmemLimit = 232448;
-
-// ---- element access: 8 consecutive elements as f32
-__device__ __forceinline__ void load8(const __nv_bfloat16 *p, float (&u)[8]) {
-  const uint4 w = *reinterpret_cast<const uint4 *>(p);
-  u[0] = __uint_as_float(w.x << 16); u[1] = __uint_as_float(w.x & 0xffff0000u);
-  u[2] = __uint_as_float(w.y << 16); u[3] = __uint_as_float(w.y & 0xffff0000u);
-  u[4] = __uint_as_float(w.z << 16); u[5] = __uint_as_float(w.z & 0xffff0000u);
-  u[6] = __uint_as_float(w.w << 16); u[7] = __uint_as_float(w.w & 0xffff0000u);
-}
-__device__ __forceinline__ void load8(const float *p, float (&u)[8]) {
-  const float4 a = *reinterpret_cast<const float4 *>(p);
-  const float4 b = *reinterpret_cast<const float4 *>(p + 4);
-  u[0] = a.x; u[1] = a.y; u[2] = a.z; u[3] = a.w;
-  u[4] = b.x; u[5] = b.y; u[6] = b.z; u[7] = b.w;
-}
-
-// One 8-element step of a dot product, the same operation sequence wherever a
-// dot product is formed (point pass and Gram block), so both agree bit for bit.
-__device__ __forceinline__ float2 dot8_step(float2 acc, const float (&u)[8], const float *s) {
-  const float4 s0 = *reinterpret_cast<const float4 *>(s);
-  const float4 s1 = *reinterpret_cast<const float4 *>(s + 4);
-  acc = __ffma2_rn(make_float2(u[0], u[1]), make_float2(s0.x, s0.y), acc);
-  acc = __ffma2_rn(make_float2(u[2], u[3]), make_float2(s0.z, s0.w), acc);
-  acc = __ffma2_rn(make_float2(u[4], u[5]), make_float2(s1.x, s1.y), acc);
-  acc = __ffma2_rn(make_float2(u[6], u[7]), make_float2(s1.z, s1.w), acc);
-  return acc;
-}
-
-__device__ __forceinline__ float cos_dist(float2 acc, float inv_a, float inv_b) {
-  const float dot = __fadd_rn(acc.x, acc.y);
-  const float dd = __fmaf_rn(-__fmul_rn(dot, inv_a), inv_b, 1.0f);
-  return fminf(fmaxf(dd, 0.f), 2.f);
-}
-
-// Order key of a distance: larger distance -> larger key; selected points
-// (distance -1) -> 0, below every unselected point.
-__device__ __forceinline__ uint32_t dist_key(float d) {
-  return d < 0.f ? 0u : (__float_as_uint(d) | 0x80000000u);
-}
-
-// (distance desc, index asc): true if (da, ia) comes before (db, ib).
-__device__ __forceinline__ bool before(float da, int ia, float db, int ib) {
-  return da > db || (da == db && ia < ib);
-}
 
 struct Smem {
   float *dist;       // [n]
   float *inv;        // [n]
-  float *cvec;       // [kCand][d] candidate vectors (f32)
+  float *cvec;       // [kCand][kCStride] candidate vectors (f32)
   float *pvec;       // [kCand][d] this round's picks (f32)
   float *gram;       // [kCand][kCand]
   uint32_t *hist;    // [256]
@@ -108,9 +68,8 @@ struct Points {
 
 // Lower every unselected point's distance by the picks pvec[0..np) (or set it,
 // for the seed).  NP >= np accumulators are carried; the extra ones are not used.
-template <int NP, typename T>
-__device__ void point_pass(const Smem &s, const Points<T> &pt, int n, int d, int np,
-                           bool first) {
+template <int NP, int D, typename T>
+__device__ void point_pass(const Smem &s, const Points<T> &pt, int n, int np, bool first) {
   for (int i = threadIdx.x; i < n; i += kThreads) {
     float di = s.dist[i];
     if (!first && di < 0.f) continue;
@@ -118,7 +77,8 @@ __device__ void point_pass(const Smem &s, const Points<T> &pt, int n, int d, int
     float2 acc[NP];
 #pragma unroll
     for (int k = 0; k < NP; ++k) acc[k] = make_float2(0.f, 0.f);
-    for (int t = 0; t < d; t += 8) {
+#pragma unroll
+    for (int t = 0; t < D; t += 8) {
       float u[8];
       load8(p + t, u);
 #pragma unroll
@@ -136,18 +96,18 @@ __device__ void point_pass(const Smem &s, const Points<T> &pt, int n, int d, int
   }
 }
 
-template <typename T>
-__device__ void point_pass_dispatch(const Smem &s, const Points<T> &pt, int n, int d, int np,
+template <int D, typename T>
+__device__ void point_pass_dispatch(const Smem &s, const Points<T> &pt, int n, int np,
                                     bool first) {
   switch ((np + 3) >> 2) {
-    case 1: point_pass<4>(s, pt, n, d, np, first); break;
-    case 2: point_pass<8>(s, pt, n, d, np, first); break;
-    case 3: point_pass<12>(s, pt, n, d, np, first); break;
-    case 4: point_pass<16>(s, pt, n, d, np, first); break;
-    case 5: point_pass<20>(s, pt, n, d, np, first); break;
-    case 6: point_pass<24>(s, pt, n, d, np, first); break;
-    case 7: point_pass<28>(s, pt, n, d, np, first); break;
-    default: point_pass<32>(s, pt, n, d, np, first); break;
+    case 1: point_pass<4, D>(s, pt, n, np, first); break;
+    case 2: point_pass<8, D>(s, pt, n, np, first); break;
+    case 3: point_pass<12, D>(s, pt, n, np, first); break;
+    case 4: point_pass<16, D>(s, pt, n, np, first); break;
+    case 5: point_pass<20, D>(s, pt, n, np, first); break;
+    case 6: point_pass<24, D>(s, pt, n, np, first); break;
+    case 7: point_pass<28, D>(s, pt, n, np, first); break;
+    default: point_pass<32, D>(s, pt, n, np, first); break;
   }
 }
 
@@ -230,17 +190,17 @@ __device__ void select_best(const Smem &s, int n, int want) {
   }
 }
 
-template <typename T>
+template <typename T, int D>
 __global__ void __launch_bounds__(kThreads, 1)
     fps_kernel(const FpsGeom g, const T *__restrict__ beacons_in, const T *__restrict__ window,
                T *__restrict__ beacons_out) {
   extern __shared__ __align__(16) float sm[];
-  const int d = g.head_dim;
+  constexpr int d = D;
   const int n = g.nb_in + g.W;
   const int m = g.n_pick;
   Smem s;
   s.cvec = sm;
-  s.pvec = s.cvec + kCand * kMaxDim;
+  s.pvec = s.cvec + kCand * kCStride;
   s.gram = s.pvec + kCand * kMaxDim;
   s.pinv = s.gram + kCand * kCand;
   s.cdist = s.pinv + kCand;
@@ -261,7 +221,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int i = tid; i < n; i += kThreads) {
     const T *p = pt(i);
     float ss = 0.f;
-    for (int t = 0; t < d; t += 8) {
+#pragma unroll
+    for (int t = 0; t < D; t += 8) {
       float u[8];
       load8(p + t, u);
 #pragma unroll
@@ -277,7 +238,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (tid == 0) s.pinv[0] = s.inv[0];
   __syncthreads();
-  point_pass_dispatch(s, pt, n, d, 1, true);
+  point_pass_dispatch<D>(s, pt, n, 1, true);
   __syncthreads();
   if (tid == 0) s.dist[0] = -1.f;
   __syncthreads();
@@ -312,18 +273,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       float u[8];
       load8(pt(s.cidx[a]) + t, u);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) s.cvec[a * kMaxDim + t + j] = u[j];
+      for (int j = 0; j < 8; ++j) s.cvec[a * kCStride + t + j] = u[j];
     }
     __syncthreads();
     // Gram block: gram[a][b] = u_a . u_b with a as the point and b as the pick
+    // (lanes take consecutive points a of one pick b: the b row is a broadcast
+    // and the a rows fall in distinct banks)
     for (int e = tid; e < nc * nc; e += kThreads) {
-      const int a = e / nc, b = e - a * nc;
+      const int b = e / nc, a = e - b * nc;
       float2 acc = make_float2(0.f, 0.f);
-      for (int t = 0; t < d; t += 8) {
+      for (int t = 0; t < D; t += 8) {
         float u[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) u[j] = s.cvec[a * kMaxDim + t + j];
-        acc = dot8_step(acc, u, s.cvec + b * kMaxDim + t);
+        load8(s.cvec + a * kCStride + t, u);
+        acc = dot8_step(acc, u, s.cvec + b * kCStride + t);
       }
       s.gram[a * kCand + b] = __fadd_rn(acc.x, acc.y);
     }
@@ -370,14 +332,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int e = tid; e < np * d; e += kThreads) {
       const int k = e / d, t = e - k * d;
       const int a = s.pick[k];
-      s.pvec[k * kMaxDim + t] = s.cvec[a * kMaxDim + t];
+      s.pvec[k * kMaxDim + t] = s.cvec[a * kCStride + t];
       out[static_cast<size_t>(picked + k) * d + t] = pt(s.cidx[a])[t];
     }
     if (tid < np) s.pinv[tid] = s.inv[s.cidx[s.pick[tid]]];
     __syncthreads();
     if (tid < np) s.dist[s.cidx[s.pick[tid]]] = -1.f;
     __syncthreads();
-    point_pass_dispatch(s, pt, n, d, np, false);
+    point_pass_dispatch<D>(s, pt, n, np, false);
     __syncthreads();
     picked += np;
   }
@@ -385,19 +347,32 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 size_t fps_smem_bytes(const FpsGeom &g) {
   const size_t n = static_cast<size_t>(g.nb_in) + g.W;
-  return sizeof(float) * (2 * kCand * kMaxDim + kCand * kCand + kCand + kCand + 4 + 2 * n) +
+  return sizeof(float) * (kCand * kCStride + kCand * kMaxDim + kCand * kCand + kCand + kCand +
+                          4 + 2 * n) +
          sizeof(uint32_t) * 256 + sizeof(int) * (kCand + 4 + kCand + 8);
 }
 
-template <typename T>
+template <typename T, int D>
 bkv_status launch_typed(const FpsGeom &g, const void *bin, const void *win, void *bout,
                         cudaStream_t stream) {
   static int attr_done[64];
-  if (!ensure_smem_limit(fps_kernel<T>, kSmemLimit, attr_done)) return BKV_ERR_CUDA;
+  if (!ensure_smem_limit(fps_kernel<T, D>, kSmemLimit, attr_done)) return BKV_ERR_CUDA;
   const unsigned grid = static_cast<unsigned>(g.n_layers) * static_cast<unsigned>(g.n_q_heads);
-  fps_kernel<T><<<grid, kThreads, fps_smem_bytes(g), stream>>>(
+  fps_kernel<T, D><<<grid, kThreads, fps_smem_bytes(g), stream>>>(
       g, static_cast<const T *>(bin), static_cast<const T *>(win), static_cast<T *>(bout));
   return cudaGetLastError() == cudaSuccess ? BKV_OK : BKV_ERR_CUDA;
+}
+
+template <typename T>
+bkv_status launch_dim(const FpsGeom &g, const void *bin, const void *win, void *bout,
+                      cudaStream_t stream) {
+  switch (g.head_dim) {
+    case 32: return launch_typed<T, 32>(g, bin, win, bout, stream);
+    case 64: return launch_typed<T, 64>(g, bin, win, bout, stream);
+    case 96: return launch_typed<T, 96>(g, bin, win, bout, stream);
+    case 128: return launch_typed<T, 128>(g, bin, win, bout, stream);
+    default: return BKV_ERR_UNSUPPORTED;
+  }
 }
 
 }  // namespace
@@ -405,7 +380,7 @@ bkv_status launch_typed(const FpsGeom &g, const void *bin, const void *win, void
 size_t fps_workspace_bytes(const FpsGeom &) { return 0; }
 
 bool fps_supported(const FpsGeom &g) {
-  return g.head_dim <= kMaxDim && g.head_dim % 8 == 0 &&
+  return (g.head_dim == 32 || g.head_dim == 64 || g.head_dim == 96 || g.head_dim == 128) &&
          fps_smem_bytes(g) <= static_cast<size_t>(kSmemLimit);
 }
 
@@ -414,8 +389,8 @@ bkv_status launch_fps(const FpsGeom &g, const void *beacons_in, const void *wind
   if (!fps_supported(g)) return BKV_ERR_UNSUPPORTED;
   if (g.n_pick <= 0) return BKV_OK;
   if (g.dtype == BKV_BF16)
-    return launch_typed<__nv_bfloat16>(g, beacons_in, window, beacons_out, stream);
-  return launch_typed<float>(g, beacons_in, window, beacons_out, stream);
+    return launch_dim<__nv_bfloat16>(g, beacons_in, window, beacons_out, stream);
+  return launch_dim<float>(g, beacons_in, window, beacons_out, stream);
 }
 
 }  // namespace bkv

@@ -55,6 +55,66 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// max(a, b, c) in one instruction (three-input max, sm_100).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+__device__ __forceinline__ float max32(const float (&v)[32]) {
+  float r[11];
+#pragma unroll
+  for (int i = 0; i < 10; ++i) r[i] = max3f(v[3 * i], v[3 * i + 1], v[3 * i + 2]);
+  r[10] = fmaxf(v[30], v[31]);
+  const float a = max3f(r[0], r[1], r[2]), b = max3f(r[3], r[4], r[5]);
+  const float c = max3f(r[6], r[7], r[8]), e = max3f(r[9], r[10], a);
+  return max3f(b, c, e);
+}
+
+// 2^x on the FMA pipe, for a pair of x <= 0: Cody-Waite reduction x = j + f
+// with j = rint(x) (by adding 1.5 * 2^23) and f in [-0.5, 0.5]; a cubic
+// p(f) ~ 2^f (coefficients from fit_exp2_poly.py, max relative error 7.6e-5);
+// then 2^j is added into p's exponent field.  x is clamped at -126, so the
+// smallest result is about 1e-38 instead of 0.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 t = __fadd2_rn(x, make_float2(kMagic, kMagic));
+  const float2 j = __fadd2_rn(t, make_float2(-kMagic, -kMagic));
+  const float2 f = __ffma2_rn(j, make_float2(-1.f, -1.f), x);
+  float2 p = __ffma2_rn(f, make_float2(0.05517051f, 0.05517051f),
+                        make_float2(0.24260840f, 0.24260840f));
+  p = __ffma2_rn(p, f, make_float2(0.69326091f, 0.69326091f));
+  p = __ffma2_rn(p, f, make_float2(0.99992824f, 0.99992824f));
+  const uint32_t ex = __float_as_uint(t.x) << 23, ey = __float_as_uint(t.y) << 23;
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + ex),
+                     __uint_as_float(__float_as_uint(p.y) + ey));
+}
+
+// Sum of 2^(v[i] * kz - m) over one 32-column chunk.  The first kPolyPairs
+// pairs go through exp2_poly2 (FMA pipe), the rest through ex2.approx (MUFU),
+// so that both pipes share the load.
+constexpr int kPolyPairs = 7;
+__device__ __forceinline__ float chunk_exp_sum(const float (&v)[32], float kz, float m) {
+  const float2 kz2 = make_float2(kz, kz), nm2 = make_float2(-m, -m);
+  float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int p = 0; p < 16; ++p) {
+    const float2 a = __ffma2_rn(make_float2(v[2 * p], v[2 * p + 1]), kz2, nm2);
+    float2 e;
+    if (p < kPolyPairs) {
+      e = exp2_poly2(a);
+    } else {
+      e.x = ex2_approx(a.x);
+      e.y = ex2_approx(a.y);
+    }
+    acc = __fadd2_rn(acc, e);
+  }
+  return acc.x + acc.y;
+}
+
 __device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
@@ -102,7 +162,8 @@ __device__ __forceinline__ void load_obs_rows_sw128(uint8_t *dst, int nrows, int
 constexpr int kP1Rows = 128;
 constexpr int kP1Keys = 256;
 constexpr int kP1Stages = 3;
-constexpr int kP1Threads = 384;  // warp 0 TMA, warp 1 MMA, warps 4..11 epilogue
+constexpr int kP1EpiWarps = 16;  // 4 warpgroups, 64 of the 256 columns each
+constexpr int kP1Threads = 128 + 32 * kP1EpiWarps;  // warp 0 TMA, warp 1 MMA, 4.. epilogue
 constexpr int kP1ABytes = kP1Rows * kRowBytes;     // 32 KB
 constexpr int kP1StageBytes = kP1Keys * kRowBytes; // 64 KB
 constexpr int kP1SmallBytes = 2048;                // barriers, TMEM slot, exchange
@@ -116,7 +177,6 @@ __global__ void __launch_bounds__(kP1Threads, 1)
   // small objects first, then the 1024-aligned operand tiles
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem_raw);  // 16 barriers
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem_raw + 128);
-  float *xchg = reinterpret_cast<float *>(smem_raw + 1024);  // [128][2]
   const uint32_t raw_base = smem_u32(smem_raw);
   const uint32_t tile_base = (raw_base + kP1SmallBytes + 1023u) & ~1023u;
   uint8_t *sA = smem_raw + (tile_base - raw_base);
@@ -141,7 +201,7 @@ __global__ void __launch_bounds__(kP1Threads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull0 + 8 * a, 1);
-      mbar_init(tempty0 + 8 * a, 8);  // one arrive per epilogue warp
+      mbar_init(tempty0 + 8 * a, kP1EpiWarps);  // one arrive per epilogue warp
     }
     mbar_init(done, 1);
     fence_barrier_init();
@@ -205,7 +265,9 @@ __global__ void __launch_bounds__(kP1Threads, 1)
       mbar_wait(done, 0, kWhereP1Drain);
     }
   } else if (warp >= 4) {
-    // ---- epilogue: two warpgroups split the 256 columns of each tile
+    // ---- epilogue: four warpgroups, each owning 64 of the 256 columns of a
+    // tile; TMEM lane = observation row, so every thread keeps its row's
+    // online max and sum of 2^(x log2 e) over its columns
     const int wg = (warp - 4) >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
@@ -217,53 +279,57 @@ __global__ void __launch_bounds__(kP1Threads, 1)
       if (!mbar_wait(tfull0 + 8 * acc, (t >> 1) & 1, kWhereP1Epi)) { ok = false; break; }
       tc_fence_after();
       const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) +
-                             acc * kP1Keys + wg * 128;
-      const long long key_base = static_cast<long long>(t) * kP1Keys + wg * 128;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        float v[32];
-        tmem_ld_32x32b_x32(taddr + c * 32, v);
-        tmem_ld_wait();
+                             acc * kP1Keys + wg * 64;
+      const long long key_base = static_cast<long long>(t) * kP1Keys + wg * 64;
+      float va[32], vb[32];
+      tmem_ld_32x32b_x32(taddr, va);
+      tmem_ld_32x32b_x32(taddr + 32, vb);
+      tmem_ld_wait_regs(va);
+      tmem_reg_fence(vb);
+      // the accumulator buffer is free as soon as both loads have landed
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        float (&cur)[32] = c ? vb : va;
         const long long k0 = key_base + c * 32;
         if (k0 + 32 > L) {
 #pragma unroll
           for (int i = 0; i < 32; ++i)
-            if (k0 + i >= L) v[i] = -INFINITY;
+            if (k0 + i >= L) cur[i] = -INFINITY;
         }
-        float cm = v[0];
-#pragma unroll
-        for (int i = 1; i < 32; ++i) cm = fmaxf(cm, v[i]);
-        const float mz = cm * kz;
+        const float mz = max32(cur) * kz;
         if (mz > m) {
           ssum *= ex2_approx(m - mz);
           m = mz;
         }
-        if (m == -INFINITY) continue;  // every column seen so far is masked
-        float cs0 = 0.f, cs1 = 0.f;
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          cs0 += ex2_approx(fmaf(v[i], kz, -m));
-          cs1 += ex2_approx(fmaf(v[i + 1], kz, -m));
-        }
-        ssum += cs0 + cs1;
+        if (m != -INFINITY) ssum += chunk_exp_sum(cur, kz, m);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
     }
-    // combine the two column halves of each row
-    if (wg == 1) {
-      xchg[row * 2] = m;
-      xchg[row * 2 + 1] = ok ? ssum : -1.f;
+    // combine the four column quarters of each row; the exchange reuses the
+    // key stages, free once the last tile's MMAs have completed
+    float *xchg = reinterpret_cast<float *>(sB);  // [3][128][2]
+    if (wg > 0) {
+      xchg[((wg - 1) * kP1Rows + row) * 2] = m;
+      xchg[((wg - 1) * kP1Rows + row) * 2 + 1] = ok ? ssum : -1.f;
     }
-    named_barrier_sync(1, 256);
+    named_barrier_sync(1, 32 * kP1EpiWarps);
     if (wg == 0) {
-      const float m1 = xchg[row * 2], s1 = xchg[row * 2 + 1];
       const int o = rb * kP1Rows + row;
-      if (ok && s1 >= 0.f && o < g.n_obs) {
-        const float M = fmaxf(m, m1);
-        const float S = (m == -INFINITY ? 0.f : ssum * ex2_approx(m - M)) +
-                        (m1 == -INFINITY ? 0.f : s1 * ex2_approx(m1 - M));
+      float M = m;
+      bool all_ok = ok;
+      for (int w = 0; w < 3; ++w) {
+        M = fmaxf(M, xchg[(w * kP1Rows + row) * 2]);
+        all_ok &= xchg[(w * kP1Rows + row) * 2 + 1] >= 0.f;
+      }
+      if (all_ok && o < g.n_obs) {
+        float S = m == -INFINITY ? 0.f : ssum * ex2_approx(m - M);
+        for (int w = 0; w < 3; ++w) {
+          const float mw = xchg[(w * kP1Rows + row) * 2];
+          const float sw = xchg[(w * kP1Rows + row) * 2 + 1];
+          if (mw != -INFINITY) S += sw * ex2_approx(mw - M);
+        }
         c_out[static_cast<size_t>(head) * g.n_obs_pad + o] = (M + log2f(S)) * kLn2;
       }
     }
@@ -426,7 +492,7 @@ __global__ void __launch_bounds__(kP2Threads, 1)
         for (; col + 32 <= Nu; col += 32) {
           float v[32];
           tmem_ld_32x32b_x32(taddr + col, v);
-          tmem_ld_wait();
+          tmem_ld_wait_regs(v);
 #pragma unroll
           for (int i = 0; i < 32; i += 4) {
             const float4 c4 = *reinterpret_cast<const float4 *>(cu + col + i);
@@ -437,7 +503,7 @@ __global__ void __launch_bounds__(kP2Threads, 1)
         if (col < Nu) {  // Nu is a multiple of 16
           float v[16];
           tmem_ld_32x32b_x16(taddr + col, v);
-          tmem_ld_wait();
+          tmem_ld_wait_regs(v);
 #pragma unroll
           for (int i = 0; i < 16; i += 4) {
             const float4 c4 = *reinterpret_cast<const float4 *>(cu + col + i);
@@ -527,13 +593,32 @@ bkv_status launch_score_colmax_tc(const ScoreGeom &g, const void *k, const void 
   static int attr_done[64];
   if (!ensure_smem_limit(score_colmax_kernel, kSmemLimit, attr_done)) return BKV_ERR_CUDA;
   const int n_tiles = static_cast<int>((g.L + kP2Keys - 1) / kP2Keys);
-  // Split the keys of a head into chunks so that the grid covers the 148 SMs
-  // several times; each chunk reloads the observation rows once.
+  // Split the keys of a head into chunks so that the CTAs fill whole waves of
+  // the SMs (one CTA per SM): the fewest chunks whose last wave is at least
+  // 95% full, else the best fill found.  Each chunk reloads its observation
+  // rows once, so chunks keep at least 8 tiles.
+  int sms = 148;
+  {
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  }
   const long long units = static_cast<long long>(g.n_heads()) * g.n_groups;
-  int n_chunks = static_cast<int>(std::max(1LL, (4LL * 148 + units - 1) / units));
-  n_chunks = std::min(n_chunks, std::max(1, n_tiles / 8));
-  const int chunk_tiles = (n_tiles + n_chunks - 1) / n_chunks;
-  n_chunks = (n_tiles + chunk_tiles - 1) / chunk_tiles;
+  int n_chunks = 1, chunk_tiles = n_tiles;
+  double best_fill = 0.0;
+  for (int nc = 1; nc <= std::max(1, n_tiles / 8) && nc <= 32; ++nc) {
+    const int ct = (n_tiles + nc - 1) / nc;
+    const int ncr = (n_tiles + ct - 1) / ct;
+    const long long ctas = units * ncr;
+    const long long waves = (ctas + sms - 1) / sms;
+    const double fill = static_cast<double>(ctas) / static_cast<double>(waves * sms);
+    if (fill > best_fill + 1e-9) {
+      best_fill = fill;
+      n_chunks = ncr;
+      chunk_tiles = ct;
+    }
+    if (fill >= 0.95) break;
+  }
   const long long grid = units * n_chunks;
   score_colmax_kernel<<<static_cast<unsigned>(grid), kP2Threads, smem, stream>>>(
       map, g, static_cast<const uint16_t *>(recent), static_cast<const uint16_t *>(beacons), c,

@@ -23,9 +23,25 @@ namespace {
 
 constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
-constexpr int kSmallWords = 256 + 2 * kWarps + 8;  // histogram, warp counts, scalars
+// histogram, per-warp histograms, warp counts and offsets, scalars
+constexpr int kSmallWords = 256 + kWarps * 256 + 4 * kWarps + 8;
 constexpr int kSmemLimit = 232448;
 constexpr long long kMaxSmemKeys = (kSmemLimit - kSmallWords * 4) / 4;
+
+// Exclusive prefix sums of the per-warp counts cnt[0..kWarps) into off[], and
+// their total into *total (warp 0 only; the caller synchronises).
+__device__ __forceinline__ void scan_warp_counts(const uint32_t *cnt, uint32_t *off,
+                                                 uint32_t *total, int lane) {
+  const uint32_t c = cnt[lane];
+  uint32_t incl = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  off[lane] = incl - c;
+  if (lane == 31) *total = incl;
+}
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   if (f == 0.f) f = 0.f;  // -0 -> +0
@@ -43,9 +59,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     select_topk_kernel(const SelectInput in, long long L, long long K, int32_t *__restrict__ idx,
                        float *__restrict__ s_out, uint32_t *__restrict__ gkeys, int keys_in_smem) {
   extern __shared__ uint32_t sh[];
-  uint32_t *hist = sh;                  // [256]
-  uint32_t *wcnt = sh + 256;            // [2][kWarps]
-  uint32_t *scal = sh + 256 + 2 * kWarps;  // [8]
+  uint32_t *hist = sh;                           // [256]
+  uint32_t *whist = sh + 256;                    // [kWarps][256]
+  uint32_t *wcnt = whist + kWarps * 256;         // [2][kWarps] counts
+  uint32_t *woff = wcnt + 2 * kWarps;            // [2][kWarps] offsets
+  uint32_t *scal = woff + 2 * kWarps;            // [8]
   const int row = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   uint32_t *keys = keys_in_smem ? sh + kSmallWords : gkeys + static_cast<size_t>(row) * L;
@@ -62,11 +80,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t prefix = 0, mask = 0;
   long long krem = K;  // rank of the wanted key among those matching the prefix
   for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int b = tid; b < 256; b += kThreads) hist[b] = 0;
-    __syncthreads();
+    // per-warp histograms (atomics contend only inside a warp), then summed
+    uint32_t *mine = whist + warp * 256;
+    for (int b = lane; b < 256; b += 32) mine[b] = 0;
+    __syncwarp();
     for (long long j = tid; j < L; j += kThreads) {
       const uint32_t key = keys[j];
-      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+      if ((key & mask) == prefix) atomicAdd(&mine[(key >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    for (int b = tid; b < 256; b += kThreads) {
+      uint32_t sum = 0;
+#pragma unroll 8
+      for (int w = 0; w < kWarps; ++w) sum += whist[w * 256 + b];
+      hist[b] = sum;
     }
     __syncthreads();
     if (warp == 0) {
@@ -119,24 +146,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t eq_bal = __ballot_sync(0xffffffffu, eq);
     if (lane == 0) wcnt[warp] = __popc(eq_bal);
     __syncthreads();
-    uint32_t eq_before = 0, eq_total = 0;
-    for (int w = 0; w < kWarps; ++w) {
-      const uint32_t c = wcnt[w];
-      if (w < warp) eq_before += c;
-      eq_total += c;
-    }
-    eq_before += __popc(eq_bal & ((1u << lane) - 1u));
+    if (warp == 0) scan_warp_counts(wcnt, woff, &scal[4], lane);
+    __syncthreads();
+    const uint32_t eq_before = woff[warp] + __popc(eq_bal & ((1u << lane) - 1u));
+    const uint32_t eq_total = scal[4];
     const bool kept = gt || (eq && eq_so_far + eq_before < need_eq);
     const uint32_t k_bal = __ballot_sync(0xffffffffu, kept);
     if (lane == 0) wcnt[kWarps + warp] = __popc(k_bal);
     __syncthreads();
-    uint32_t k_before = 0, k_total = 0;
-    for (int w = 0; w < kWarps; ++w) {
-      const uint32_t c = wcnt[kWarps + w];
-      if (w < warp) k_before += c;
-      k_total += c;
-    }
-    k_before += __popc(k_bal & ((1u << lane) - 1u));
+    if (warp == 0) scan_warp_counts(wcnt + kWarps, woff + kWarps, &scal[5], lane);
+    __syncthreads();
+    const uint32_t k_before = woff[kWarps + warp] + __popc(k_bal & ((1u << lane) - 1u));
+    const uint32_t k_total = scal[5];
     if (kept) {
       const long long pos = kept_so_far + k_before;
       if (pos < K) out[pos] = static_cast<int32_t>(j);
