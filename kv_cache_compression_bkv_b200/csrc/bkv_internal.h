@@ -96,6 +96,10 @@ struct FpsGeom {
 };
 size_t fps_workspace_bytes(const FpsGeom &g);
 bool fps_supported(const FpsGeom &g);
+// fps_tc.cu: bf16, head_dim 128, the union of a query head in shared memory
+bool fps_tc_supported(const FpsGeom &g);
+bkv_status launch_fps_tc(const FpsGeom &g, const void *beacons_in, const void *window,
+                         void *beacons_out, cudaStream_t stream);
 bkv_status launch_fps(const FpsGeom &g, const void *beacons_in, const void *window,
                       void *beacons_out, void *ws, size_t ws_bytes, cudaStream_t stream);
 
@@ -116,5 +120,6 @@ bool ensure_smem_limit(Kernel kernel, int bytes, int *done_flags /* [64] */) {
 // ---- per-file device status accessors (bkv_device_status.cuh)
 int take_status_score_tc(cudaStream_t, int *);
 int take_status_select(cudaStream_t, int *);
+int take_status_fps_tc(cudaStream_t, int *);
 
 }  // namespace bkv

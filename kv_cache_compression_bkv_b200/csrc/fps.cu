@@ -50,6 +50,7 @@ struct Smem {
   float *pvec;       // [kCand][d] this round's picks (f32)
   float *gram;       // [kCand][kCand]
   uint32_t *hist;    // [256]
+  uint32_t *whist;   // [kWarps][256]
   int *cidx;         // [kCand + 1] candidates, then the bound
   float *cdist;      // [kCand + 1]
   int *pick;         // [kCand] candidate slots picked this round
@@ -111,85 +112,6 @@ __device__ void point_pass_dispatch(const Smem &s, const Points<T> &pt, int n, i
   }
 }
 
-// The `want` best unselected points in (distance desc, index asc) order, into
-// s.cidx / s.cdist (unordered).  Requires `want` <= number of unselected.
-__device__ void select_best(const Smem &s, int n, int want) {
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  uint32_t prefix = 0, mask = 0;
-  int krem = want;
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int b = tid; b < 256; b += kThreads) s.hist[b] = 0;
-    __syncthreads();
-    for (int i = tid; i < n; i += kThreads) {
-      const uint32_t key = dist_key(s.dist[i]);
-      if (key != 0u && (key & mask) == prefix) atomicAdd(&s.hist[(key >> shift) & 255u], 1u);
-    }
-    __syncthreads();
-    if (warp == 0) {
-      uint32_t cnt[8], local = 0;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        cnt[j] = s.hist[255 - 8 * lane - j];
-        local += cnt[j];
-      }
-      uint32_t incl = local;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const uint32_t o = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += o;
-      }
-      const uint32_t excl = incl - local;
-      if (static_cast<int>(excl) < krem && krem <= static_cast<int>(incl)) {
-        uint32_t acc = excl;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (static_cast<int>(acc + cnt[j]) >= krem) {
-            s.scal[0] = 255 - 8 * lane - j;
-            s.scal[1] = static_cast<int>(acc);
-            break;
-          }
-          acc += cnt[j];
-        }
-      }
-    }
-    __syncthreads();
-    prefix |= static_cast<uint32_t>(s.scal[0]) << shift;
-    mask |= 255u << shift;
-    krem -= s.scal[1];
-    __syncthreads();
-  }
-  // emit: every key above the threshold, and the lowest-index krem keys equal
-  // to it (an ordered scan only over the equal keys)
-  if (tid == 0) { s.scal[2] = 0; s.scal[3] = 0; }
-  __syncthreads();
-  int eq_base = 0;
-  for (int base = 0; base < n; base += kThreads) {
-    const int i = base + tid;
-    const uint32_t key = i < n ? dist_key(s.dist[i]) : 0u;
-    const bool gt = key > prefix;
-    const bool eq = key == prefix && key != 0u;
-    const uint32_t eb = __ballot_sync(0xffffffffu, eq);
-    if (lane == 0) s.hist[warp] = __popc(eb);
-    __syncthreads();
-    int before_me = 0, total = 0;
-    for (int w = 0; w < kWarps; ++w) {
-      const int c = static_cast<int>(s.hist[w]);
-      if (w < warp) before_me += c;
-      total += c;
-    }
-    before_me += __popc(eb & ((1u << lane) - 1u));
-    if (gt || (eq && eq_base + before_me < krem)) {
-      const int pos = atomicAdd(&s.scal[2], 1);
-      if (pos < want) {
-        s.cidx[pos] = i;
-        s.cdist[pos] = s.dist[i];
-      }
-    }
-    eq_base += total;
-    __syncthreads();
-  }
-}
-
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads, 1)
     fps_kernel(const FpsGeom g, const T *__restrict__ beacons_in, const T *__restrict__ window,
@@ -207,7 +129,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   s.dist = s.cdist + (kCand + 4);
   s.inv = s.dist + n;
   s.hist = reinterpret_cast<uint32_t *>(s.inv + n);
-  s.cidx = reinterpret_cast<int *>(s.hist + 256);
+  s.whist = s.hist + 256;
+  s.cidx = reinterpret_cast<int *>(s.whist + kWarps * 256);
   s.pick = s.cidx + (kCand + 4);
   s.scal = s.pick + kCand;
 
@@ -248,7 +171,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int unsel = n - picked;
     const int nc = min(kCand, unsel);           // candidates this round
     const bool bounded = unsel > kCand;         // a (kCand+1)-th point exists
-    select_best(s, n, bounded ? kCand + 1 : nc);
+    select_best<kThreads>(s.dist, n, bounded ? kCand + 1 : nc, s.whist, s.hist, s.scal, s.cidx,
+                          s.cdist);
     __syncthreads();
     // order the selected points: rank by (distance desc, index asc)
     const int want = bounded ? kCand + 1 : nc;
@@ -349,7 +273,7 @@ size_t fps_smem_bytes(const FpsGeom &g) {
   const size_t n = static_cast<size_t>(g.nb_in) + g.W;
   return sizeof(float) * (kCand * kCStride + kCand * kMaxDim + kCand * kCand + kCand + kCand +
                           4 + 2 * n) +
-         sizeof(uint32_t) * 256 + sizeof(int) * (kCand + 4 + kCand + 8);
+         sizeof(uint32_t) * (256 + kWarps * 256) + sizeof(int) * (kCand + 4 + kCand + 8);
 }
 
 template <typename T, int D>
@@ -379,15 +303,22 @@ bkv_status launch_dim(const FpsGeom &g, const void *bin, const void *win, void *
 
 size_t fps_workspace_bytes(const FpsGeom &) { return 0; }
 
-bool fps_supported(const FpsGeom &g) {
+namespace {
+bool fps_simt_supported(const FpsGeom &g) {
   return (g.head_dim == 32 || g.head_dim == 64 || g.head_dim == 96 || g.head_dim == 128) &&
          fps_smem_bytes(g) <= static_cast<size_t>(kSmemLimit);
 }
+}  // namespace
 
+bool fps_supported(const FpsGeom &g) { return fps_tc_supported(g) || fps_simt_supported(g); }
+
+// bf16 unions that fit in shared memory take the tensor-core kernel
+// (fps_tc.cu); f32 inputs and larger unions take the CUDA-core kernel above.
 bkv_status launch_fps(const FpsGeom &g, const void *beacons_in, const void *window,
                       void *beacons_out, void *, size_t, cudaStream_t stream) {
-  if (!fps_supported(g)) return BKV_ERR_UNSUPPORTED;
   if (g.n_pick <= 0) return BKV_OK;
+  if (fps_tc_supported(g)) return launch_fps_tc(g, beacons_in, window, beacons_out, stream);
+  if (!fps_simt_supported(g)) return BKV_ERR_UNSUPPORTED;
   if (g.dtype == BKV_BF16)
     return launch_dim<__nv_bfloat16>(g, beacons_in, window, beacons_out, stream);
   return launch_dim<float>(g, beacons_in, window, beacons_out, stream);

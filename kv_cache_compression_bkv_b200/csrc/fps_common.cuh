@@ -54,5 +54,132 @@ __device__ __forceinline__ bool before(float da, int ia, float db, int ib) {
   return da > db || (da == db && ia < ib);
 }
 
+
+// The `want` best unselected points by (distance desc, index asc), written
+// unordered to cidx/cdist (want <= number of unselected points).  An MSB-first
+// radix select over the distance keys: a min/max reduction first finds the
+// leading bits that every key shares, so the histogram passes start at the
+// first bit that differs (distances of one head tend to share their exponent,
+// which would otherwise pile every key into one or two bins); each warp counts
+// into its own histogram.  Then every key above the threshold and the
+// lowest-index keys equal to it are emitted.
+// Scratch: whist[kThreads / 32 * 256], hist[256], scal[>= 8].
+template <int kThreads>
+__device__ void select_best(const float *dist, int n, int want, uint32_t *whist, uint32_t *hist,
+                            int *scal, int *cidx, float *cdist) {
+  constexpr int kWarps = kThreads / 32;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // common prefix of the live keys
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
+  for (int i = tid; i < n; i += kThreads) {
+    const uint32_t key = dist_key(dist[i]);
+    if (key != 0u) {
+      kmin = min(kmin, key);
+      kmax = max(kmax, key);
+    }
+  }
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  if (lane == 0) {
+    hist[2 * warp] = kmin;
+    hist[2 * warp + 1] = kmax;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    uint32_t a = 0xffffffffu, b = 0u;
+    for (int w = 0; w < kWarps; ++w) {
+      a = min(a, hist[2 * w]);
+      b = max(b, hist[2 * w + 1]);
+    }
+    scal[6] = static_cast<int>(a);
+    scal[7] = static_cast<int>(b);
+  }
+  __syncthreads();
+  const uint32_t gmin = static_cast<uint32_t>(scal[7]) == 0u ? 0u : static_cast<uint32_t>(scal[6]);
+  const uint32_t diff = gmin ^ static_cast<uint32_t>(scal[7]);
+  int hi = diff == 0u ? 0 : 32 - __clz(diff);  // bits [hi, 32) are shared
+  uint32_t mask = hi >= 32 ? 0u : ~((1u << hi) - 1u);
+  uint32_t prefix = gmin & mask;
+  int krem = want;
+  for (; hi > 0; hi -= 8) {
+    const int lo = hi > 8 ? hi - 8 : 0;
+    uint32_t *mine = whist + warp * 256;
+    for (int b = lane; b < 256; b += 32) mine[b] = 0;
+    __syncwarp();
+    for (int i = tid; i < n; i += kThreads) {
+      const uint32_t key = dist_key(dist[i]);
+      if (key != 0u && (key & mask) == prefix) atomicAdd(&mine[(key >> lo) & 255u], 1u);
+    }
+    __syncthreads();
+    for (int b = tid; b < 256; b += kThreads) {
+      uint32_t sum = 0;
+      for (int w = 0; w < kWarps; ++w) sum += whist[w * 256 + b];
+      hist[b] = sum;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      uint32_t cnt[8], local = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        cnt[j] = hist[255 - 8 * lane - j];
+        local += cnt[j];
+      }
+      uint32_t incl = local;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+      }
+      const uint32_t excl = incl - local;
+      if (static_cast<int>(excl) < krem && krem <= static_cast<int>(incl)) {
+        uint32_t acc = excl;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (static_cast<int>(acc + cnt[j]) >= krem) {
+            scal[0] = 255 - 8 * lane - j;
+            scal[1] = static_cast<int>(acc);
+            break;
+          }
+          acc += cnt[j];
+        }
+      }
+    }
+    __syncthreads();
+    prefix |= static_cast<uint32_t>(scal[0]) << lo;
+    mask |= ((hi - lo) >= 32 ? 0xffffffffu : ((1u << (hi - lo)) - 1u)) << lo;
+    krem -= scal[1];
+    __syncthreads();
+  }
+  // emission: keys above the threshold, and the lowest-index krem keys equal
+  if (tid == 0) scal[2] = 0;
+  __syncthreads();
+  int eq_base = 0;
+  for (int base = 0; base < n; base += kThreads) {
+    const int i = base + tid;
+    const uint32_t key = i < n ? dist_key(dist[i]) : 0u;
+    const bool gt = key > prefix;
+    const bool eq = key == prefix && key != 0u;
+    const uint32_t eb = __ballot_sync(0xffffffffu, eq);
+    if (lane == 0) hist[warp] = __popc(eb);
+    __syncthreads();
+    int before_me = 0, total = 0;
+    for (int w = 0; w < kWarps; ++w) {
+      const int c = static_cast<int>(hist[w]);
+      if (w < warp) before_me += c;
+      total += c;
+    }
+    before_me += __popc(eb & ((1u << lane) - 1u));
+    if (gt || (eq && eq_base + before_me < krem)) {
+      const int pos = atomicAdd(&scal[2], 1);
+      if (pos < want) {
+        cidx[pos] = i;
+        cdist[pos] = dist[i];
+      }
+    }
+    eq_base += total;
+    __syncthreads();
+  }
+}
+
 }  // namespace fpsk
 }  // namespace bkv

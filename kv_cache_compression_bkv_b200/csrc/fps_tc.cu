@@ -1,0 +1,450 @@
+// fps_tc.cu -- Continual farthest-point sampling (BeaconKV, Fig. 7) of bf16
+// queries with head_dim 128, the distance pass of every round on tcgen05.
+//
+// Same exact speculative rounds as fps.cu (select the T+1 best unselected
+// points; Gram block of the T candidates; replay the greedy choice among
+// them while the best one provably beats every other point; lower all
+// distances by the round's picks), with T = 64 and a different distance pass:
+// the union [beacons; window] of a query head is streamed by TMA in tiles of
+// 128 points (128-byte swizzle, no multicast) into a 3-stage ring, one thread
+// issues D[128 points][N] = tile . picks^T (M=128, N = picks rounded up to 16,
+// K = 128) into a double-buffered TMEM accumulator, and four epilogue warps
+// (TMEM lane = point) turn the dot products into cosine distances and lower
+// the shared-memory distance array.  The candidates' Gram block is formed on
+// the CUDA cores in f32; bf16 products are exact in f32 on either path, the
+// two sums may differ in their last bit, which can only reorder picks whose
+// distances agree to about 1e-7.
+//
+// The grid is persistent: one CTA per SM loops over the query heads.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+
+#include "bkv_internal.h"
+#include "fps_common.cuh"
+#include "sm100.cuh"
+#include "tma_host.h"
+
+BKV_DEFINE_STATUS_ACCESSOR(take_status_fps_tc)
+
+namespace bkv {
+namespace {
+
+using namespace sm100;
+using namespace fpsk;
+
+constexpr int kThreads = 256;  // warp 0 TMA, warp 1 MMA, warps 4..7 distance epilogue
+constexpr int kWarps = kThreads / 32;
+constexpr int kCand = 64;      // candidates per round (T)
+constexpr int kDim = 128;
+constexpr int kTileRows = 128;
+constexpr int kStages = 3;
+constexpr int kTileBytes = kTileRows * kDim * 2;  // 32 KB
+constexpr int kBBlock = kCand * 128;              // one 64-element K block of the picks
+constexpr int kBBytes = 2 * kBBlock;              // 16 KB
+constexpr int kCStride = kDim + 4;
+constexpr int kSmallBytes = 4096;
+constexpr int kFixedBytes = kSmallBytes + 1024 + kStages * kTileBytes + kBBytes +
+                            kCand * kCStride * 4 + kCand * kCand * 4 + kWarps * 256 * 4;
+constexpr int kSmemLimit = 232448;
+constexpr uint32_t kTmemCols = 128;  // two accumulators of up to 64 columns
+constexpr int kAbort = 15;           // index of the abort flag in scal[]
+
+enum { kWhereProd = 401, kWhereMma = 402, kWhereEpi = 403, kWhereDrain = 404 };
+
+struct Layout {
+  uint64_t *bars;   // full[3] empty[3] tfull[2] tempty[2] done
+  uint32_t *tmem_slot;
+  int *scal;        // [16]
+  uint32_t *hist;   // [256]
+  int *cidx;        // [kCand + 1]
+  float *cdist;     // [kCand + 1]
+  int *pick;        // [kCand]
+  float *pinv;      // [kCand]
+  uint8_t *stages;  // [kStages][kTileBytes]
+  uint8_t *bop;     // picks, K-major 128-byte swizzle: [2][kCand rows][128 B]
+  float *cvec;      // [kCand][kCStride]
+  float *gram;      // [kCand][kCand]
+  uint32_t *whist;  // [kWarps][256] per-warp histograms of the selection
+  float *dist;      // [n]
+  float *inv;       // [n]
+};
+
+struct Head {
+  const __nv_bfloat16 *B, *Wp;
+  int nb, W;
+  __device__ const __nv_bfloat16 *point(int i) const {
+    return i < nb ? B + static_cast<size_t>(i) * kDim : Wp + static_cast<size_t>(i - nb) * kDim;
+  }
+};
+
+// One distance pass over every tile of the head: producer (warp 0), MMA
+// issuer (warp 1) and epilogue (warps 4..7) run their own loops; `seq` is the
+// number of tiles all passes so far have moved through the ring, so every
+// role derives the same stage and phase for each tile.
+__device__ void distance_pass(const Layout &s, const CUtensorMap *bmap, const CUtensorMap *wmap,
+                              uint32_t tmem, int qh, const FpsGeom &g, int n_btiles, int n_tiles,
+                              uint32_t seq, int np, bool first) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t full0 = smem_u32(&s.bars[0]), empty0 = smem_u32(&s.bars[3]);
+  const uint32_t tfull0 = smem_u32(&s.bars[6]), tempty0 = smem_u32(&s.bars[8]);
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int j = 0; j < n_tiles; ++j) {
+        const uint32_t q = seq + j, st = q % kStages;
+        if (!mbar_wait(empty0 + 8 * st, ((q / kStages) & 1) ^ 1, kWhereProd)) {
+          s.scal[kAbort] = 1;
+          break;
+        }
+        mbar_arrive_expect_tx(full0 + 8 * st, kTileBytes);
+        const uint32_t dst = smem_u32(s.stages + st * kTileBytes);
+        const CUtensorMap *map = j < n_btiles ? bmap : wmap;
+        const int y = j < n_btiles ? qh * g.M + j * kTileRows
+                                   : qh * g.W + (j - n_btiles) * kTileRows;
+        tma_load_2d(dst, map, full0 + 8 * st, 0, y);
+        tma_load_2d(dst + kTileRows * 128, map, full0 + 8 * st, 64, y);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const int npad = (np + 15) & ~15;
+      const uint32_t idesc = idesc_bf16_f32(kTileRows, npad);
+      const uint32_t b_base = smem_u32(s.bop);
+      for (int j = 0; j < n_tiles; ++j) {
+        const uint32_t q = seq + j, st = q % kStages, a = q & 1;
+        if (!mbar_wait(full0 + 8 * st, (q / kStages) & 1, kWhereMma) ||
+            !mbar_wait(tempty0 + 8 * a, ((q >> 1) & 1) ^ 1, kWhereMma)) {
+          s.scal[kAbort] = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a_base = smem_u32(s.stages + st * kTileBytes);
+#pragma unroll
+        for (int kb = 0; kb < 2; ++kb) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = smem_desc_k_sw128(a_base + kb * (kTileRows * 128) + kk * 32);
+            const uint64_t bd = smem_desc_k_sw128(b_base + kb * kBBlock + kk * 32);
+            umma_f16(tmem + a * 64, ad, bd, idesc, (kb | kk) != 0);
+          }
+        }
+        umma_commit(empty0 + 8 * st);
+        umma_commit(tfull0 + 8 * a);
+      }
+    }
+  } else if (warp >= 4) {
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    for (int j = 0; j < n_tiles; ++j) {
+      const uint32_t q = seq + j, a = q & 1;
+      if (!mbar_wait(tfull0 + 8 * a, (q >> 1) & 1, kWhereEpi)) {
+        s.scal[kAbort] = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + a * 64;
+      float v0[32], v1[32];
+      tmem_ld_32x32b_x32(taddr, v0);
+      if (np > 32) tmem_ld_32x32b_x32(taddr + 32, v1);
+      tmem_ld_wait_regs(v0);
+      tmem_reg_fence(v1);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty0 + 8 * a);
+      int i;
+      bool valid;
+      if (j < n_btiles) {
+        i = j * kTileRows + r;
+        valid = i < g.nb_in;
+      } else {
+        const int w = (j - n_btiles) * kTileRows + r;
+        i = g.nb_in + w;
+        valid = w < g.W;
+      }
+      if (!valid) continue;
+      float di = first ? 0.f : s.dist[i];
+      if (!first && di < 0.f) continue;  // already selected
+      const float inv_i = s.inv[i];
+#pragma unroll
+      for (int k = 0; k < 64; ++k) {
+        if (k < np) {
+          const float dot = k < 32 ? v0[k] : v1[k - 32];
+          const float dd = cos_dist(make_float2(dot, 0.f), inv_i, s.pinv[k]);
+          di = (first && k == 0) ? dd : fminf(di, dd);
+        }
+      }
+      s.dist[i] = di;
+    }
+  }
+}
+
+// The picks of this round into the B operand (rows padded with zeros to a
+// multiple of 16) and the output beacons.
+__device__ void stage_picks(const Layout &s, const Head &h, __nv_bfloat16 *out, int picked,
+                            int np) {
+  const int npad = (np + 15) & ~15;
+  for (int e = threadIdx.x; e < npad * 16; e += kThreads) {
+    const int k = e >> 4, c16 = e & 15, kb = c16 >> 3, c = c16 & 7;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (k < np) {
+      const __nv_bfloat16 *src = h.point(s.cidx[s.pick[k]]) + c16 * 8;
+      v = *reinterpret_cast<const uint4 *>(src);
+      *reinterpret_cast<uint4 *>(out + static_cast<size_t>(picked + k) * kDim + c16 * 8) = v;
+    }
+    *reinterpret_cast<uint4 *>(s.bop + kb * kBBlock + sw128_offset(k, c)) = v;
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    fps_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__ CUtensorMap wmap,
+                  const FpsGeom g, const __nv_bfloat16 *__restrict__ beacons_in,
+                  const __nv_bfloat16 *__restrict__ window, __nv_bfloat16 *__restrict__ beacons_out,
+                  int n_qheads) {
+  extern __shared__ uint8_t smem_raw[];
+  const int n = g.nb_in + g.W;
+  const int m = g.n_pick;
+  Layout s;
+  s.bars = reinterpret_cast<uint64_t *>(smem_raw);
+  s.tmem_slot = reinterpret_cast<uint32_t *>(smem_raw + 128);
+  s.scal = reinterpret_cast<int *>(smem_raw + 192);
+  s.hist = reinterpret_cast<uint32_t *>(smem_raw + 256);
+  s.cidx = reinterpret_cast<int *>(smem_raw + 1280);
+  s.cdist = reinterpret_cast<float *>(smem_raw + 1552);
+  s.pick = reinterpret_cast<int *>(smem_raw + 1824);
+  s.pinv = reinterpret_cast<float *>(smem_raw + 2096);
+  const uint32_t raw_base = smem_u32(smem_raw);
+  const uint32_t big = (raw_base + kSmallBytes + 1023u) & ~1023u;
+  s.stages = smem_raw + (big - raw_base);
+  s.bop = s.stages + kStages * kTileBytes;
+  s.cvec = reinterpret_cast<float *>(s.bop + kBBytes);
+  s.gram = s.cvec + kCand * kCStride;
+  s.whist = reinterpret_cast<uint32_t *>(s.gram + kCand * kCand);
+  s.dist = reinterpret_cast<float *>(s.whist + kWarps * 256);
+  s.inv = s.dist + n;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n_btiles = (g.nb_in + kTileRows - 1) / kTileRows;
+  const int n_tiles = n_btiles + (g.W + kTileRows - 1) / kTileRows;
+  if (tid == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(smem_u32(&s.bars[i]), 1);
+      mbar_init(smem_u32(&s.bars[3 + i]), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(smem_u32(&s.bars[6 + a]), 1);
+      mbar_init(smem_u32(&s.bars[8 + a]), 4);  // one arrive per epilogue warp
+    }
+    mbar_init(smem_u32(&s.bars[10]), 1);
+    fence_barrier_init();
+    prefetch_tensormap(&bmap);
+    prefetch_tensormap(&wmap);
+    s.scal[kAbort] = 0;
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(s.tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s.tmem_slot;
+  uint32_t seq = 0;
+
+  for (int qh = blockIdx.x; qh < n_qheads; qh += gridDim.x) {
+    Head h{beacons_in + static_cast<size_t>(qh) * g.M * kDim,
+           window + static_cast<size_t>(qh) * g.W * kDim, g.nb_in, g.W};
+    __nv_bfloat16 *out = beacons_out + static_cast<size_t>(qh) * g.M * kDim;
+    // inverse norms (0 for a zero vector, which makes its distance 1)
+    for (int i = tid; i < n; i += kThreads) {
+      const __nv_bfloat16 *p = h.point(i);
+      float ss = 0.f;
+#pragma unroll
+      for (int t = 0; t < kDim; t += 8) {
+        float u[8];
+        load8(p + t, u);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) ss = fmaf(u[j], u[j], ss);
+      }
+      s.inv[i] = ss > 0.f ? 1.0f / sqrtf(ss) : 0.f;
+    }
+    if (tid == 0) {
+      s.cidx[0] = 0;  // the seed U[0] is the first pick
+      s.pick[0] = 0;
+    }
+    __syncthreads();
+    if (tid == 0) s.pinv[0] = s.inv[0];
+    stage_picks(s, h, out, 0, 1);
+    fence_proxy_async_smem();
+    __syncthreads();
+    distance_pass(s, &bmap, &wmap, tmem, qh, g, n_btiles, n_tiles, seq, 1, true);
+    seq += n_tiles;
+    __syncthreads();
+    if (s.scal[kAbort]) break;
+    if (tid == 0) s.dist[0] = -1.f;
+    __syncthreads();
+
+    int picked = 1;
+    while (picked < m) {
+      const int unsel = n - picked;
+      const int nc = min(kCand, unsel);
+      const bool bounded = unsel > kCand;
+      const int want = bounded ? kCand + 1 : nc;
+      select_best<kThreads>(s.dist, n, want, s.whist, s.hist, s.scal, s.cidx, s.cdist);
+      __syncthreads();
+      int my_i = 0, my_rank = 0;
+      float my_d = 0.f;
+      if (tid < want) {
+        my_i = s.cidx[tid];
+        my_d = s.cdist[tid];
+        for (int j = 0; j < want; ++j)
+          if (j != tid && before(s.cdist[j], s.cidx[j], my_d, my_i)) ++my_rank;
+      }
+      __syncthreads();
+      if (tid < want) {
+        s.cidx[my_rank] = my_i;
+        s.cdist[my_rank] = my_d;
+      }
+      __syncthreads();
+      for (int e = tid; e < nc * (kDim / 8); e += kThreads) {
+        const int a = e >> 4, t = (e & 15) * 8;
+        float u[8];
+        load8(h.point(s.cidx[a]) + t, u);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) s.cvec[a * kCStride + t + j] = u[j];
+      }
+      __syncthreads();
+      // Gram block: lanes take consecutive candidates a of one pick b
+      for (int e = tid; e < nc * nc; e += kThreads) {
+        const int b = e / nc, a = e - b * nc;
+        float2 acc = make_float2(0.f, 0.f);
+#pragma unroll 4
+        for (int t = 0; t < kDim; t += 8) {
+          float u[8];
+          load8(s.cvec + a * kCStride + t, u);
+          acc = dot8_step(acc, u, s.cvec + b * kCStride + t);
+        }
+        s.gram[a * kCand + b] = __fadd_rn(acc.x, acc.y);
+      }
+      __syncthreads();
+      // replay the greedy choice among the candidates (warp 0, two per lane)
+      if (warp == 0) {
+        const int a0 = lane, a1 = lane + 32;
+        bool t0 = a0 >= nc, t1 = a1 >= nc;  // taken or absent
+        float c0 = t0 ? -3.f : s.cdist[a0], c1 = t1 ? -3.f : s.cdist[a1];
+        const int i0 = t0 ? 0x7fffffff : s.cidx[a0], i1 = t1 ? 0x7fffffff : s.cidx[a1];
+        const float inv0 = t0 ? 0.f : s.inv[i0], inv1 = t1 ? 0.f : s.inv[i1];
+        const float bd = bounded ? s.cdist[kCand] : -3.f;
+        const int bi = bounded ? s.cidx[kCand] : 0x7fffffff;
+        int np = 0;
+        while (picked + np < m) {
+          float best_d = t0 ? -3.f : c0;
+          int best_i = t0 ? 0x7fffffff : i0, best_a = a0;
+          if (!t1 && before(c1, i1, best_d, best_i)) {
+            best_d = c1;
+            best_i = i1;
+            best_a = a1;
+          }
+          for (int off = 16; off > 0; off >>= 1) {
+            const float od = __shfl_xor_sync(0xffffffffu, best_d, off);
+            const int oi = __shfl_xor_sync(0xffffffffu, best_i, off);
+            const int oa = __shfl_xor_sync(0xffffffffu, best_a, off);
+            if (before(od, oi, best_d, best_i)) {
+              best_d = od;
+              best_i = oi;
+              best_a = oa;
+            }
+          }
+          if (best_d < 0.f) break;
+          if (bounded && !before(best_d, best_i, bd, bi)) break;
+          if (lane == 0) s.pick[np] = best_a;
+          ++np;
+          if (best_a == a0) t0 = true;
+          if (best_a == a1) t1 = true;
+          const float inv_b = s.inv[best_i];
+          if (!t0) c0 = fminf(c0, cos_dist(make_float2(s.gram[a0 * kCand + best_a], 0.f), inv0, inv_b));
+          if (!t1) c1 = fminf(c1, cos_dist(make_float2(s.gram[a1 * kCand + best_a], 0.f), inv1, inv_b));
+        }
+        if (lane == 0) s.scal[4] = np;
+      }
+      __syncthreads();
+      const int np = s.scal[4];
+      if (tid < np) s.pinv[tid] = s.inv[s.cidx[s.pick[tid]]];
+      stage_picks(s, h, out, picked, np);
+      __syncthreads();
+      if (tid < np) s.dist[s.cidx[s.pick[tid]]] = -1.f;
+      fence_proxy_async_smem();
+      __syncthreads();
+      distance_pass(s, &bmap, &wmap, tmem, qh, g, n_btiles, n_tiles, seq, np, false);
+      seq += n_tiles;
+      __syncthreads();
+      if (s.scal[kAbort]) break;
+      picked += np;
+    }
+    if (s.scal[kAbort]) break;
+  }
+
+  // drain: every TMA load and MMA issued by this CTA has completed before the
+  // CTA exits and frees its TMEM
+  if (warp == 0 && lane == 0 && seq > 0) {
+    const uint32_t first = seq > kStages ? seq - kStages : 0;
+    for (uint32_t q = first; q < seq; ++q)
+      mbar_wait(smem_u32(&s.bars[q % kStages]), (q / kStages) & 1, kWhereDrain);
+  }
+  if (warp == 1 && lane == 0) {
+    umma_commit(smem_u32(&s.bars[10]));
+    mbar_wait(smem_u32(&s.bars[10]), 0, kWhereDrain);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace
+
+size_t fps_tc_smem_bytes(const FpsGeom &g) {
+  return static_cast<size_t>(kFixedBytes) + 8 * (static_cast<size_t>(g.nb_in) + g.W);
+}
+
+bool fps_tc_supported(const FpsGeom &g) {
+  return g.dtype == BKV_BF16 && g.head_dim == kDim &&
+         fps_tc_smem_bytes(g) <= static_cast<size_t>(kSmemLimit) &&
+         static_cast<long long>(g.n_layers) * g.n_q_heads * std::max(g.M, g.W) < (1LL << 31) - 256;
+}
+
+bkv_status launch_fps_tc(const FpsGeom &g, const void *beacons_in, const void *window,
+                         void *beacons_out, cudaStream_t stream) {
+  const int n_qheads = g.n_layers * g.n_q_heads;
+  // Tensor maps over every head's beacon slots and window rows.  A map needs
+  // a non-empty tensor: an absent part (no beacons, or no window) points at
+  // the other one and is never read.
+  const void *bsrc = g.nb_in > 0 ? beacons_in : window;
+  const void *wsrc = g.W > 0 ? window : beacons_in;
+  const unsigned long long brows =
+      static_cast<unsigned long long>(n_qheads) * static_cast<unsigned long long>(g.nb_in > 0 ? g.M : g.W);
+  const unsigned long long wrows =
+      static_cast<unsigned long long>(n_qheads) * static_cast<unsigned long long>(g.W > 0 ? g.W : g.M);
+  CUtensorMap bmap, wmap;
+  if (!make_bf16_rows_map(&bmap, bsrc, brows, kTileRows) ||
+      !make_bf16_rows_map(&wmap, wsrc, wrows, kTileRows))
+    return BKV_ERR_CUDA;
+  static int attr_done[64];
+  const int smem = static_cast<int>(fps_tc_smem_bytes(g));
+  if (!ensure_smem_limit(fps_tc_kernel, kSmemLimit, attr_done)) return BKV_ERR_CUDA;
+  int sms = 148, dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = std::max(1, std::min(n_qheads, sms));
+  fps_tc_kernel<<<grid, kThreads, smem, stream>>>(
+      bmap, wmap, g, static_cast<const __nv_bfloat16 *>(beacons_in),
+      static_cast<const __nv_bfloat16 *>(window), static_cast<__nv_bfloat16 *>(beacons_out),
+      n_qheads);
+  return cudaGetLastError() == cudaSuccess ? BKV_OK : BKV_ERR_CUDA;
+}
+
+}  // namespace bkv

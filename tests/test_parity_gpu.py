@@ -102,6 +102,11 @@ FPS_CASES = {
     "no_beacons": lambda: small(W=40, M=16, n_beacons_in=0),
     "window_lt_M": lambda: small(W=5, M=16, n_beacons_in=4),
     "window_only_one": lambda: small(W=1, M=4, n_beacons_in=0, R=1),
+    "ragged_tiles": lambda: small(W=333, M=40, n_beacons_in=37),
+    "many_rounds": lambda: small(n_q_heads=2, n_kv_heads=1, W=1200, M=128, n_beacons_in=100),
+    # a union too large for the shared-memory distance array of the
+    # tensor-core kernel: the CUDA-core kernel handles it
+    "large_union": lambda: small(n_q_heads=2, n_kv_heads=1, W=9000, M=32, n_beacons_in=32),
 }
 
 
