@@ -171,8 +171,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int unsel = n - picked;
     const int nc = min(kCand, unsel);           // candidates this round
     const bool bounded = unsel > kCand;         // a (kCand+1)-th point exists
-    select_best<kThreads>(s.dist, n, bounded ? kCand + 1 : nc, s.whist, s.hist, s.scal, s.cidx,
-                          s.cdist);
+    select_best<kThreads>(s.dist, n, unsel, bounded ? kCand + 1 : nc, s.whist, s.hist, s.scal,
+                          s.cidx, s.cdist);
     __syncthreads();
     // order the selected points: rank by (distance desc, index asc)
     const int want = bounded ? kCand + 1 : nc;

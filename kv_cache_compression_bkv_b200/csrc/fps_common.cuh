@@ -65,8 +65,8 @@ __device__ __forceinline__ bool before(float da, int ia, float db, int ib) {
 // lowest-index keys equal to it are emitted.
 // Scratch: whist[kThreads / 32 * 256], hist[256], scal[>= 8].
 template <int kThreads>
-__device__ void select_best(const float *dist, int n, int want, uint32_t *whist, uint32_t *hist,
-                            int *scal, int *cidx, float *cdist) {
+__device__ void select_best(const float *dist, int n, int n_live, int want, uint32_t *whist,
+                            uint32_t *hist, int *scal, int *cidx, float *cdist) {
   constexpr int kWarps = kThreads / 32;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // common prefix of the live keys
@@ -101,6 +101,7 @@ __device__ void select_best(const float *dist, int n, int want, uint32_t *whist,
   uint32_t mask = hi >= 32 ? 0u : ~((1u << hi) - 1u);
   uint32_t prefix = gmin & mask;
   int krem = want;
+  int n_eq = n_live;  // live keys matching the prefix
   for (; hi > 0; hi -= 8) {
     const int lo = hi > 8 ? hi - 8 : 0;
     uint32_t *mine = whist + warp * 256;
@@ -148,11 +149,34 @@ __device__ void select_best(const float *dist, int n, int want, uint32_t *whist,
     prefix |= static_cast<uint32_t>(scal[0]) << lo;
     mask |= ((hi - lo) >= 32 ? 0xffffffffu : ((1u << (hi - lo)) - 1u)) << lo;
     krem -= scal[1];
+    n_eq = static_cast<int>(hist[scal[0]]);
     __syncthreads();
   }
-  // emission: keys above the threshold, and the lowest-index krem keys equal
   if (tid == 0) scal[2] = 0;
   __syncthreads();
+  if (n_eq == krem) {
+    // every key equal to the threshold is kept: the selection is the keys
+    // >= threshold, emitted in any order (one atomic per warp)
+    for (int base = 0; base < n; base += kThreads) {
+      const int i = base + tid;
+      const uint32_t key = i < n ? dist_key(dist[i]) : 0u;
+      const bool keep = key != 0u && key >= prefix;
+      const uint32_t bal = __ballot_sync(0xffffffffu, keep);
+      int wbase = 0;
+      if (lane == 0 && bal) wbase = atomicAdd(&scal[2], __popc(bal));
+      wbase = __shfl_sync(0xffffffffu, wbase, 0);
+      if (keep) {
+        const int pos = wbase + __popc(bal & ((1u << lane) - 1u));
+        if (pos < want) {
+          cidx[pos] = i;
+          cdist[pos] = dist[i];
+        }
+      }
+    }
+    return;
+  }
+  // emission: keys above the threshold, and the lowest-index krem keys equal
+  // to it in index order
   int eq_base = 0;
   for (int base = 0; base < n; base += kThreads) {
     const int i = base + tid;

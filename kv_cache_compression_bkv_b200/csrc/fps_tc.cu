@@ -35,7 +35,7 @@ namespace {
 using namespace sm100;
 using namespace fpsk;
 
-constexpr int kThreads = 256;  // warp 0 TMA, warp 1 MMA, warps 4..7 distance epilogue
+constexpr int kThreads = 384;  // warp 0 TMA, warp 1 MMA, warps 4..11 distance epilogue
 constexpr int kWarps = kThreads / 32;
 constexpr int kCand = 64;      // candidates per round (T)
 constexpr int kDim = 128;
@@ -79,6 +79,10 @@ struct Head {
     return i < nb ? B + static_cast<size_t>(i) * kDim : Wp + static_cast<size_t>(i - nb) * kDim;
   }
 };
+
+__device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
 
 // One distance pass over every tile of the head: producer (warp 0), MMA
 // issuer (warp 1) and epilogue (warps 4..7) run their own loops; `seq` is the
@@ -135,24 +139,31 @@ __device__ void distance_pass(const Layout &s, const CUtensorMap *bmap, const CU
       }
     }
   } else if (warp >= 4) {
+    // epilogue warpgroup w consumes accumulator w, i.e. every other tile
+    const int wg = (warp - 4) >> 2;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
+    const int npad = (np + 15) & ~15;
+    bool ok = true;  // warp-uniform; after a timeout the warp keeps only the barriers
     for (int j = 0; j < n_tiles; ++j) {
       const uint32_t q = seq + j, a = q & 1;
-      if (!mbar_wait(tfull0 + 8 * a, (q >> 1) & 1, kWhereEpi)) {
+      if (static_cast<int>(a) != wg) continue;
+      if (ok && !mbar_wait_warp(tfull0 + 8 * a, (q >> 1) & 1, kWhereEpi)) {
         s.scal[kAbort] = 1;
-        break;
+        ok = false;
       }
-      tc_fence_after();
-      const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + a * 64;
       float v0[32], v1[32];
-      tmem_ld_32x32b_x32(taddr, v0);
-      if (np > 32) tmem_ld_32x32b_x32(taddr + 32, v1);
-      tmem_ld_wait_regs(v0);
-      tmem_reg_fence(v1);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(tempty0 + 8 * a);
+      if (ok) {
+        tc_fence_after();
+        const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + a * 64;
+        tmem_ld_32x32b_x32(taddr, v0);
+        if (npad > 32) tmem_ld_32x32b_x32(taddr + 32, v1);
+        tmem_ld_wait_regs(v0);
+        tmem_reg_fence(v1);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tempty0 + 8 * a);
+      }
       int i;
       bool valid;
       if (j < n_btiles) {
@@ -163,19 +174,66 @@ __device__ void distance_pass(const Layout &s, const CUtensorMap *bmap, const CU
         i = g.nb_in + w;
         valid = w < g.W;
       }
-      if (!valid) continue;
-      float di = first ? 0.f : s.dist[i];
-      if (!first && di < 0.f) continue;  // already selected
-      const float inv_i = s.inv[i];
+      const uint32_t st = q % kStages;
+      if (first) {
+        // the seed pass also takes every point's inverse norm from its row of
+        // the staged tile (0 for a zero vector, whose distance is then 1)
+        if (ok && !mbar_wait_warp(full0 + 8 * st, (q / kStages) & 1, kWhereEpi)) {
+          s.scal[kAbort] = 1;
+          ok = false;
+        }
+        if (ok) {
+          const uint8_t *row = s.stages + st * kTileBytes;
+          float ss = 0.f;
 #pragma unroll
-      for (int k = 0; k < 64; ++k) {
-        if (k < np) {
-          const float dot = k < 32 ? v0[k] : v1[k - 32];
-          const float dd = cos_dist(make_float2(dot, 0.f), inv_i, s.pinv[k]);
-          di = (first && k == 0) ? dd : fminf(di, dd);
+          for (int c16 = 0; c16 < 16; ++c16) {
+            float u[8];
+            load8(reinterpret_cast<const __nv_bfloat16 *>(
+                      row + (c16 >> 3) * (kTileRows * 128) + sw128_offset(r, c16 & 7)),
+                  u);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) ss = fmaf(u[e], u[e], ss);
+          }
+          if (valid) s.inv[i] = ss > 0.f ? 1.0f / sqrtf(ss) : 0.f;
+        }
+        named_barrier_sync(2 + wg, 128);
+      }
+      if (ok && warp == 4 + 4 * wg && lane == 0) mbar_arrive(empty0 + 8 * st);
+      if (!ok) continue;
+      if (!valid) continue;
+      float di = first ? 2.f : s.dist[i];
+      if (di < 0.f) continue;  // already selected
+      // x_k = 1 - dot_k * inv_i * inv_k, as cos_dist computes it; padded
+      // picks carry a NaN inverse norm, which min ignores
+      const float inv_i = s.inv[i];
+      const float2 ninv = make_float2(-inv_i, -inv_i);
+      float mn = INFINITY;
+#pragma unroll
+      for (int k = 0; k < 32; k += 4) {
+        if (k < npad) {
+          const float4 pv = *reinterpret_cast<const float4 *>(s.pinv + k);
+          const float2 x0 = __ffma2_rn(__fmul2_rn(make_float2(v0[k], v0[k + 1]), ninv),
+                                       make_float2(pv.x, pv.y), make_float2(1.f, 1.f));
+          const float2 x1 = __ffma2_rn(__fmul2_rn(make_float2(v0[k + 2], v0[k + 3]), ninv),
+                                       make_float2(pv.z, pv.w), make_float2(1.f, 1.f));
+          mn = fminf(mn, fminf(fminf(x0.x, x0.y), fminf(x1.x, x1.y)));
         }
       }
-      s.dist[i] = di;
+      if (npad > 32) {
+#pragma unroll
+        for (int k = 0; k < 32; k += 4) {
+          if (k + 32 < npad) {
+            const float4 pv = *reinterpret_cast<const float4 *>(s.pinv + 32 + k);
+            const float2 x0 = __ffma2_rn(__fmul2_rn(make_float2(v1[k], v1[k + 1]), ninv),
+                                         make_float2(pv.x, pv.y), make_float2(1.f, 1.f));
+            const float2 x1 = __ffma2_rn(__fmul2_rn(make_float2(v1[k + 2], v1[k + 3]), ninv),
+                                         make_float2(pv.z, pv.w), make_float2(1.f, 1.f));
+            mn = fminf(mn, fminf(fminf(x0.x, x0.y), fminf(x1.x, x1.y)));
+          }
+        }
+      }
+      // min(di, clamp(x, 0, 2)) == max(min(di, x), 0) for di in [0, 2]
+      s.dist[i] = fmaxf(fminf(di, mn), 0.f);
     }
   }
 }
@@ -230,11 +288,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) {
       mbar_init(smem_u32(&s.bars[i]), 1);
-      mbar_init(smem_u32(&s.bars[3 + i]), 1);
+      mbar_init(smem_u32(&s.bars[3 + i]), 2);  // the MMA's commit + the epilogue
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(smem_u32(&s.bars[6 + a]), 1);
-      mbar_init(smem_u32(&s.bars[8 + a]), 4);  // one arrive per epilogue warp
+      mbar_init(smem_u32(&s.bars[8 + a]), 4);  // one arrive per warp of its warpgroup
     }
     mbar_init(smem_u32(&s.bars[10]), 1);
     fence_barrier_init();
@@ -256,25 +314,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     Head h{beacons_in + static_cast<size_t>(qh) * g.M * kDim,
            window + static_cast<size_t>(qh) * g.W * kDim, g.nb_in, g.W};
     __nv_bfloat16 *out = beacons_out + static_cast<size_t>(qh) * g.M * kDim;
-    // inverse norms (0 for a zero vector, which makes its distance 1)
-    for (int i = tid; i < n; i += kThreads) {
-      const __nv_bfloat16 *p = h.point(i);
-      float ss = 0.f;
-#pragma unroll
-      for (int t = 0; t < kDim; t += 8) {
-        float u[8];
-        load8(p + t, u);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) ss = fmaf(u[j], u[j], ss);
-      }
-      s.inv[i] = ss > 0.f ? 1.0f / sqrtf(ss) : 0.f;
-    }
     if (tid == 0) {
       s.cidx[0] = 0;  // the seed U[0] is the first pick
       s.pick[0] = 0;
+      // its inverse norm, summed in the order the seed pass uses for every point
+      float ss = 0.f;
+      for (int t = 0; t < kDim; t += 8) {
+        float u[8];
+        load8(h.point(0) + t, u);
+        for (int e = 0; e < 8; ++e) ss = fmaf(u[e], u[e], ss);
+      }
+      s.pinv[0] = ss > 0.f ? 1.0f / sqrtf(ss) : 0.f;
     }
+    if (tid > 0 && tid < 16) s.pinv[tid] = __int_as_float(0x7fc00000);
     __syncthreads();
-    if (tid == 0) s.pinv[0] = s.inv[0];
     stage_picks(s, h, out, 0, 1);
     fence_proxy_async_smem();
     __syncthreads();
@@ -291,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int nc = min(kCand, unsel);
       const bool bounded = unsel > kCand;
       const int want = bounded ? kCand + 1 : nc;
-      select_best<kThreads>(s.dist, n, want, s.whist, s.hist, s.scal, s.cidx, s.cdist);
+      select_best<kThreads>(s.dist, n, unsel, want, s.whist, s.hist, s.scal, s.cidx, s.cdist);
       __syncthreads();
       int my_i = 0, my_rank = 0;
       float my_d = 0.f;
@@ -315,62 +368,82 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < 8; ++j) s.cvec[a * kCStride + t + j] = u[j];
       }
       __syncthreads();
-      // Gram block: lanes take consecutive candidates a of one pick b
-      for (int e = tid; e < nc * nc; e += kThreads) {
-        const int b = e / nc, a = e - b * nc;
-        float2 acc = make_float2(0.f, 0.f);
-#pragma unroll 4
+      // Gram block, 4 x 4 dot products per thread (a = ta + 16 r, b = tb + 16 r'):
+      // each loaded 8-element slice feeds four dot products, and the lanes of
+      // a phase read rows in distinct banks
+      if (tid < 256) {
+        const int ta = tid & 15, tb = tid >> 4;
+        float2 acc[4][4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) acc[r][q] = make_float2(0.f, 0.f);
+#pragma unroll 2
         for (int t = 0; t < kDim; t += 8) {
-          float u[8];
-          load8(s.cvec + a * kCStride + t, u);
-          acc = dot8_step(acc, u, s.cvec + b * kCStride + t);
+          float u[4][8], w[4][8];
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            load8(s.cvec + (ta + 16 * r) * kCStride + t, u[r]);
+            load8(s.cvec + (tb + 16 * r) * kCStride + t, w[r]);
+          }
+#pragma unroll
+          for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+#pragma unroll
+              for (int j = 0; j < 8; j += 2)
+                acc[r][q] = __ffma2_rn(make_float2(u[r][j], u[r][j + 1]),
+                                       make_float2(w[q][j], w[q][j + 1]), acc[r][q]);
         }
-        s.gram[a * kCand + b] = __fadd_rn(acc.x, acc.y);
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            s.gram[(tb + 16 * q) * kCand + ta + 16 * r] = __fadd_rn(acc[r][q].x, acc[r][q].y);
       }
       __syncthreads();
-      // replay the greedy choice among the candidates (warp 0, two per lane)
+      // replay the greedy choice among the candidates (warp 0, two per lane).
+      // The argmax in (distance desc, index asc) order takes two warp
+      // reductions: the largest distance key, then the lowest index holding it.
       if (warp == 0) {
         const int a0 = lane, a1 = lane + 32;
         bool t0 = a0 >= nc, t1 = a1 >= nc;  // taken or absent
-        float c0 = t0 ? -3.f : s.cdist[a0], c1 = t1 ? -3.f : s.cdist[a1];
+        float c0 = t0 ? 0.f : s.cdist[a0], c1 = t1 ? 0.f : s.cdist[a1];
         const int i0 = t0 ? 0x7fffffff : s.cidx[a0], i1 = t1 ? 0x7fffffff : s.cidx[a1];
         const float inv0 = t0 ? 0.f : s.inv[i0], inv1 = t1 ? 0.f : s.inv[i1];
         const float bd = bounded ? s.cdist[kCand] : -3.f;
         const int bi = bounded ? s.cidx[kCand] : 0x7fffffff;
         int np = 0;
         while (picked + np < m) {
-          float best_d = t0 ? -3.f : c0;
-          int best_i = t0 ? 0x7fffffff : i0, best_a = a0;
-          if (!t1 && before(c1, i1, best_d, best_i)) {
-            best_d = c1;
-            best_i = i1;
-            best_a = a1;
-          }
-          for (int off = 16; off > 0; off >>= 1) {
-            const float od = __shfl_xor_sync(0xffffffffu, best_d, off);
-            const int oi = __shfl_xor_sync(0xffffffffu, best_i, off);
-            const int oa = __shfl_xor_sync(0xffffffffu, best_a, off);
-            if (before(od, oi, best_d, best_i)) {
-              best_d = od;
-              best_i = oi;
-              best_a = oa;
-            }
-          }
-          if (best_d < 0.f) break;
+          // distances are >= 0, so their bits order like the values; +1 keeps
+          // 0 free for "taken"
+          const uint32_t k0 = t0 ? 0u : __float_as_uint(c0) + 1u;
+          const uint32_t k1 = t1 ? 0u : __float_as_uint(c1) + 1u;
+          const uint32_t kbest = __reduce_max_sync(0xffffffffu, max(k0, k1));
+          if (kbest == 0u) break;  // no candidate left
+          const uint32_t mine = min(k0 == kbest ? static_cast<uint32_t>(i0) : 0xffffffffu,
+                                    k1 == kbest ? static_cast<uint32_t>(i1) : 0xffffffffu);
+          const int best_i = static_cast<int>(__reduce_min_sync(0xffffffffu, mine));
+          const float best_d = __uint_as_float(kbest - 1u);
           if (bounded && !before(best_d, best_i, bd, bi)) break;
+          const bool own0 = k0 == kbest && i0 == best_i, own1 = k1 == kbest && i1 == best_i;
+          const uint32_t owners = __ballot_sync(0xffffffffu, own0 || own1);
+          const int src = __ffs(owners) - 1;
+          const int best_a = __shfl_sync(0xffffffffu, own0 ? a0 : a1, src);
           if (lane == 0) s.pick[np] = best_a;
           ++np;
-          if (best_a == a0) t0 = true;
-          if (best_a == a1) t1 = true;
+          if (own0) t0 = true;
+          if (own1) t1 = true;
           const float inv_b = s.inv[best_i];
-          if (!t0) c0 = fminf(c0, cos_dist(make_float2(s.gram[a0 * kCand + best_a], 0.f), inv0, inv_b));
-          if (!t1) c1 = fminf(c1, cos_dist(make_float2(s.gram[a1 * kCand + best_a], 0.f), inv1, inv_b));
+          if (!t0) c0 = fminf(c0, cos_dist(make_float2(s.gram[best_a * kCand + a0], 0.f), inv0, inv_b));
+          if (!t1) c1 = fminf(c1, cos_dist(make_float2(s.gram[best_a * kCand + a1], 0.f), inv1, inv_b));
         }
         if (lane == 0) s.scal[4] = np;
       }
       __syncthreads();
       const int np = s.scal[4];
-      if (tid < np) s.pinv[tid] = s.inv[s.cidx[s.pick[tid]]];
+      if (tid < ((np + 15) & ~15))
+        s.pinv[tid] = tid < np ? s.inv[s.cidx[s.pick[tid]]] : __int_as_float(0x7fc00000);
       stage_picks(s, h, out, picked, np);
       __syncthreads();
       if (tid < np) s.dist[s.cidx[s.pick[tid]]] = -1.f;

@@ -276,7 +276,7 @@ __global__ void __launch_bounds__(kP1Threads, 1)
     bool ok = true;
     for (int t = 0; t < n_tiles && ok; ++t) {
       const int acc = t & 1;
-      if (!mbar_wait(tfull0 + 8 * acc, (t >> 1) & 1, kWhereP1Epi)) { ok = false; break; }
+      if (!mbar_wait_warp(tfull0 + 8 * acc, (t >> 1) & 1, kWhereP1Epi)) { ok = false; break; }
       tc_fence_after();
       const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) +
                              acc * kP1Keys + wg * 64;
@@ -482,7 +482,7 @@ __global__ void __launch_bounds__(kP2Threads, 1)
     for (int it = 0; it < n_tiles && ok; ++it) {
       float y = -INFINITY;
       for (int u = 0; u < n_sub; ++u) {
-        if (!mbar_wait(tfull0 + 8 * u, it & 1, kWhereP2Epi)) { ok = false; break; }
+        if (!mbar_wait_warp(tfull0 + 8 * u, it & 1, kWhereP2Epi)) { ok = false; break; }
         tc_fence_after();
         const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + u * 256;
         const float *cu = ct + u * N0;

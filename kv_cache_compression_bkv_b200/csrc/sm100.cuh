@@ -71,6 +71,13 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int whe
   }
 }
 
+// mbar_wait by every lane of a warp, with one outcome for the whole warp (so
+// that the warp-collective tcgen05 instructions after it are executed by all
+// lanes or by none).
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, int where) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, where));
+}
+
 // ---------------------------------------------------------------- fences
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
