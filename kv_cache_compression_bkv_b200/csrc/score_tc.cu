@@ -11,9 +11,12 @@
 //     rows, N = 256 keys.  TMEM lane = observation row, so each epilogue
 //     thread owns one row and keeps an online (max, sum of exp2) over the
 //     columns it reads; no cross-thread reduction per element.
-//   pass 2 (column max)       D[j][o] = K_tile . Q_grp^T, M = 128 keys, N =
-//     up to 2 x 256 observation rows.  TMEM lane = key, so each epilogue
-//     thread owns one key and reduces max_o (acc - c_o / scale) in registers.
+//   pass 2 (column max)       D[j][o] = K_tile . Q_grp^T - c_o / scale, M = 128
+//     keys, N = up to 2 x 256 observation rows.  The subtraction is one more
+//     K=16 step of the same MMA: every key carries a block (1, 1, 1, 0, ...)
+//     and every observation row (-c_hi, -c_mid, -c_lo, 0, ...), the three
+//     bf16 parts of c_o / scale.  TMEM lane = key, so each epilogue thread owns
+//     one key and takes the max over its columns in registers.
 //
 // Both passes: warp 0 issues TMA loads of the key tiles (128-byte swizzle, no
 // multicast) into a ring of shared-memory stages; warp 1 allocates TMEM and
@@ -23,6 +26,7 @@
 // 16-byte loads and written to shared memory in the same swizzled layout.
 // Every wait is bounded (sm100.cuh).
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
@@ -346,12 +350,15 @@ __global__ void __launch_bounds__(kP1Threads, 1)
 // ------------------------------------------------------------------ pass 2
 constexpr int kP2Keys = 128;
 constexpr int kP2MaxRows = 512;
-constexpr int kP2Threads = 256;  // warp 0 TMA, warp 1 MMA, warps 2..3 loaders, 4..7 epilogue
+constexpr int kP2Threads = 384;  // warp 0 TMA, warp 1 MMA, warps 4..7 / 8..11 epilogue
+                                 // warpgroups for the two column sub-chunks
 constexpr int kP2TileBytes = kP2Keys * kRowBytes;  // 32 KB
-constexpr int kP2SmallBytes = 256 + kP2MaxRows * 4; // barriers + TMEM slot, c / scale
+constexpr int kP2SmallBytes = 256 + 2 * 128 * 4;  // barriers + TMEM slot, exchange
+constexpr int kP2ExtraRowBytes = 32;              // the extra K=16 step, 32-byte swizzle
 
 __host__ __device__ constexpr int p2_smem_bytes(int rows_pad, int stages) {
-  return kP2SmallBytes + 1024 + rows_pad * kRowBytes + stages * kP2TileBytes;
+  return kP2SmallBytes + 1024 + rows_pad * kRowBytes + stages * kP2TileBytes +
+         kP2Keys * kP2ExtraRowBytes + rows_pad * kP2ExtraRowBytes;
 }
 
 __global__ void __launch_bounds__(kP2Threads, 1)
@@ -362,7 +369,7 @@ __global__ void __launch_bounds__(kP2Threads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem_raw);  // 16 barriers
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem_raw + 128);
-  float *ct = reinterpret_cast<float *>(smem_raw + 256);   // [512] c_o / scale
+  float *ybuf = reinterpret_cast<float *>(smem_raw + 256);  // [2][128] sub-chunk 1 maxima
   const uint32_t raw_base = smem_u32(smem_raw);
   const uint32_t tile_base = (raw_base + kP2SmallBytes + 1023u) & ~1023u;
 
@@ -388,6 +395,8 @@ __global__ void __launch_bounds__(kP2Threads, 1)
 
   uint8_t *sQ = smem_raw + (tile_base - raw_base);
   uint8_t *sK = sQ + rows_pad * kRowBytes;
+  uint8_t *sXk = sK + n_stages * kP2TileBytes;      // keys' extra step: (1, 1, 1, 0, ...)
+  uint8_t *sXq = sXk + kP2Keys * kP2ExtraRowBytes;  // rows' extra step: -c_o / scale
 
   const uint32_t full0 = smem_u32(&bars[0]);    // [<=4]
   const uint32_t empty0 = smem_u32(&bars[4]);   // [<=4]
@@ -402,7 +411,7 @@ __global__ void __launch_bounds__(kP2Threads, 1)
     }
     for (int u = 0; u < 2; ++u) {
       mbar_init(tfull0 + 8 * u, 1);
-      mbar_init(tempty0 + 8 * u, 4);  // one arrive per epilogue warp
+      mbar_init(tempty0 + 8 * u, 4);  // one arrive per warp of its warpgroup
     }
     mbar_init(done, 1);
     fence_barrier_init();
@@ -413,9 +422,32 @@ __global__ void __launch_bounds__(kP2Threads, 1)
     tmem_relinquish();
   }
   const float inv_scale = 1.0f / g.scale;
-  for (int r = threadIdx.x; r < kP2MaxRows; r += blockDim.x)
-    ct[r] = (r < nrows) ? c_in[static_cast<size_t>(head) * g.n_obs_pad + r0 + r] * inv_scale
-                        : INFINITY;
+  for (int r = threadIdx.x; r < kP2Keys; r += blockDim.x) {
+    const uint32_t one = 0x3F80u;  // bf16 1.0
+    *reinterpret_cast<uint4 *>(sXk + sw32_offset(r, 0)) =
+        make_uint4(one | (one << 16), one, 0u, 0u);
+    *reinterpret_cast<uint4 *>(sXk + sw32_offset(r, 1)) = make_uint4(0u, 0u, 0u, 0u);
+  }
+  for (int r = threadIdx.x; r < rows_pad; r += blockDim.x) {
+    // c / scale as hi + mid + lo in bf16 (exact splits in f32); padded rows
+    // get a huge negative offset so that they never win the max
+    uint32_t w0, w1;
+    if (r < nrows) {
+      const float c = c_in[static_cast<size_t>(head) * g.n_obs_pad + r0 + r] * inv_scale;
+      const __nv_bfloat16 hi = __float2bfloat16_rn(-c);
+      const float r1 = -c - __bfloat162float(hi);
+      const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+      w0 = static_cast<uint32_t>(__bfloat16_as_ushort(hi)) |
+           (static_cast<uint32_t>(__bfloat16_as_ushort(mid)) << 16);
+      w1 = static_cast<uint32_t>(__bfloat16_as_ushort(lo));
+    } else {
+      w0 = 0xF149u;  // bf16 -1e30
+      w1 = 0u;
+    }
+    *reinterpret_cast<uint4 *>(sXq + sw32_offset(r, 0)) = make_uint4(w0, w1, 0u, 0u);
+    *reinterpret_cast<uint4 *>(sXq + sw32_offset(r, 1)) = make_uint4(0u, 0u, 0u, 0u);
+  }
   load_obs_rows_sw128(sQ, rows_pad, r0, g, recent, beacons, layer, kvh);
   fence_proxy_async_smem();
   tc_fence_before();
@@ -467,6 +499,8 @@ __global__ void __launch_bounds__(kP2Threads, 1)
               umma_f16(d, ad, bd, idesc, (kb | kk) != 0);
             }
           }
+          umma_f16(d, smem_desc_k_sw32(smem_u32(sXk)),
+                   smem_desc_k_sw32(smem_u32(sXq) + u * N0 * kP2ExtraRowBytes), idesc, 1u);
           umma_commit(tfull0 + 8 * u);
         }
         umma_commit(empty0 + 8 * s);
@@ -475,49 +509,72 @@ __global__ void __launch_bounds__(kP2Threads, 1)
       mbar_wait(done, 0, kWhereP2Drain);
     }
   } else if (warp >= 4) {
+    // warpgroup u reduces column sub-chunk u: per key (TMEM lane) the max over
+    // its observation rows of acc - c_o / scale; sub-chunk 1's maxima reach
+    // warpgroup 0 through shared memory
+    const int u = (warp - 4) >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;  // key within the tile
     float *yout = ypart + (static_cast<size_t>(gi) * g.n_heads() + head) * static_cast<size_t>(L);
-    bool ok = true;
-    for (int it = 0; it < n_tiles && ok; ++it) {
-      float y = -INFINITY;
-      for (int u = 0; u < n_sub; ++u) {
-        if (!mbar_wait_warp(tfull0 + 8 * u, it & 1, kWhereP2Epi)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + u * 256;
-        const float *cu = ct + u * N0;
-        const int Nu = u == 0 ? N0 : N1;
-        int col = 0;
+    if (u < n_sub) {
+      const int Nu = u == 0 ? N0 : N1;
+      const int n32 = Nu >> 5;
+      bool ok = true;  // warp-uniform; after a timeout only the barriers remain
+      for (int it = 0; it < n_tiles; ++it) {
+        float y0 = -INFINITY, y1 = -INFINITY;
+        if (ok && !mbar_wait_warp(tfull0 + 8 * u, it & 1, kWhereP2Epi)) ok = false;
+        if (ok) {
+          tc_fence_after();
+          const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + u * 256;
+          auto reduce32 = [&](const float (&v)[32], int) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+              y0 = max3f(y0, v[i], v[i + 1]);
+              y1 = max3f(y1, v[i + 2], v[i + 3]);
+            }
+          };
+          // two TMEM loads in flight: chunk c+1 lands while chunk c is reduced
+          float va[32], vb[32];
+          int c = 0;
+          if (n32 > 0) {
+            tmem_ld_32x32b_x32(taddr, va);
+            tmem_ld_wait_regs(va);
+          }
 #pragma unroll 1
-        for (; col + 32 <= Nu; col += 32) {
-          float v[32];
-          tmem_ld_32x32b_x32(taddr + col, v);
-          tmem_ld_wait_regs(v);
-#pragma unroll
-          for (int i = 0; i < 32; i += 4) {
-            const float4 c4 = *reinterpret_cast<const float4 *>(cu + col + i);
-            y = fmaxf(y, fmaxf(fmaxf(v[i] - c4.x, v[i + 1] - c4.y),
-                               fmaxf(v[i + 2] - c4.z, v[i + 3] - c4.w)));
+          for (; c + 2 <= n32; c += 2) {
+            tmem_ld_32x32b_x32(taddr + (c + 1) * 32, vb);
+            reduce32(va, c * 32);
+            tmem_ld_wait_regs(vb);
+            if (c + 2 < n32) tmem_ld_32x32b_x32(taddr + (c + 2) * 32, va);
+            reduce32(vb, (c + 1) * 32);
+            if (c + 2 < n32) tmem_ld_wait_regs(va);
           }
-        }
-        if (col < Nu) {  // Nu is a multiple of 16
-          float v[16];
-          tmem_ld_32x32b_x16(taddr + col, v);
-          tmem_ld_wait_regs(v);
+          if (c < n32) reduce32(va, c * 32);
+          if (Nu & 16) {  // Nu is a multiple of 16
+            float v[16];
+            tmem_ld_32x32b_x16(taddr + n32 * 32, v);
+            tmem_ld_wait_regs(v);
 #pragma unroll
-          for (int i = 0; i < 16; i += 4) {
-            const float4 c4 = *reinterpret_cast<const float4 *>(cu + col + i);
-            y = fmaxf(y, fmaxf(fmaxf(v[i] - c4.x, v[i + 1] - c4.y),
-                               fmaxf(v[i + 2] - c4.z, v[i + 3] - c4.w)));
+            for (int i = 0; i < 16; i += 4) {
+              y0 = max3f(y0, v[i], v[i + 1]);
+              y1 = max3f(y1, v[i + 2], v[i + 3]);
+            }
           }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(tempty0 + 8 * u);
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(tempty0 + 8 * u);
+        float y = fmaxf(y0, y1);
+        if (n_sub == 2) {
+          if (u == 1) ybuf[(it & 1) * 128 + row] = y;
+          named_barrier_sync(1, 256);
+          if (u == 0) y = fmaxf(y, ybuf[(it & 1) * 128 + row]);
+        }
+        if (u == 0 && ok) {
+          const long long j = static_cast<long long>(t0 + it) * kP2Keys + row;
+          if (j < L) yout[j] = y * g.scale;
+        }
       }
-      if (!ok) break;
-      const long long j = static_cast<long long>(t0 + it) * kP2Keys + row;
-      if (j < L) yout[j] = y * g.scale;
     }
   }
   tc_fence_before();

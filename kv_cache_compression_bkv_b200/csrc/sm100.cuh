@@ -213,6 +213,25 @@ __device__ __forceinline__ uint64_t smem_desc_k_sw128(uint32_t addr) {
   return d;
 }
 
+// Shared-memory matrix descriptor of a K-major operand whose K extent is one
+// 16-element step stored with the 32-byte swizzle: rows of 32 B, 8-row atoms
+// of 256 B stacked at a 256 B stride.
+__device__ __forceinline__ uint64_t smem_desc_k_sw32(uint32_t addr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((addr & 0x3FFFFu) >> 4);         // start address
+  d |= static_cast<uint64_t>(1u) << 16;                        // leading byte offset (unused)
+  d |= static_cast<uint64_t>(256u >> 4) << 32;                 // stride byte offset: 8-row atom
+  d |= static_cast<uint64_t>(1u) << 46;                        // descriptor version (sm100)
+  d |= static_cast<uint64_t>(6u) << 61;                        // swizzle: 32 B
+  return d;
+}
+
+// Byte offset of the 16-byte chunk `c` (0..1) of row `r` in a tile stored with
+// the 32-byte swizzle: chunk index XOR bit 2 of the row.
+__host__ __device__ constexpr uint32_t sw32_offset(uint32_t r, uint32_t c) {
+  return r * 32u + ((c ^ ((r >> 2) & 1u)) << 4);
+}
+
 // Instruction descriptor of kind::f16 with bf16 A/B, f32 D, both K-major.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
   return (1u << 4)                                  // D format: f32
