@@ -57,6 +57,28 @@ def load_peaks():
                 sm_max_mhz=1965.0, source="fallback")
 
 
+def load_traffic():
+    """DRAM bytes per launch of each phase's kernel from profiles/traffic.json
+    (an ncu capture), or None for a kernel whose sources changed since."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return {}
+    with open(path) as f:
+        rec = json.load(f)
+    out = {}
+    for phase, r in rec.items():
+        m = hashlib.sha256()
+        try:
+            for src in r["sources"]:
+                with open(os.path.join(ROOT, src), "rb") as f:
+                    m.update(f.read())
+        except OSError:
+            continue
+        out[phase] = r["bytes_per_launch"] if m.hexdigest() == r["sha256"] else None
+    return out
+
+
 # ----------------------------------------------------------------------------
 # algorithmic work per phase (per step, one rank)
 # ----------------------------------------------------------------------------
@@ -393,6 +415,7 @@ def main():
 
     peaks = load_peaks()
     wm = work_model(wl)
+    traffic = load_traffic() if args.workload == "qwen3_14b" and not args.layers else {}
     phases = {}
     for p in PHASES:
         m = wm[p]
@@ -400,12 +423,13 @@ def main():
         sec = phase_ms[p] / 1e3
         ach = rate(m["work"], m["unit"], sec) if sec > 0 else 0.0
         phases[p] = {"ms": phase_ms[p], "bound": m["bound"], "achieved": ach, "peak": pk,
-                     "unit": pu, "frac": ach / pk if pk else None}
+                     "unit": pu, "frac": ach / pk if pk else None,
+                     "traffic": traffic.get(p)}
     dom = max(PHASES, key=lambda p: phase_ms[p])
     dm = phases[dom]
     per_launch = wm[dom]["work"]
     roofline = {"bound": dm["bound"], "achieved": dm["achieved"], "peak": dm["peak"],
-                "unit": dm["unit"], "frac": dm["frac"], "traffic": None, "kernel": dom,
+                "unit": dm["unit"], "frac": dm["frac"], "traffic": traffic.get(dom), "kernel": dom,
                 "peak_source": peaks["source"] + (" sustained" if dm["bound"] == "tensor" else ""),
                 "work_per_launch": per_launch}
     t_tensor = wm["step_flop"] / (peaks["bf16_tflops_sustained"] * 1e12)

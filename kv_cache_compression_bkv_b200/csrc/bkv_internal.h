@@ -7,7 +7,7 @@
 #include <stddef.h>
 #include <stdint.h>
 
-#include "../../include/bkv.h"
+#include "bkv.h"
 
 namespace bkv {
 

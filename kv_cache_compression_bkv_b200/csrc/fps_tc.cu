@@ -88,29 +88,35 @@ __device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
 // issuer (warp 1) and epilogue (warps 4..7) run their own loops; `seq` is the
 // number of tiles all passes so far have moved through the ring, so every
 // role derives the same stage and phase for each tile.
+// Issue the TMA loads of tiles [j0, j1) of the pass that starts at `seq`
+// (producer thread only).  Returns false after a timeout.
+__device__ bool issue_tiles(const Layout &s, const CUtensorMap *bmap, const CUtensorMap *wmap,
+                            int qh, const FpsGeom &g, int n_btiles, uint32_t seq, int j0,
+                            int j1) {
+  const uint32_t full0 = smem_u32(&s.bars[0]), empty0 = smem_u32(&s.bars[3]);
+  for (int j = j0; j < j1; ++j) {
+    const uint32_t q = seq + j, st = q % kStages;
+    if (!mbar_wait(empty0 + 8 * st, ((q / kStages) & 1) ^ 1, kWhereProd)) return false;
+    mbar_arrive_expect_tx(full0 + 8 * st, kTileBytes);
+    const uint32_t dst = smem_u32(s.stages + st * kTileBytes);
+    const CUtensorMap *map = j < n_btiles ? bmap : wmap;
+    const int y = j < n_btiles ? qh * g.M + j * kTileRows : qh * g.W + (j - n_btiles) * kTileRows;
+    tma_load_2d(dst, map, full0 + 8 * st, 0, y);
+    tma_load_2d(dst + kTileRows * 128, map, full0 + 8 * st, 64, y);
+  }
+  return true;
+}
+
 __device__ void distance_pass(const Layout &s, const CUtensorMap *bmap, const CUtensorMap *wmap,
                               uint32_t tmem, int qh, const FpsGeom &g, int n_btiles, int n_tiles,
-                              uint32_t seq, int np, bool first) {
+                              uint32_t seq, int np, bool first, int prefetched) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t full0 = smem_u32(&s.bars[0]), empty0 = smem_u32(&s.bars[3]);
   const uint32_t tfull0 = smem_u32(&s.bars[6]), tempty0 = smem_u32(&s.bars[8]);
   if (warp == 0) {
-    if (lane == 0) {
-      for (int j = 0; j < n_tiles; ++j) {
-        const uint32_t q = seq + j, st = q % kStages;
-        if (!mbar_wait(empty0 + 8 * st, ((q / kStages) & 1) ^ 1, kWhereProd)) {
-          s.scal[kAbort] = 1;
-          break;
-        }
-        mbar_arrive_expect_tx(full0 + 8 * st, kTileBytes);
-        const uint32_t dst = smem_u32(s.stages + st * kTileBytes);
-        const CUtensorMap *map = j < n_btiles ? bmap : wmap;
-        const int y = j < n_btiles ? qh * g.M + j * kTileRows
-                                   : qh * g.W + (j - n_btiles) * kTileRows;
-        tma_load_2d(dst, map, full0 + 8 * st, 0, y);
-        tma_load_2d(dst + kTileRows * 128, map, full0 + 8 * st, 64, y);
-      }
-    }
+    if (lane == 0 &&
+        !issue_tiles(s, bmap, wmap, qh, g, n_btiles, seq, prefetched, n_tiles))
+      s.scal[kAbort] = 1;
   } else if (warp == 1) {
     if (lane == 0) {
       const int npad = (np + 15) & ~15;
@@ -331,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     stage_picks(s, h, out, 0, 1);
     fence_proxy_async_smem();
     __syncthreads();
-    distance_pass(s, &bmap, &wmap, tmem, qh, g, n_btiles, n_tiles, seq, 1, true);
+    distance_pass(s, &bmap, &wmap, tmem, qh, g, n_btiles, n_tiles, seq, 1, true, 0);
     seq += n_tiles;
     __syncthreads();
     if (s.scal[kAbort]) break;
@@ -344,20 +350,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int nc = min(kCand, unsel);
       const bool bounded = unsel > kCand;
       const int want = bounded ? kCand + 1 : nc;
+      // the next distance pass streams the same tiles whatever this round
+      // picks: start its first loads now, behind the round's selection work
+      const int pre = min(kStages, n_tiles);
+      if (tid == 0 && !issue_tiles(s, &bmap, &wmap, qh, g, n_btiles, seq, 0, pre))
+        s.scal[kAbort] = 1;
       select_best<kThreads>(s.dist, n, unsel, want, s.whist, s.hist, s.scal, s.cidx, s.cdist);
       __syncthreads();
-      int my_i = 0, my_rank = 0;
-      float my_d = 0.f;
-      if (tid < want) {
-        my_i = s.cidx[tid];
-        my_d = s.cdist[tid];
-        for (int j = 0; j < want; ++j)
-          if (j != tid && before(s.cdist[j], s.cidx[j], my_d, my_i)) ++my_rank;
-      }
-      __syncthreads();
-      if (tid < want) {
-        s.cidx[my_rank] = my_i;
-        s.cdist[my_rank] = my_d;
+      // the candidates need no order; only the bound (the last of the kCand+1
+      // selected in (distance desc, index asc) order) moves to slot kCand
+      if (bounded && warp == 0) {
+        float wd = 3.f;
+        int wi = -1, ws = -1;
+        for (int j = lane; j < want; j += 32) {
+          const float dj = s.cdist[j];
+          const int ij = s.cidx[j];
+          if (ws < 0 || before(wd, wi, dj, ij)) {
+            wd = dj;
+            wi = ij;
+            ws = j;
+          }
+        }
+        for (int off = 16; off > 0; off >>= 1) {
+          const float od = __shfl_xor_sync(0xffffffffu, wd, off);
+          const int oi = __shfl_xor_sync(0xffffffffu, wi, off);
+          const int os = __shfl_xor_sync(0xffffffffu, ws, off);
+          if (os >= 0 && (ws < 0 || before(wd, wi, od, oi))) {
+            wd = od;
+            wi = oi;
+            ws = os;
+          }
+        }
+        if (lane == 0 && ws != kCand) {
+          s.cidx[ws] = s.cidx[kCand];
+          s.cdist[ws] = s.cdist[kCand];
+          s.cidx[kCand] = wi;
+          s.cdist[kCand] = wd;
+        }
       }
       __syncthreads();
       for (int e = tid; e < nc * (kDim / 8); e += kThreads) {
@@ -449,7 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (tid < np) s.dist[s.cidx[s.pick[tid]]] = -1.f;
       fence_proxy_async_smem();
       __syncthreads();
-      distance_pass(s, &bmap, &wmap, tmem, qh, g, n_btiles, n_tiles, seq, np, false);
+      distance_pass(s, &bmap, &wmap, tmem, qh, g, n_btiles, n_tiles, seq, np, false, pre);
       seq += n_tiles;
       __syncthreads();
       if (s.scal[kAbort]) break;

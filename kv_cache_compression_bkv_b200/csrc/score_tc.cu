@@ -349,7 +349,6 @@ __global__ void __launch_bounds__(kP1Threads, 1)
 
 // ------------------------------------------------------------------ pass 2
 constexpr int kP2Keys = 128;
-constexpr int kP2MaxRows = 512;
 constexpr int kP2Threads = 384;  // warp 0 TMA, warp 1 MMA, warps 4..7 / 8..11 epilogue
                                  // warpgroups for the two column sub-chunks
 constexpr int kP2TileBytes = kP2Keys * kRowBytes;  // 32 KB
