@@ -226,6 +226,21 @@ def oracle_sample(wl, seed: int, n_heads: int, L_sample: int):
     return n_heads * L_sample, dt, len(threads)
 
 
+def max_over_ranks(x: float, dist, device) -> float:
+    """The largest of every rank's x (the slowest rank's time); x itself
+    without a process group.  Every rank must call it at the same point."""
+    if dist is None:
+        return x
+    tt = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    return float(tt.item())
+
+
+def weak_scaling_value(entries_per_rank: int, world: int, ms_max: float) -> float:
+    """Entries processed by all ranks per second, timed by the slowest rank."""
+    return world * entries_per_rank / (ms_max / 1e3)
+
+
 def cpu_threads() -> int:
     try:
         return len(os.sched_getaffinity(0))
@@ -370,13 +385,9 @@ def main():
     ms_local = t_start.elapsed_time(t_end) / args.steps
     phase_ms = {p: sum(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(args.steps)) / args.steps
                 for j, p in enumerate(PHASES)}
-    ms = ms_local
-    if dist is not None:
-        tt = torch.tensor([ms_local], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(ms_local, dist, dev)
     entries = wl.n_layers * wl.n_kv_heads * wl.L
-    value = world * entries / (ms / 1e3)
+    value = weak_scaling_value(entries, world, ms)
 
     # ---- end to end: pinned host inputs in, compacted cache out, every step
     e2e_steps = args.e2e_steps or max(3, min(args.steps, 10))
@@ -402,11 +413,7 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if dist is not None:
-        tt = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dist, dev)
 
     if rank != 0:
         if dist is not None:
@@ -461,7 +468,7 @@ def main():
         "roofline": roofline,
         "phases": phases,
         "cpu_baseline": cpu,
-        "e2e": {"value": world * entries / (e2e_ms / 1e3), "unit": UNIT,
+        "e2e": {"value": weak_scaling_value(entries, world, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "clocks": clk,
         "gpu_launches": (5 if wl.W else 4) * args.steps,

@@ -1,0 +1,103 @@
+"""A continual decoding trace driven through the C ABI.
+
+The caller's side of BeaconKV's periodic compression: the cache grows by one
+row per decode step, and every `interval` steps one bkv_compress_step call
+updates the beacons by Continual FPS over the queries of that interval (the
+window), scores the cache with the recent and beacon queries, keeps the
+budget K and compacts into the other of two cache buffers.  The decode step
+itself is not simulated: the keys, values and queries of each interval come
+from the seeded trace generator (synth.trace_*) and are appended in one copy.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import torch
+
+from . import bkv, synth
+
+
+@dataclass
+class TraceEvent:
+    index: int          # compression event number (0-based)
+    step: int           # decode steps generated so far
+    L: int              # cache rows scored
+    new_len: int        # rows kept
+    n_beacons_in: int
+    n_beacons_out: int
+    ms: float           # device time of the compress_step call
+
+
+@dataclass
+class TraceRun:
+    tr: synth.Trace
+    seed: int
+    device: torch.device
+    layers: int | None = None      # use only the first `layers` layers
+    events: list[TraceEvent] = field(default_factory=list)
+
+    def __post_init__(self):
+        tr = self.tr
+        self.Ly = self.layers or tr.n_layers
+        Ly, Hq, Hkv, d, dt = self.Ly, tr.n_q_heads, tr.n_kv_heads, tr.head_dim, tr.torch_dtype
+        self.cap = tr.K + tr.interval
+        self.keys = torch.empty(Ly, Hkv, tr.steps, d, dtype=dt)
+        self.values = torch.empty(Ly, Hkv, tr.steps, d, dtype=dt)
+        self.queries = torch.empty(Ly, Hq, tr.steps, d, dtype=dt)
+        for l in range(Ly):
+            for h in range(Hkv):
+                k, v = synth.trace_keys_values(tr, self.seed, l, h)
+                self.keys[l, h] = k.to(dt)
+                self.values[l, h] = v.to(dt)
+            for q in range(Hq):
+                self.queries[l, q] = synth.trace_queries(tr, self.seed, l, q).to(dt)
+        dev = self.device
+        self.cache = [(torch.zeros(Ly, Hkv, self.cap, d, dtype=dt, device=dev),
+                       torch.zeros(Ly, Hkv, self.cap, d, dtype=dt, device=dev)) for _ in range(2)]
+        self.beacons = [torch.zeros(Ly, Hq, tr.M, d, dtype=dt, device=dev) for _ in range(2)]
+        self.window = torch.empty(Ly, Hq, tr.interval, d, dtype=dt, device=dev)
+        self.recent = torch.empty(Ly, Hq, tr.R, d, dtype=dt, device=dev)
+        self.idx_flat = torch.empty(Ly * Hkv * tr.K, dtype=torch.int32, device=dev)
+        self.last_idx = None    # kept positions of the last event, [Ly][Hkv][kept]
+        self.geom = bkv.Geometry(Ly, Hq, Hkv, d, self.cap, dt)
+        self.ws = torch.empty(bkv.bkv_workspace_size(self.geom, self.cap, tr.R, tr.M,
+                                                     tr.interval, tr.K),
+                              dtype=torch.uint8, device=dev)
+        self.cur = 0            # which cache / beacon buffer holds the state
+        self.L = 0              # cache rows
+        self.n_beacons = 0
+
+    def run(self, on_event=None):
+        """Run the whole trace; on_event(run, event) sees the state after each
+        compression (the current buffers; run.last_idx = kept positions)."""
+        tr = self.tr
+        stream = torch.cuda.current_stream(self.device)
+        for e, t0 in enumerate(range(0, tr.steps, tr.interval)):
+            t1 = t0 + tr.interval
+            kc, vc = self.cache[self.cur]
+            kc[:, :, self.L:self.L + tr.interval].copy_(self.keys[:, :, t0:t1])
+            vc[:, :, self.L:self.L + tr.interval].copy_(self.values[:, :, t0:t1])
+            self.window.copy_(self.queries[:, :, t0:t1])
+            self.recent.copy_(self.queries[:, :, t1 - tr.R:t1])
+            L = self.L + tr.interval
+            kd, vd = self.cache[1 - self.cur]
+            bin_, bout = self.beacons[self.cur], self.beacons[1 - self.cur]
+            keep = min(tr.K, L)
+            idx = self.idx_flat[:self.Ly * tr.n_kv_heads * keep].view(self.Ly, tr.n_kv_heads, keep)
+            ev0 = torch.cuda.Event(enable_timing=True)
+            ev1 = torch.cuda.Event(enable_timing=True)
+            ev0.record(stream)
+            nb, nl = bkv.bkv_compress_step(
+                self.geom, kc, vc, L, tr.K, self.recent, tr.R,
+                bin_ if self.n_beacons else None, self.n_beacons, tr.M, self.window,
+                tr.interval, bout, 0.0, self.geom, kd, vd, None, idx, self.ws, stream)
+            ev1.record(stream)
+            torch.cuda.synchronize(self.device)
+            event = TraceEvent(e, t1, L, nl, self.n_beacons, nb, ev0.elapsed_time(ev1))
+            self.events.append(event)
+            self.cur = 1 - self.cur
+            self.L, self.n_beacons = nl, nb
+            self.last_idx = idx
+            if on_event is not None:
+                on_event(self, event)
+        return self.events
