@@ -189,7 +189,7 @@ class ClockSampler:
 # ----------------------------------------------------------------------------
 # the float64 oracle on a bounded sample (CPU baseline / reference arm)
 # ----------------------------------------------------------------------------
-def oracle_sample(wl, seed: int, n_heads: int, L_sample: int):
+def oracle_sample(wl, seed: int, n_heads: int, L_sample: int, aggregate: str = "max"):
     """Run the oracle's whole step on n_heads (layer, KV head)s, one thread
     each, with each head's keys cut to its first L_sample rows.  Returns
     (entries, seconds, threads)."""
@@ -213,7 +213,8 @@ def oracle_sample(wl, seed: int, n_heads: int, L_sample: int):
 
     def run(job):
         k, v, r, b, w = job
-        out = oracle.compress_head(k, v, r, b, wls.beacons_in, w, wls.M, wls.K)
+        out = oracle.compress_head(k, v, r, b, wls.beacons_in, w, wls.M, wls.K,
+                                   aggregate=aggregate)
         done.append(len(out["idx"]))
 
     threads = [threading.Thread(target=run, args=(j,)) for j in jobs]
@@ -224,6 +225,15 @@ def oracle_sample(wl, seed: int, n_heads: int, L_sample: int):
         t.join()
     dt = time.perf_counter() - t0
     return n_heads * L_sample, dt, len(threads)
+
+
+def workload_config(wl, args) -> dict:
+    cfg = {"workload": wl.name, "n_layers": wl.n_layers, "n_q_heads": wl.n_q_heads,
+           "n_kv_heads": wl.n_kv_heads, "head_dim": wl.head_dim, "L": wl.L, "R": wl.R,
+           "M": wl.M, "K": wl.K, "W": wl.W}
+    if args.aggregate != "max":
+        cfg["aggregate"] = args.aggregate
+    return cfg
 
 
 def max_over_ranks(x: float, dist, device) -> float:
@@ -253,16 +263,16 @@ def run_reference(args, wl, rank, world):
         return
     n_thr = max(1, min(cpu_threads(), 16))
     # size the per-step sample so that warmup + steps stay within ~2.5 minutes
-    ent, dt, _ = oracle_sample(wl, args.seed, 1, 1024)
+    ent, dt, _ = oracle_sample(wl, args.seed, 1, 1024, args.aggregate)
     per_key = dt / 1024.0
     budget = 150.0 / max(1, args.steps + args.warmup)
     L_sample = int(max(256, min(wl.L, budget / max(per_key, 1e-9))))
     L_sample = max(256, L_sample // 256 * 256)
     for _ in range(args.warmup):
-        oracle_sample(wl, args.seed, n_thr, L_sample)
+        oracle_sample(wl, args.seed, n_thr, L_sample, args.aggregate)
     tot_e, tot_t = 0, 0.0
     for _ in range(args.steps):
-        e, t, _ = oracle_sample(wl, args.seed, n_thr, L_sample)
+        e, t, _ = oracle_sample(wl, args.seed, n_thr, L_sample, args.aggregate)
         tot_e += e
         tot_t += t
     value = tot_e / tot_t
@@ -273,7 +283,7 @@ def run_reference(args, wl, rank, world):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": wl.name},
+            "config": workload_config(wl, args),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": n_thr, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -296,6 +306,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=None,
                     help="use only this many layers (small cases for profiler captures)")
+    ap.add_argument("--aggregate", default="max", choices=["max", "mean"],
+                    help="aggregation over the observation rows (mean: Table 2's ablation)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -349,7 +361,8 @@ def main():
         return bkv.bkv_compress_step(g, t["k"], t["v"], wl.L, wl.K, t["recent"], wl.R,
                                      t["beacons"], wl.beacons_in, wl.M,
                                      t["window"] if wl.W else None, wl.W, bout, 0.0, dstg, kd,
-                                     vd, None, idx, ws, stream, events)
+                                     vd, None, idx, ws, stream, events,
+                                     aggregate=args.aggregate)
 
     for _ in range(args.warmup):
         step()
@@ -422,7 +435,9 @@ def main():
 
     peaks = load_peaks()
     wm = work_model(wl)
-    traffic = load_traffic() if args.workload == "qwen3_14b" and not args.layers else {}
+    # the captured counters are those of the default configuration
+    traffic = (load_traffic() if args.workload == "qwen3_14b" and not args.layers
+               and args.aggregate == "max" else {})
     phases = {}
     for p in PHASES:
         m = wm[p]
@@ -446,7 +461,7 @@ def main():
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         n_thr = max(1, min(cpu_threads(), 4))
-        e, t, used = oracle_sample(wl, args.seed, n_thr, wl.L)
+        e, t, used = oracle_sample(wl, args.seed, n_thr, wl.L, args.aggregate)
         cpu = {"value": e / t, "unit": UNIT, "cores": used, "kind": "oracle",
                "sample": f"{n_thr} (layer, KV head)s of {wl.name}, the whole step each "
                          f"(FPS over W={wl.W}, scoring all L={wl.L} keys, top-K, compaction), "
@@ -457,11 +472,9 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": wl.name, "n_layers": wl.n_layers, "n_q_heads": wl.n_q_heads,
-                   "n_kv_heads": wl.n_kv_heads, "head_dim": wl.head_dim, "L": wl.L, "R": wl.R,
-                   "M": wl.M, "K": wl.K, "W": wl.W,
-                   "l2": "inputs larger than L2 (K/V cache %.1f GB per step)"
-                         % (2 * inp.k.numel() * inp.k.element_size() / 1e9)},
+        "config": dict(workload_config(wl, args),
+                       l2="inputs larger than L2 (K/V cache %.1f GB per step)"
+                          % (2 * inp.k.numel() * inp.k.element_size() / 1e9)),
         "step_us": ms * 1e3,
         "pct_roofline": 100.0 * t_roof / (ms / 1e3),
         "t_roof_us": t_roof * 1e6,

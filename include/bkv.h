@@ -65,6 +65,12 @@ typedef enum {
 
 typedef enum { BKV_F32 = 0, BKV_BF16 = 1 } bkv_dtype;
 
+/* How the per-row softmax probabilities p_oj of a KV head's observation rows
+ * become one score per key (Table 2 of the BeaconKV page compares the two):
+ *   BKV_AGG_MAX   s_j = max over the rows o of p_oj   (the method's choice)
+ *   BKV_AGG_MEAN  s_j = mean over the rows o of p_oj  (the ablation) */
+typedef enum { BKV_AGG_MAX = 0, BKV_AGG_MEAN = 1 } bkv_aggregate;
+
 /* Geometry shared by a KV cache and the query tensors that go with it. */
 typedef struct {
   int32_t n_layers;
@@ -93,6 +99,16 @@ bkv_status bkv_score(const bkv_cache_desc *desc, const void *k, int64_t L,
                      const void *recent_q, int32_t R, const void *beacons,
                      int32_t n_beacons, int32_t M, float scale, float *scores,
                      void *workspace, size_t workspace_bytes, void *stream);
+
+/* The same scores with mean aggregation (Table 2 "Mean"): arguments, layout
+ * and requirements as bkv_score, and
+ *   scores    device out, f32 [Ly][Hkv][L]: s[j] = the mean over the KV
+ *             head's G*(R+n_beacons) observation rows of that row's softmax
+ *             at j (each row's softmax sums to 1 over j, so s sums to 1). */
+bkv_status bkv_score_mean(const bkv_cache_desc *desc, const void *k, int64_t L,
+                          const void *recent_q, int32_t R, const void *beacons,
+                          int32_t n_beacons, int32_t M, float scale, float *scores,
+                          void *workspace, size_t workspace_bytes, void *stream);
 
 /* Top-K budget selection (Fig. 5(c); Table 1 "maximum KV cache budget").
  *   scores  device, f32 [n_rows][L] (any finite values)
@@ -158,18 +174,22 @@ typedef struct {
   void *stream;
   /* Optional tracing: NULL, or BKV_STEP_EVENTS cudaEvent_t handles (as void*)
    * that the step records on `stream` at its phase boundaries: [0] start,
-   * [1] after Continual FPS, [2] after the row statistics, [3] after the max
+   * [1] after Continual FPS, [2] after the row statistics, [3] after the
    * aggregation, [4] after top-K, [5] after compaction.  A skipped phase
    * records its event at once. */
   void **phase_events;
+  int32_t aggregate;           /* bkv_aggregate; 0 (a zeroed struct) = max */
 } bkv_step_args;
 
 #define BKV_STEP_EVENTS 6
 
 /* The periodic compression step: when W > 0, Continual FPS updates the
  * beacons first (a reading: the page only shows the beacons being used for
- * scoring); then scoring with the (updated) beacons, top-K and compaction
- * into the destination cache.  When K >= L every row is kept and copied.
+ * scoring); then scoring with the (updated) beacons, aggregated as
+ * args->aggregate says, top-K and compaction into the destination cache.
+ * When K >= L every row is kept and copied.  scores_out holds bkv_score's
+ * (max) or bkv_score_mean's (mean) scores; an aggregate other than the two
+ * values of bkv_aggregate is BKV_ERR_INVALID_ARG.
  *   n_beacons_out  host out (optional): beacons valid after the step
  *   new_len        host out (optional): min(K, L) */
 bkv_status bkv_compress_step(const bkv_step_args *args, int32_t *n_beacons_out,

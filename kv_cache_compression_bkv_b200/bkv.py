@@ -19,12 +19,13 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libbkv.so")
 
 BKV_F32, BKV_BF16 = 0, 1
+AGGREGATE = {"max": 0, "mean": 1}   # bkv_aggregate
 STATUS = {0: "BKV_OK", 1: "BKV_ERR_INVALID_ARG", 2: "BKV_ERR_UNSUPPORTED",
           3: "BKV_ERR_WORKSPACE", 4: "BKV_ERR_CUDA", 5: "BKV_ERR_TIMEOUT",
           6: "BKV_ERR_DEVICE_ASSERT"}
 EXPORTS = ("bkv_workspace_size", "bkv_score", "bkv_select_topk", "bkv_compact",
            "bkv_update_beacons", "bkv_compress_step", "bkv_read_device_status",
-           "bkv_status_string", "bkv_score_noalloc")
+           "bkv_status_string", "bkv_score_noalloc", "bkv_score_mean")
 SCORE_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -51,7 +52,8 @@ class StepArgs(ctypes.Structure):
                 ("scores_out", ctypes.c_void_p), ("idx_out", ctypes.c_void_p),
                 ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
                 ("stream", ctypes.c_void_p),
-                ("phase_events", ctypes.POINTER(ctypes.c_void_p))]
+                ("phase_events", ctypes.POINTER(ctypes.c_void_p)),
+                ("aggregate", ctypes.c_int32)]
 
 STEP_EVENTS = 6
 
@@ -76,6 +78,7 @@ def _load() -> ctypes.CDLL:
         "bkv_read_device_status": ([P, ctypes.POINTER(I32)], ctypes.c_int),
         "bkv_status_string": ([ctypes.c_int], ctypes.c_char_p),
         "bkv_score_noalloc": ([D, P, I64, P, I32, P, I32, I32, F, P, P], ctypes.c_int),
+        "bkv_score_mean": ([D, P, I64, P, I32, P, I32, I32, F, P, P, SZ, P], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -150,6 +153,16 @@ def bkv_score(geom: Geometry, k, L: int, recent_q, R: int, beacons, n_beacons: i
                          _stream(stream)), "bkv_score")
 
 
+def bkv_score_mean(geom: Geometry, k, L: int, recent_q, R: int, beacons, n_beacons: int,
+                   M: int, scale: float, scores, workspace, stream=None) -> None:
+    """bkv_score with mean instead of max aggregation over the observation rows."""
+    d = geom.desc()
+    _check(LIB.bkv_score_mean(ctypes.byref(d), _ptr(k), L, _ptr(recent_q), R, _ptr(beacons),
+                              n_beacons, M, scale, _ptr(scores), _ptr(workspace),
+                              0 if workspace is None else workspace.numel() * workspace.element_size(),
+                              _stream(stream)), "bkv_score_mean")
+
+
 def bkv_score_noalloc(geom: Geometry, k, L: int, recent_q, R: int, beacons, n_beacons: int,
                       M: int, scale: float, scores, stream=None) -> None:
     """bkv_score on the library's built-in scratch array, for callers that
@@ -190,11 +203,12 @@ def bkv_update_beacons(geom: Geometry, beacons_in, n_beacons_in: int, M: int, wi
 def bkv_compress_step(geom: Geometry, k, v, L: int, K: int, recent_q, R: int, beacons_in,
                       n_beacons_in: int, M: int, window, W: int, beacons_out, scale: float,
                       dst: Geometry, k_dst, v_dst, scores_out=None, idx_out=None,
-                      workspace=None, stream=None, phase_events=None) -> tuple[int, int]:
+                      workspace=None, stream=None, phase_events=None,
+                      aggregate: str = "max") -> tuple[int, int]:
     """One whole compression step; returns (beacons valid after, new cache length).
 
     phase_events: optional list of STEP_EVENTS torch.cuda.Event (timing enabled)
-    recorded at the step's phase boundaries.
+    recorded at the step's phase boundaries.  aggregate: "max" or "mean".
     """
     a = StepArgs()
     a.cache = geom.desc()
@@ -211,6 +225,7 @@ def bkv_compress_step(geom: Geometry, k, v, L: int, K: int, recent_q, R: int, be
     a.workspace = _ptr(workspace)
     a.workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     a.stream = _stream(stream)
+    a.aggregate = AGGREGATE[aggregate]
     if phase_events is not None:
         if len(phase_events) != STEP_EVENTS:
             raise ValueError(f"phase_events needs {STEP_EVENTS} events")

@@ -122,12 +122,12 @@ bkv_status check_score_args(const bkv_cache_desc *d, const void *k, long long L,
 
 // Scoring into the workspace: c and ypart; returns the geometry used.
 bkv_status run_score(const ScoreGeom &g, int dtype, const void *k, const void *recent,
-                     const void *beacons, const ScoreWorkspace &w, cudaStream_t s) {
+                     const void *beacons, const ScoreWorkspace &w, bool mean, cudaStream_t s) {
   bkv_status st;
   if (dtype == BKV_BF16) {
     st = launch_score_rowstats_tc(g, k, recent, beacons, w.c, s);
     if (st != BKV_OK) return st;
-    return launch_score_colmax_tc(g, k, recent, beacons, w.c, w.ypart, s);
+    return launch_score_colmax_tc(g, k, recent, beacons, w.c, w.ypart, mean, s);
   }
   st = launch_score_rowstats_simt(g, static_cast<const float *>(k),
                                   static_cast<const float *>(recent),
@@ -135,15 +135,35 @@ bkv_status run_score(const ScoreGeom &g, int dtype, const void *k, const void *r
   if (st != BKV_OK) return st;
   return launch_score_colmax_simt(g, static_cast<const float *>(k),
                                   static_cast<const float *>(recent),
-                                  static_cast<const float *>(beacons), w.c, w.ypart, s);
+                                  static_cast<const float *>(beacons), w.c, w.ypart, mean, s);
 }
 
-SelectInput score_select_input(const ScoreGeom &g, const ScoreWorkspace &w) {
+SelectInput score_select_input(const ScoreGeom &g, const ScoreWorkspace &w, bool mean) {
   SelectInput in;
   in.src = w.ypart;
   in.n_parts = g.n_groups;
   in.part_stride = static_cast<size_t>(g.n_heads()) * static_cast<size_t>(g.L);
+  in.mean = mean ? 1 : 0;
+  in.inv_count = 1.0f / static_cast<float>(g.n_obs);
   return in;
+}
+
+bkv_status score_entry(const bkv_cache_desc *desc, const void *k, int64_t L,
+                       const void *recent_q, int32_t R, const void *beacons, int32_t n_beacons,
+                       int32_t M, float scale, float *scores, void *workspace,
+                       size_t workspace_bytes, void *stream, bool mean) {
+  bkv_status st = check_score_args(desc, k, L, recent_q, R, beacons, n_beacons, M);
+  if (st != BKV_OK) return st;
+  if (!scores || !aligned16(scores) || !std::isfinite(scale) || scale < 0.f)
+    return BKV_ERR_INVALID_ARG;
+  const ScoreGeom g = make_score_geom(desc, L, R, n_beacons, M, scale);
+  if (!workspace || !aligned16(workspace) || workspace_bytes < score_workspace_bytes(g))
+    return BKV_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const ScoreWorkspace w = carve_score_workspace(g, workspace);
+  st = run_score(g, desc->dtype, k, recent_q, beacons, w, mean, s);
+  if (st != BKV_OK) return st;
+  return launch_finalize_scores(score_select_input(g, w, mean), g.n_heads(), L, scores, s);
 }
 
 }  // namespace
@@ -183,18 +203,16 @@ size_t bkv_workspace_size(const bkv_cache_desc *desc, int64_t L, int32_t R, int3
 bkv_status bkv_score(const bkv_cache_desc *desc, const void *k, int64_t L, const void *recent_q,
                      int32_t R, const void *beacons, int32_t n_beacons, int32_t M, float scale,
                      float *scores, void *workspace, size_t workspace_bytes, void *stream) {
-  bkv_status st = check_score_args(desc, k, L, recent_q, R, beacons, n_beacons, M);
-  if (st != BKV_OK) return st;
-  if (!scores || !aligned16(scores) || !std::isfinite(scale) || scale < 0.f)
-    return BKV_ERR_INVALID_ARG;
-  const ScoreGeom g = make_score_geom(desc, L, R, n_beacons, M, scale);
-  if (!workspace || !aligned16(workspace) || workspace_bytes < score_workspace_bytes(g))
-    return BKV_ERR_WORKSPACE;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const ScoreWorkspace w = carve_score_workspace(g, workspace);
-  st = run_score(g, desc->dtype, k, recent_q, beacons, w, s);
-  if (st != BKV_OK) return st;
-  return launch_finalize_scores(score_select_input(g, w), g.n_heads(), L, scores, s);
+  return score_entry(desc, k, L, recent_q, R, beacons, n_beacons, M, scale, scores, workspace,
+                     workspace_bytes, stream, false);
+}
+
+bkv_status bkv_score_mean(const bkv_cache_desc *desc, const void *k, int64_t L,
+                          const void *recent_q, int32_t R, const void *beacons,
+                          int32_t n_beacons, int32_t M, float scale, float *scores,
+                          void *workspace, size_t workspace_bytes, void *stream) {
+  return score_entry(desc, k, L, recent_q, R, beacons, n_beacons, M, scale, scores, workspace,
+                     workspace_bytes, stream, true);
 }
 
 bkv_status bkv_select_topk(const float *scores, int32_t n_rows, int64_t L, int64_t K,
@@ -204,7 +222,7 @@ bkv_status bkv_select_topk(const float *scores, int32_t n_rows, int64_t L, int64
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (K >= L) return launch_iota_rows(idx, n_rows, L, s);
   if (workspace_bytes < select_workspace_bytes(n_rows, L)) return BKV_ERR_WORKSPACE;
-  SelectInput in{scores, 1, 0};
+  SelectInput in{scores, 1, 0, 0, 1.f};
   return launch_select_topk(in, n_rows, L, K, idx, nullptr, workspace, workspace_bytes, s);
 }
 
@@ -282,6 +300,8 @@ bkv_status bkv_compress_step(const bkv_step_args *a, int32_t *n_beacons_out, int
                                    nb_used > 0 ? score_beacons : nullptr, nb_used, a->M);
   if (st != BKV_OK) return st;
   if (a->K < 1 || !a->v || !std::isfinite(a->scale) || a->scale < 0.f) return BKV_ERR_INVALID_ARG;
+  if (a->aggregate != BKV_AGG_MAX && a->aggregate != BKV_AGG_MEAN) return BKV_ERR_INVALID_ARG;
+  const bool mean = a->aggregate == BKV_AGG_MEAN;
   if (update) {
     if (a->n_beacons_in < 0 || a->n_beacons_in > a->M || !a->beacons_out ||
         (a->n_beacons_in > 0 && !a->beacons_in))
@@ -347,7 +367,7 @@ bkv_status bkv_compress_step(const bkv_step_args *a, int32_t *n_beacons_out, int
       st = launch_score_rowstats_tc(g, a->k, a->recent_q, bq, w.c, s);
       if (st != BKV_OK) return st;
       if (!mark(2)) return BKV_ERR_CUDA;
-      st = launch_score_colmax_tc(g, a->k, a->recent_q, bq, w.c, w.ypart, s);
+      st = launch_score_colmax_tc(g, a->k, a->recent_q, bq, w.c, w.ypart, mean, s);
     } else {
       st = launch_score_rowstats_simt(g, static_cast<const float *>(a->k),
                                       static_cast<const float *>(a->recent_q),
@@ -356,14 +376,14 @@ bkv_status bkv_compress_step(const bkv_step_args *a, int32_t *n_beacons_out, int
       if (!mark(2)) return BKV_ERR_CUDA;
       st = launch_score_colmax_simt(g, static_cast<const float *>(a->k),
                                     static_cast<const float *>(a->recent_q),
-                                    static_cast<const float *>(bq), w.c, w.ypart, s);
+                                    static_cast<const float *>(bq), w.c, w.ypart, mean, s);
     }
     if (st != BKV_OK) return st;
   } else if (!mark(2)) {
     return BKV_ERR_CUDA;
   }
   if (!mark(3)) return BKV_ERR_CUDA;
-  const SelectInput in = score_select_input(g, w);
+  const SelectInput in = score_select_input(g, w, mean);
   const bool copy_all = keep >= a->L;
   if (!copy_all) {
     st = launch_select_topk(in, g.n_heads(), a->L, keep, idx, a->scores_out, sel_ws, sel_b, s);

@@ -37,7 +37,8 @@ void finish_score_geom(ScoreGeom *g);
 // Workspace sections of the scoring passes.
 struct ScoreWorkspace {
   float *c;      // [n_heads][n_obs_pad]  row normalisers (natural log units)
-  float *ypart;  // [n_groups][n_heads][L] max over a group of (x - c)
+  float *ypart;  // [n_groups][n_heads][L] per group of rows: max of (x - c)
+                 // (max aggregation) or sum of exp(x - c) (mean aggregation)
 };
 size_t score_workspace_bytes(const ScoreGeom &g);
 ScoreWorkspace carve_score_workspace(const ScoreGeom &g, void *ws);
@@ -46,31 +47,35 @@ ScoreWorkspace carve_score_workspace(const ScoreGeom &g, void *ws);
 bkv_status launch_score_rowstats_tc(const ScoreGeom &g, const void *k, const void *recent,
                                     const void *beacons, float *c, cudaStream_t stream);
 bkv_status launch_score_colmax_tc(const ScoreGeom &g, const void *k, const void *recent,
-                                  const void *beacons, const float *c, float *ypart,
+                                  const void *beacons, const float *c, float *ypart, bool mean,
                                   cudaStream_t stream);
 
 // ---- score_simt.cu: f32, head_dim <= 128 (multiple of 4), CUDA cores
 bkv_status launch_score_rowstats_simt(const ScoreGeom &g, const float *k, const float *recent,
                                       const float *beacons, float *c, cudaStream_t stream);
 bkv_status launch_score_colmax_simt(const ScoreGeom &g, const float *k, const float *recent,
-                                    const float *beacons, const float *c, float *ypart,
+                                    const float *beacons, const float *c, float *ypart, bool mean,
                                     cudaStream_t stream);
 
 // ---- select_topk.cu
-// Selection input: per row r and position j, the key is
-//   max over p < n_parts of  src[p * part_stride + r * L + j].
-// When s_out is given, exp(key) is also written to s_out[r * L + j] (used when
-// src holds log-domain partial scores).
+// Selection input: per row r and position j, with v_p = src[p * part_stride +
+// r * L + j] for p < n_parts, the key is
+//   mean == 0:  max_p v_p                 (log-domain partial maxima)
+//   mean != 0:  inv_count * sum_p v_p     (partial sums of probabilities)
+// When s_out is given, the score is also written to s_out[r * L + j]: exp(key)
+// for the max form, the key itself for the mean form.
 struct SelectInput {
   const float *src;
   int n_parts;
   size_t part_stride;
+  int mean;
+  float inv_count;
 };
 size_t select_workspace_bytes(int n_rows, long long L);
 bkv_status launch_select_topk(const SelectInput &in, int n_rows, long long L, long long K,
                               int32_t *idx, float *s_out, void *ws, size_t ws_bytes,
                               cudaStream_t stream);
-// s[r][j] = exp(max_p src[p][r][j]) for every row and position.
+// s[r][j] = the score of SelectInput's comment, for every row and position.
 bkv_status launch_finalize_scores(const SelectInput &in, int n_rows, long long L, float *s,
                                   cudaStream_t stream);
 // idx[r][i] = i for i < n.

@@ -1,9 +1,10 @@
-// score_simt.cu -- attention-based scores with max aggregation on the CUDA
-// cores, for f32 caches (small correctness workloads; BeaconKV Fig. 5(b)/(c)).
-// Same two passes as the tensor-core path:
+// score_simt.cu -- attention-based scores with max (or mean) aggregation on
+// the CUDA cores, for f32 caches (small correctness workloads; BeaconKV
+// Fig. 5(b)/(c), Table 2).  Same two passes as the tensor-core path:
 //   pass 1: c_o = log sum_j exp(scale * q_o . k_j), one warp per observation
 //           row, an online (max, sum) per lane, merged across the warp;
-//   pass 2: y_j = max_o (scale * q_o . k_j - c_o), one thread per key.
+//   pass 2: y_j = max_o (scale * q_o . k_j - c_o), one thread per key (for
+//           the mean: y_j = sum_o exp(scale * q_o . k_j - c_o)).
 #include <cuda_runtime.h>
 
 #include "bkv_internal.h"
@@ -81,6 +82,9 @@ __global__ void __launch_bounds__(256) rowstats_simt_kernel(const ScoreGeom g,
 constexpr int kKeysPerBlock = 128;
 constexpr int kObsChunk = 32;
 
+// Per key j: max over the rows of (x_oj - c_o), or with kMean the sum over
+// the rows of exp(x_oj - c_o).
+template <bool kMean>
 __global__ void __launch_bounds__(kKeysPerBlock) colmax_simt_kernel(
     const ScoreGeom g, const float *__restrict__ k, const float *__restrict__ recent,
     const float *__restrict__ beacons, const float *__restrict__ c_in,
@@ -92,7 +96,7 @@ __global__ void __launch_bounds__(kKeysPerBlock) colmax_simt_kernel(
   const int d = g.head_dim;
   const long long j = static_cast<long long>(blockIdx.x) * kKeysPerBlock + threadIdx.x;
   const float *kj = k + (static_cast<size_t>(head) * g.cap + (j < g.L ? j : 0)) * d;
-  float y = -INFINITY;
+  float y = kMean ? 0.f : -INFINITY;
   for (int o0 = 0; o0 < g.n_obs; o0 += kObsChunk) {
     const int n = min(kObsChunk, g.n_obs - o0);
     __syncthreads();
@@ -103,7 +107,10 @@ __global__ void __launch_bounds__(kKeysPerBlock) colmax_simt_kernel(
     for (int r = threadIdx.x; r < n; r += blockDim.x)
       c_sh[r] = c_in[static_cast<size_t>(head) * g.n_obs_pad + o0 + r];
     __syncthreads();
-    for (int r = 0; r < n; ++r) y = fmaxf(y, g.scale * dot_f32(q_sh[r], kj, d) - c_sh[r]);
+    for (int r = 0; r < n; ++r) {
+      const float a = g.scale * dot_f32(q_sh[r], kj, d) - c_sh[r];
+      y = kMean ? y + expf(a) : fmaxf(y, a);
+    }
   }
   if (j < g.L) ypart[static_cast<size_t>(head) * g.L + j] = y;
 }
@@ -119,9 +126,12 @@ bkv_status launch_score_rowstats_simt(const ScoreGeom &g, const float *k, const 
 
 bkv_status launch_score_colmax_simt(const ScoreGeom &g, const float *k, const float *recent,
                                     const float *beacons, const float *c, float *ypart,
-                                    cudaStream_t stream) {
+                                    bool mean, cudaStream_t stream) {
   dim3 grid(static_cast<unsigned>((g.L + kKeysPerBlock - 1) / kKeysPerBlock), g.n_heads());
-  colmax_simt_kernel<<<grid, kKeysPerBlock, 0, stream>>>(g, k, recent, beacons, c, ypart);
+  if (mean)
+    colmax_simt_kernel<true><<<grid, kKeysPerBlock, 0, stream>>>(g, k, recent, beacons, c, ypart);
+  else
+    colmax_simt_kernel<false><<<grid, kKeysPerBlock, 0, stream>>>(g, k, recent, beacons, c, ypart);
   return cudaGetLastError() == cudaSuccess ? BKV_OK : BKV_ERR_CUDA;
 }
 

@@ -1,5 +1,5 @@
-// score_tc.cu -- attention-based scores with max aggregation on the sm_100a
-// tensor cores (BeaconKV, Fig. 5(b)/(c); Table 2 "Max").
+// score_tc.cu -- attention-based scores with max (or mean) aggregation on the
+// sm_100a tensor cores (BeaconKV, Fig. 5(b)/(c); Table 2 "Max" and "Mean").
 //
 // For one (layer, KV head) with observation rows q_o and keys k_j (bf16,
 // head_dim 128) the scores are
@@ -16,7 +16,9 @@
 //     K=16 step of the same MMA: every key carries a block (1, 1, 1, 0, ...)
 //     and every observation row (-c_hi, -c_mid, -c_lo, 0, ...), the three
 //     bf16 parts of c_o / scale.  TMEM lane = key, so each epilogue thread owns
-//     one key and takes the max over its columns in registers.
+//     one key and takes the max over its columns in registers.  The mean
+//     variant sums exp(scale * acc) over the columns instead (s_j is that sum
+//     over all rows divided by their count).
 //
 // Both passes: warp 0 issues TMA loads of the key tiles (128-byte swizzle, no
 // multicast) into a ring of shared-memory stages; warp 1 allocates TMEM and
@@ -97,18 +99,20 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
                      __uint_as_float(__float_as_uint(p.y) + ey));
 }
 
-// Sum of 2^(v[i] * kz - m) over one 32-column chunk.  The first kPolyPairs
-// pairs go through exp2_poly2 (FMA pipe), the rest through ex2.approx (MUFU),
-// so that both pipes share the load.
+// Sum of 2^(v[i] * kz - m) over one chunk of N (32 or 16) columns.  About
+// 7 of every 16 pairs go through exp2_poly2 (FMA pipe), the rest through
+// ex2.approx (MUFU), so that both pipes share the load.
 constexpr int kPolyPairs = 7;
-__device__ __forceinline__ float chunk_exp_sum(const float (&v)[32], float kz, float m) {
+template <int N>
+__device__ __forceinline__ float chunk_exp_sum(const float (&v)[N], float kz, float m) {
+  constexpr int kPoly = (kPolyPairs * N + 16) / 32;
   const float2 kz2 = make_float2(kz, kz), nm2 = make_float2(-m, -m);
   float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-  for (int p = 0; p < 16; ++p) {
+  for (int p = 0; p < N / 2; ++p) {
     const float2 a = __ffma2_rn(make_float2(v[2 * p], v[2 * p + 1]), kz2, nm2);
     float2 e;
-    if (p < kPolyPairs) {
+    if (p < kPoly) {
       e = exp2_poly2(a);
     } else {
       e.x = ex2_approx(a.x);
@@ -348,29 +352,39 @@ __global__ void __launch_bounds__(kP1Threads, 1)
 }
 
 // ------------------------------------------------------------------ pass 2
+// Max aggregation: two epilogue warpgroups, one per column sub-chunk.  Mean
+// aggregation (an exp per element instead of a max) splits each sub-chunk's
+// 32-column pieces between two warpgroups, four in all.
 constexpr int kP2Keys = 128;
-constexpr int kP2Threads = 384;  // warp 0 TMA, warp 1 MMA, warps 4..7 / 8..11 epilogue
-                                 // warpgroups for the two column sub-chunks
 constexpr int kP2TileBytes = kP2Keys * kRowBytes;  // 32 KB
-constexpr int kP2SmallBytes = 256 + 2 * 128 * 4;  // barriers + TMEM slot, exchange
 constexpr int kP2ExtraRowBytes = 32;              // the extra K=16 step, 32-byte swizzle
 
-__host__ __device__ constexpr int p2_smem_bytes(int rows_pad, int stages) {
-  return kP2SmallBytes + 1024 + rows_pad * kRowBytes + stages * kP2TileBytes +
+__host__ __device__ constexpr int p2_epi_warpgroups(bool mean) { return mean ? 4 : 2; }
+// warp 0 TMA, warp 1 MMA, warps 4.. the epilogue warpgroups
+__host__ __device__ constexpr int p2_threads(bool mean) { return 128 + 128 * p2_epi_warpgroups(mean); }
+// barriers + TMEM slot, then [2][warpgroups - 1][128] partials for the combine
+__host__ __device__ constexpr int p2_small_bytes(bool mean) {
+  return 256 + 2 * (p2_epi_warpgroups(mean) - 1) * 128 * 4;
+}
+__host__ __device__ constexpr int p2_smem_bytes(int rows_pad, int stages, bool mean) {
+  return p2_small_bytes(mean) + 1024 + rows_pad * kRowBytes + stages * kP2TileBytes +
          kP2Keys * kP2ExtraRowBytes + rows_pad * kP2ExtraRowBytes;
 }
 
-__global__ void __launch_bounds__(kP2Threads, 1)
+template <bool kMean>
+__global__ void __launch_bounds__(p2_threads(kMean), 1)
     score_colmax_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreGeom g,
                         const uint16_t *__restrict__ recent, const uint16_t *__restrict__ beacons,
                         const float *__restrict__ c_in, float *__restrict__ ypart, int n_chunks,
                         int chunk_tiles, int n_stages) {
+  constexpr int kEpiWG = p2_epi_warpgroups(kMean);
+  constexpr int kSplit = kEpiWG / 2;  // warpgroups per column sub-chunk
   extern __shared__ uint8_t smem_raw[];
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem_raw);  // 16 barriers
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem_raw + 128);
-  float *ybuf = reinterpret_cast<float *>(smem_raw + 256);  // [2][128] sub-chunk 1 maxima
+  float *ybuf = reinterpret_cast<float *>(smem_raw + 256);  // partials of warpgroups 1..
   const uint32_t raw_base = smem_u32(smem_raw);
-  const uint32_t tile_base = (raw_base + kP2SmallBytes + 1023u) & ~1023u;
+  const uint32_t tile_base = (raw_base + p2_small_bytes(kMean) + 1023u) & ~1023u;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int bid = blockIdx.x;
@@ -410,7 +424,7 @@ __global__ void __launch_bounds__(kP2Threads, 1)
     }
     for (int u = 0; u < 2; ++u) {
       mbar_init(tfull0 + 8 * u, 1);
-      mbar_init(tempty0 + 8 * u, 4);  // one arrive per warp of its warpgroup
+      mbar_init(tempty0 + 8 * u, 4 * kSplit);  // one arrive per warp reading it
     }
     mbar_init(done, 1);
     fence_barrier_init();
@@ -508,70 +522,92 @@ __global__ void __launch_bounds__(kP2Threads, 1)
       mbar_wait(done, 0, kWhereP2Drain);
     }
   } else if (warp >= 4) {
-    // warpgroup u reduces column sub-chunk u: per key (TMEM lane) the max over
-    // its observation rows of acc - c_o / scale; sub-chunk 1's maxima reach
-    // warpgroup 0 through shared memory
-    const int u = (warp - 4) >> 2;
+    // Warpgroup e = u * kSplit + h reads column sub-chunk u, its 32-column
+    // pieces h, h + kSplit, ...; per key (TMEM lane) it reduces
+    // acc = q . k - c_o / scale over them: the max (max aggregation) or the
+    // sum of exp(scale * acc) (mean).  The partials of warpgroups 1.. reach
+    // warpgroup 0 through shared memory.
+    const int e = (warp - 4) >> 2;
+    const int u = e / kSplit, h = e - u * kSplit;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;  // key within the tile
+    const int n_active = n_sub * kSplit;  // warpgroups with columns to read
+    const float kz = g.scale * kLog2e;
     float *yout = ypart + (static_cast<size_t>(gi) * g.n_heads() + head) * static_cast<size_t>(L);
     if (u < n_sub) {
       const int Nu = u == 0 ? N0 : N1;
       const int n32 = Nu >> 5;
+      const int n_mine = n32 > h ? (n32 - h + kSplit - 1) / kSplit : 0;
+      const bool tail16 = (Nu & 16) && (n32 % kSplit) == h;  // Nu is a multiple of 16
       bool ok = true;  // warp-uniform; after a timeout only the barriers remain
       for (int it = 0; it < n_tiles; ++it) {
-        float y0 = -INFINITY, y1 = -INFINITY;
+        float y0 = kMean ? 0.f : -INFINITY, y1 = y0;
         if (ok && !mbar_wait_warp(tfull0 + 8 * u, it & 1, kWhereP2Epi)) ok = false;
         if (ok) {
           tc_fence_after();
           const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + u * 256;
-          auto reduce32 = [&](const float (&v)[32], int) {
+          auto piece = [&](int i) { return taddr + static_cast<uint32_t>((h + i * kSplit) * 32); };
+          auto reduce32 = [&](const float (&v)[32]) {
+            if (kMean) {
+              y0 += chunk_exp_sum(v, kz, 0.f);
+            } else {
 #pragma unroll
-            for (int i = 0; i < 32; i += 4) {
-              y0 = max3f(y0, v[i], v[i + 1]);
-              y1 = max3f(y1, v[i + 2], v[i + 3]);
+              for (int i = 0; i < 32; i += 4) {
+                y0 = max3f(y0, v[i], v[i + 1]);
+                y1 = max3f(y1, v[i + 2], v[i + 3]);
+              }
             }
           };
-          // two TMEM loads in flight: chunk c+1 lands while chunk c is reduced
+          // two TMEM loads in flight: piece i+1 lands while piece i is reduced
           float va[32], vb[32];
-          int c = 0;
-          if (n32 > 0) {
-            tmem_ld_32x32b_x32(taddr, va);
+          int i = 0;
+          if (n_mine > 0) {
+            tmem_ld_32x32b_x32(piece(0), va);
             tmem_ld_wait_regs(va);
           }
 #pragma unroll 1
-          for (; c + 2 <= n32; c += 2) {
-            tmem_ld_32x32b_x32(taddr + (c + 1) * 32, vb);
-            reduce32(va, c * 32);
+          for (; i + 2 <= n_mine; i += 2) {
+            tmem_ld_32x32b_x32(piece(i + 1), vb);
+            reduce32(va);
             tmem_ld_wait_regs(vb);
-            if (c + 2 < n32) tmem_ld_32x32b_x32(taddr + (c + 2) * 32, va);
-            reduce32(vb, (c + 1) * 32);
-            if (c + 2 < n32) tmem_ld_wait_regs(va);
+            if (i + 2 < n_mine) tmem_ld_32x32b_x32(piece(i + 2), va);
+            reduce32(vb);
+            if (i + 2 < n_mine) tmem_ld_wait_regs(va);
           }
-          if (c < n32) reduce32(va, c * 32);
-          if (Nu & 16) {  // Nu is a multiple of 16
+          if (i < n_mine) reduce32(va);
+          if (tail16) {
             float v[16];
             tmem_ld_32x32b_x16(taddr + n32 * 32, v);
             tmem_ld_wait_regs(v);
+            if (kMean) {
+              y1 += chunk_exp_sum(v, kz, 0.f);
+            } else {
 #pragma unroll
-            for (int i = 0; i < 16; i += 4) {
-              y0 = max3f(y0, v[i], v[i + 1]);
-              y1 = max3f(y1, v[i + 2], v[i + 3]);
+              for (int t = 0; t < 16; t += 4) {
+                y0 = max3f(y0, v[t], v[t + 1]);
+                y1 = max3f(y1, v[t + 2], v[t + 3]);
+              }
             }
           }
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(tempty0 + 8 * u);
         }
-        float y = fmaxf(y0, y1);
-        if (n_sub == 2) {
-          if (u == 1) ybuf[(it & 1) * 128 + row] = y;
-          named_barrier_sync(1, 256);
-          if (u == 0) y = fmaxf(y, ybuf[(it & 1) * 128 + row]);
+        float y = kMean ? y0 + y1 : fmaxf(y0, y1);
+        if (n_active > 1) {
+          float *slot = ybuf + (it & 1) * (kEpiWG - 1) * 128;
+          if (e > 0) slot[(e - 1) * 128 + row] = y;
+          named_barrier_sync(1, 128 * n_active);
+          if (e == 0) {
+            for (int f = 1; f < n_active; ++f) {
+              const float t = slot[(f - 1) * 128 + row];
+              y = kMean ? y + t : fmaxf(y, t);
+            }
+          }
         }
-        if (u == 0 && ok) {
+        if (e == 0 && ok) {
           const long long j = static_cast<long long>(t0 + it) * kP2Keys + row;
-          if (j < L) yout[j] = y * g.scale;
+          if (j < L) yout[j] = kMean ? y : y * g.scale;
         }
       }
     }
@@ -632,7 +668,7 @@ bkv_status launch_score_rowstats_tc(const ScoreGeom &g, const void *k, const voi
 }
 
 bkv_status launch_score_colmax_tc(const ScoreGeom &g, const void *k, const void *recent,
-                                  const void *beacons, const float *c, float *ypart,
+                                  const void *beacons, const float *c, float *ypart, bool mean,
                                   cudaStream_t stream) {
   CUtensorMap map;
   if (!make_key_map(&map, k, g, kP2Keys)) return BKV_ERR_CUDA;
@@ -643,11 +679,13 @@ bkv_status launch_score_colmax_tc(const ScoreGeom &g, const void *k, const void 
   }
   constexpr int kSmemLimit = 232448;  // 227 KB opt-in per block on sm_100
   int stages = 4;
-  while (stages > 2 && p2_smem_bytes(max_rows_pad, stages) > kSmemLimit) --stages;
-  const int smem = p2_smem_bytes(max_rows_pad, stages);
+  while (stages > 2 && p2_smem_bytes(max_rows_pad, stages, mean) > kSmemLimit) --stages;
+  const int smem = p2_smem_bytes(max_rows_pad, stages, mean);
   if (smem > kSmemLimit) return BKV_ERR_UNSUPPORTED;
-  static int attr_done[64];
-  if (!ensure_smem_limit(score_colmax_kernel, kSmemLimit, attr_done)) return BKV_ERR_CUDA;
+  static int attr_done[2][64];
+  if (!ensure_smem_limit(mean ? score_colmax_kernel<true> : score_colmax_kernel<false>,
+                         kSmemLimit, attr_done[mean ? 1 : 0]))
+    return BKV_ERR_CUDA;
   const int n_tiles = static_cast<int>((g.L + kP2Keys - 1) / kP2Keys);
   // Split the keys of a head into chunks so that the CTAs fill whole waves of
   // the SMs (one CTA per SM): the fewest chunks whose last wave is at least
@@ -676,9 +714,14 @@ bkv_status launch_score_colmax_tc(const ScoreGeom &g, const void *k, const void 
     if (fill >= 0.95) break;
   }
   const long long grid = units * n_chunks;
-  score_colmax_kernel<<<static_cast<unsigned>(grid), kP2Threads, smem, stream>>>(
-      map, g, static_cast<const uint16_t *>(recent), static_cast<const uint16_t *>(beacons), c,
-      ypart, n_chunks, chunk_tiles, stages);
+  const auto *rq = static_cast<const uint16_t *>(recent);
+  const auto *bq = static_cast<const uint16_t *>(beacons);
+  if (mean)
+    score_colmax_kernel<true><<<static_cast<unsigned>(grid), p2_threads(true), smem, stream>>>(
+        map, g, rq, bq, c, ypart, n_chunks, chunk_tiles, stages);
+  else
+    score_colmax_kernel<false><<<static_cast<unsigned>(grid), p2_threads(false), smem, stream>>>(
+        map, g, rq, bq, c, ypart, n_chunks, chunk_tiles, stages);
   return cudaGetLastError() == cudaSuccess ? BKV_OK : BKV_ERR_CUDA;
 }
 

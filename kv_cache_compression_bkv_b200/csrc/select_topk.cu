@@ -51,8 +51,17 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 
 __device__ __forceinline__ float load_key_value(const SelectInput &in, size_t off) {
   float v = in.src[off];
+  if (in.mean) {
+    for (int p = 1; p < in.n_parts; ++p) v += in.src[p * in.part_stride + off];
+    return v * in.inv_count;
+  }
   for (int p = 1; p < in.n_parts; ++p) v = fmaxf(v, in.src[p * in.part_stride + off]);
   return v;
+}
+
+// The score a key stands for: the max form keeps log-domain maxima.
+__device__ __forceinline__ float score_of_key(const SelectInput &in, float v) {
+  return in.mean ? v : expf(v);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -71,7 +80,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   for (long long j = tid; j < L; j += kThreads) {
     const float v = load_key_value(in, rbase + j);
-    if (s_out) s_out[rbase + j] = expf(v);
+    if (s_out) s_out[rbase + j] = score_of_key(in, v);
     keys[j] = order_key(v);
   }
   __syncthreads();
@@ -173,7 +182,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 __global__ void finalize_scores_kernel(const SelectInput in, size_t total, float *__restrict__ s) {
   for (size_t e = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; e < total;
        e += static_cast<size_t>(gridDim.x) * blockDim.x)
-    s[e] = expf(load_key_value(in, e));
+    s[e] = score_of_key(in, load_key_value(in, e));
 }
 
 __global__ void iota_rows_kernel(int32_t *idx, size_t total, long long n) {

@@ -238,7 +238,7 @@ def update_beacons_head(beacons, n_beacons: int, window, M: int, _lib=None):
 
 
 def compress_head(k_rows, v_rows, recent, beacons, n_beacons: int, window, M: int,
-                  K: int, scale: float | None = None, _lib=None):
+                  K: int, scale: float | None = None, aggregate: str = "max", _lib=None):
     """The whole step for one (layer, KV head).
 
     Order (a reading: the pages only show the beacons being used for scoring):
@@ -246,7 +246,8 @@ def compress_head(k_rows, v_rows, recent, beacons, n_beacons: int, window, M: in
     then scoring with the updated beacons, top-K and compaction.
     k_rows, v_rows: [L, d] (any dtype; compaction copies their bytes).
     recent: [G, R, d]; beacons: [G, M, d] (first n_beacons valid);
-    window: [G, W, d] or None.
+    window: [G, W, d] or None.  aggregate: "max" (the method) or "mean"
+    (Table 2's ablation).
     """
     G = np.asarray(recent).shape[0]
     if window is not None and np.asarray(window).shape[1] > 0:
@@ -259,7 +260,8 @@ def compress_head(k_rows, v_rows, recent, beacons, n_beacons: int, window, M: in
         n_used = beacons_used.shape[1]
     else:
         beacons_used, n_used, picks = np.asarray(beacons), n_beacons, None
-    s, c = score_head(k_rows, recent, beacons_used, n_used, scale, _lib=_lib)
+    s, c = score_head(k_rows, recent, beacons_used, n_used, scale, aggregate=aggregate,
+                      _lib=_lib)
     idx = select_topk(s, K, _lib=_lib)
     return {
         "beacons": beacons_used, "n_beacons": n_used, "picks": picks,

@@ -78,6 +78,9 @@ def pin_softmax(lib):
         np.testing.assert_allclose(s1, p[0], rtol=1e-12, atol=0)
         m = oracle.mean_aggregate(x, c, _lib=lib)
         np.testing.assert_allclose(m, p.mean(axis=0), rtol=1e-12, atol=0)
+        # a mean of distributions is a distribution, below the max aggregate
+        np.testing.assert_allclose(m.sum(), 1.0, rtol=0, atol=1e-12)
+        assert np.all(m <= s * (1 + 1e-13))
 
 
 def pin_score_head_composition(lib):
@@ -94,6 +97,8 @@ def pin_score_head_composition(lib):
     p = np.stack([softmax(0.25 * (k @ r)) for r in rows])
     np.testing.assert_allclose(s, p.max(axis=0), rtol=1e-12, atol=0)
     assert c.shape == (G * (R + nb),)
+    sm, _ = oracle.score_head(k, recent, beacons, nb, 0.25, aggregate="mean", _lib=lib)
+    np.testing.assert_allclose(sm, p.mean(axis=0), rtol=1e-12, atol=0)
 
 
 def _sorted_topk(s, K):

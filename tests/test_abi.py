@@ -46,9 +46,9 @@ def desc(Ly=2, Hq=8, Hkv=2, d=128, cap=1024, dt=bkv.BKV_BF16):
 
 
 def score(d, k=A, L=1000, recent=A, R=8, beacons=A, nb=16, M=16, scale=0.0, scores=A, ws=A,
-          ws_bytes=1 << 40):
-    return LIB.bkv_score(ctypes.byref(d) if d is not None else None, k, L, recent, R, beacons, nb,
-                         M, scale, scores, ws, ws_bytes, S)
+          ws_bytes=1 << 40, fn="bkv_score"):
+    return getattr(LIB, fn)(ctypes.byref(d) if d is not None else None, k, L, recent, R, beacons,
+                            nb, M, scale, scores, ws, ws_bytes, S)
 
 
 def test_workspace_size():
@@ -83,8 +83,9 @@ def test_workspace_size():
     (dict(ws=0), WORKSPACE),
     (dict(ws_bytes=1024), WORKSPACE),
 ])
-def test_score_rejects(kw, expect):
-    args = dict(d=desc())
+@pytest.mark.parametrize("fn", ["bkv_score", "bkv_score_mean"])
+def test_score_rejects(kw, expect, fn):
+    args = dict(d=desc(), fn=fn)
     args.update(kw)
     assert score(**args) == expect
 
@@ -183,6 +184,8 @@ def step_args(**kw):
     (dict(workspace_bytes=4096), WORKSPACE),
     (dict(workspace=None), WORKSPACE),
     (dict(W=100000), UNSUPPORTED),
+    (dict(aggregate=2), INVALID),                  # neither max nor mean
+    (dict(aggregate=-1), INVALID),
 ])
 def test_compress_step_rejects(kw, expect):
     a = step_args(**kw)
@@ -193,3 +196,25 @@ def test_compress_step_rejects(kw, expect):
 
 def test_compress_step_null():
     assert LIB.bkv_compress_step(None, None, None) == INVALID
+
+
+def test_step_args_layout_matches_the_header(tmp_path):
+    """The binding's StepArgs has the C struct's size and field offsets (gcc
+    compiles a probe against include/bkv.h on the host)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    fields = [f[0] for f in bkv.StepArgs._fields_]
+    src = tmp_path / "layout.c"
+    body = "".join(f'  printf("%zu\\n", offsetof(bkv_step_args, {f}));\n' for f in fields)
+    src.write_text("#include <stddef.h>\n#include <stdio.h>\n#include \"bkv.h\"\n"
+                   "int main(void) {\n  printf(\"%zu\\n\", sizeof(bkv_step_args));\n"
+                   + body + "  return 0;\n}\n")
+    exe = tmp_path / "layout"
+    subprocess.run([cc, "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    got = [int(x) for x in subprocess.run([str(exe)], capture_output=True, text=True,
+                                          check=True).stdout.split()]
+    assert got[0] == ctypes.sizeof(bkv.StepArgs)
+    assert got[1:] == [getattr(bkv.StepArgs, f).offset for f in fields]

@@ -96,6 +96,39 @@ def test_score_select_compact(case, dev):
             check_compaction(vd_raw[l, h], v_raw[l, h], idx_all[r], f"{case} V rows")
 
 
+@pytest.mark.parametrize("case", sorted(SCORE_CASES))
+def test_score_mean(case, dev):
+    """Mean aggregation (Table 2's ablation) against the oracle's mean, then
+    top-K on those scores; the mean of softmax rows sums to 1 over the keys."""
+    bkv, synth = _lib(), _synth()
+    wl = SCORE_CASES[case]()
+    inp = synth.make_step_inputs(wl, seed=12)
+    g = bkv.geometry_of(inp.k, wl.n_q_heads)
+    k = inp.k.to(dev)
+    rq, bq = inp.recent.to(dev), inp.beacons.to(dev)
+    H = wl.n_heads
+    scores = torch.full((wl.n_layers, wl.n_kv_heads, wl.L), -1.0, device=dev)
+    ws = torch.empty(bkv.bkv_workspace_size(g, wl.L, wl.R, wl.M, 0, wl.K), dtype=torch.uint8,
+                     device=dev)
+    bkv.bkv_score_mean(g, k, wl.L, rq if wl.R else None, wl.R, bq if wl.beacons_in else None,
+                       wl.beacons_in, wl.M, 0.0, scores, ws)
+    keep = min(wl.K, wl.L)
+    idx = torch.full((H, keep), -1, dtype=torch.int32, device=dev)
+    bkv.bkv_select_topk(scores, H, wl.L, wl.K, idx, ws)
+    torch.cuda.synchronize()
+    assert bkv.bkv_read_device_status()[0] == 0
+    s_all = scores.double().cpu().numpy()
+    idx_all = idx.cpu().numpy()
+    for l in range(wl.n_layers):
+        for h in range(wl.n_kv_heads):
+            kk, _, rr, bb, _ = synth.head_slice(inp, l, h)
+            s_ref, _ = oracle.score_head(f64(kk), f64(rr), f64(bb), wl.beacons_in,
+                                         aggregate="mean")
+            check_scores(s_all[l, h], s_ref, f"{case} mean scores l{l} h{h}")
+            assert abs(s_all[l, h].sum() - 1.0) < 1e-3, (case, l, h, s_all[l, h].sum())
+            check_topk(idx_all[l * wl.n_kv_heads + h], s_ref, wl.K, f"{case} mean top-K l{l} h{h}")
+
+
 FPS_CASES = {
     "tiny_f32": lambda: _synth().WORKLOADS["tiny"],
     "bf16_small": lambda: small(W=300, M=24, n_beacons_in=10),
@@ -130,7 +163,7 @@ def test_update_beacons(case, dev):
             check_fps(f64(U), picks, wl.M, f"{case} l{l} q{qh}")
 
 
-def _run_step(wl, inp, dev, scores=True):
+def _run_step(wl, inp, dev, scores=True, aggregate="max"):
     bkv = _lib()
     g = bkv.geometry_of(inp.k, wl.n_q_heads)
     keep = min(wl.K, wl.L)
@@ -150,7 +183,7 @@ def _run_step(wl, inp, dev, scores=True):
         g, t["k"], t["v"], wl.L, wl.K, t["recent"] if wl.R else None, wl.R,
         t["beacons"] if wl.beacons_in else None, wl.beacons_in, wl.M,
         t["window"] if wl.W else None, wl.W, out["bout"], 0.0, dst, out["kd"], out["vd"],
-        out["scores"], out["idx"], ws)
+        out["scores"], out["idx"], ws, aggregate=aggregate)
     torch.cuda.synchronize()
     assert bkv.bkv_read_device_status()[0] == 0
     assert nl == keep
@@ -158,7 +191,7 @@ def _run_step(wl, inp, dev, scores=True):
     return out, nb
 
 
-def _check_step_heads(wl, inp, out, nb, heads, what):
+def _check_step_heads(wl, inp, out, nb, heads, what, aggregate="max"):
     """Oracle comparison of whole-step outputs for the sampled (layer, KV head)s."""
     synth = _synth()
     G = wl.group
@@ -182,7 +215,8 @@ def _check_step_heads(wl, inp, out, nb, heads, what):
             continue  # near-tie in FPS: the oracle scores different beacons
         n_exact += 1
         ref = oracle.compress_head(f64(kk), f64(vv), f64(rr), f64(bb), wl.beacons_in,
-                                   f64(ww) if wl.W else None, wl.M, wl.K)
+                                   f64(ww) if wl.W else None, wl.M, wl.K,
+                                   aggregate=aggregate)
         if s_all is not None:
             check_scores(s_all[l, h], ref["scores"], f"{what} scores l{l} h{h}")
         check_topk(idx_all[l, h], ref["scores"], wl.K, f"{what} top-K l{l} h{h}")
@@ -205,6 +239,17 @@ def test_compress_step_small(case, dev):
     out, nb = _run_step(wl, inp, dev)
     heads = [(l, h) for l in range(wl.n_layers) for h in range(wl.n_kv_heads)]
     n_exact = _check_step_heads(wl, inp, out, nb, heads, case)
+    assert n_exact == len(heads), "FPS near-ties on a small case"
+
+
+@pytest.mark.parametrize("case", sorted(STEP_CASES))
+def test_compress_step_mean(case, dev):
+    """The whole step with mean aggregation."""
+    wl = STEP_CASES[case]()
+    inp = _synth().make_step_inputs(wl, seed=4)
+    out, nb = _run_step(wl, inp, dev, aggregate="mean")
+    heads = [(l, h) for l in range(wl.n_layers) for h in range(wl.n_kv_heads)]
+    n_exact = _check_step_heads(wl, inp, out, nb, heads, case + " mean", aggregate="mean")
     assert n_exact == len(heads), "FPS near-ties on a small case"
 
 
@@ -231,3 +276,19 @@ def test_full_size_sampled(name, dev):
     assert torch.equal(gathered.view(torch.int16), out["kd"].view(torch.int16))
     # kept positions are strictly ascending in every head
     assert bool((idx[..., 1:] > idx[..., :-1]).all())
+
+
+@pytest.mark.slow
+def test_full_size_sampled_mean(dev):
+    """Mean aggregation in the 14B launch configuration; sampled heads vs the oracle."""
+    synth = _synth()
+    wl = synth.WORKLOADS["qwen3_14b"]
+    inp = synth.make_step_inputs(wl, seed=5)
+    out, nb = _run_step(wl, inp, dev, aggregate="mean")
+    rng = np.random.default_rng(321)
+    heads = sorted({(int(rng.integers(wl.n_layers)), int(rng.integers(wl.n_kv_heads)))
+                    for _ in range(2)} | {(0, 0)})
+    n_exact = _check_step_heads(wl, inp, out, nb, heads, "qwen3_14b mean", aggregate="mean")
+    assert n_exact >= 1, "every sampled head hit an FPS near-tie"
+    sums = out["scores"].double().sum(-1)
+    assert bool(((sums - 1.0).abs() < 1e-3).all()), sums.flatten()[:8]
