@@ -292,6 +292,141 @@ def run_reference(args, wl, rank, world):
 
 
 # ----------------------------------------------------------------------------
+# Continual FPS against naive FPS over the whole query history (Fig. 7)
+# ----------------------------------------------------------------------------
+def fps_sweep(args, wl):
+    """Time bkv_update_beacons on the workload's query heads for Continual FPS
+    (beacons + the window since the last step) and for naive FPS over the
+    whole history of each length in --fps-sweep (no beacons).  One JSON line."""
+    from kv_cache_compression_bkv_b200 import bkv, synth
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    hist = [int(x) for x in args.fps_sweep.split(",") if x]
+    cases = [("continual", wl.beacons_in, wl.W)] + [("naive", 0, h) for h in hist]
+    w_max = max(W for _, _, W in cases)
+    Ly, Hq, d, M = wl.n_layers, wl.n_q_heads, wl.head_dim, wl.M
+    dt = wl.torch_dtype
+    # each query head's history, newest last; a window is its last W rows
+    history = torch.empty(Ly, Hq, w_max, d, dtype=dt, device=dev)
+    beacons = torch.empty(Ly, Hq, M, d, dtype=dt, device=dev)
+    for l in range(Ly):
+        for qh in range(Hq):
+            history[l, qh] = synth.queries(wl, args.seed, l, qh, w_max, 3).to(dt).to(dev)
+            b = torch.zeros(M, d)
+            if wl.beacons_in:
+                b[:wl.beacons_in] = synth.queries(wl, args.seed, l, qh, wl.beacons_in, 5)
+            beacons[l, qh] = b.to(dt).to(dev)
+    g = bkv.Geometry(Ly, Hq, wl.n_kv_heads, d, 1, dt)
+    out = []
+    for name, nb, W in cases:
+        window = history[:, :, w_max - W:].contiguous()
+        bout = torch.empty_like(beacons)
+        ws = torch.empty(max(1, bkv.bkv_workspace_size(g, 1, 0, M, W, 1)), dtype=torch.uint8,
+                         device=dev)
+        stream = torch.cuda.current_stream()
+
+        def call():
+            return bkv.bkv_update_beacons(g, beacons if nb else None, nb, M, window, W, bout,
+                                          ws, stream)
+
+        for _ in range(max(1, args.warmup)):
+            call()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = max(1, min(args.steps, 5))
+        e0.record(stream)
+        for _ in range(reps):
+            call()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        st, where = bkv.bkv_read_device_status()
+        if st != 0:
+            raise RuntimeError(f"device status {st} at {where}")
+        ms = e0.elapsed_time(e1) / reps
+        n = nb + W
+        out.append({"fps": name, "beacons_in": nb, "W": W, "union": n, "ms": ms,
+                    "union_bytes_per_step": Ly * Hq * n * d * dt.itemsize,
+                    "query_store_bytes": Ly * Hq * (M + W if name == "continual" else W) * d
+                                         * dt.itemsize})
+        del window, ws, bout
+    line = {"metric": "Continual vs naive FPS (bkv_update_beacons)", "unit": "ms",
+            "workload": wl.name, "n_layers": Ly, "n_q_heads": Hq, "M": M,
+            "higher_is_better": False, "data": "synthetic", "sweep": out}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------
+# Table 1's (n_recent, n_beacon) trade-off: the step's time per split
+# ----------------------------------------------------------------------------
+def rm_sweep(args, wl):
+    """Time the whole step for each (R, M) split in --rm-sweep ("R:M,..."),
+    the beacons full and the budget --budget; the keys and values are shared
+    by every split.  One JSON line."""
+    from kv_cache_compression_bkv_b200 import bkv, synth
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    pairs = [tuple(int(x) for x in p.split(":")) for p in args.rm_sweep.split(",") if p]
+    base = wl.replace(K=args.budget, n_beacons_in=-1)
+    kv = synth.make_step_inputs(base.replace(R=1, M=1, W=0), seed=args.seed)
+    k, v = kv.k.to(dev), kv.v.to(dev)
+    g = bkv.geometry_of(k, wl.n_q_heads)
+    keep = min(base.K, base.L)
+    dstg = bkv.Geometry(g.n_layers, g.n_q_heads, g.n_kv_heads, g.head_dim, keep, g.dtype)
+    kd = torch.empty(wl.n_layers, wl.n_kv_heads, keep, wl.head_dim, dtype=k.dtype, device=dev)
+    vd = torch.empty_like(kd)
+    idx = torch.empty(wl.n_layers, wl.n_kv_heads, keep, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+    out = []
+    for R, M in pairs:
+        wp = base.replace(R=R, M=M)
+        Ly, Hq, d, dt = wp.n_layers, wp.n_q_heads, wp.head_dim, wp.torch_dtype
+        recent = torch.empty(Ly, Hq, R, d, dtype=dt)
+        beacons = torch.empty(Ly, Hq, M, d, dtype=dt)
+        window = torch.empty(Ly, Hq, wp.W, d, dtype=dt)
+        for l in range(Ly):
+            for qh in range(Hq):
+                r_, b_, w_ = synth.head_queries(wp, args.seed, l, qh)
+                recent[l, qh], beacons[l, qh] = r_.to(dt), b_.to(dt)
+                if wp.W:
+                    window[l, qh] = w_.to(dt)
+        recent, beacons, window = recent.to(dev), beacons.to(dev), window.to(dev)
+        bout = torch.empty_like(beacons)
+        ws = torch.empty(bkv.bkv_workspace_size(g, wp.L, R, M, wp.W, wp.K), dtype=torch.uint8,
+                         device=dev)
+
+        def step(events=None):
+            bkv.bkv_compress_step(g, k, v, wp.L, wp.K, recent, R, beacons, M, M,
+                                  window if wp.W else None, wp.W, bout, 0.0, dstg, kd, vd,
+                                  None, idx, ws, stream, events)
+
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(bkv.STEP_EVENTS)]
+              for _ in range(args.steps)]
+        for row in ev:
+            for e in row:
+                e.record(stream)
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            step(ev[i])
+        torch.cuda.synchronize()
+        st, where = bkv.bkv_read_device_status()
+        if st != 0:
+            raise RuntimeError(f"device status {st} at {where}")
+        ph = {p: sum(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(args.steps)) / args.steps
+              for j, p in enumerate(PHASES)}
+        total = sum(ev[i][0].elapsed_time(ev[i][-1]) for i in range(args.steps)) / args.steps
+        out.append({"n_recent": R, "n_beacon": M, "ms": total, "phases_ms": ph})
+    line = {"metric": "compression step time vs (n_recent, n_beacon)", "unit": "ms",
+            "workload": wl.name, "K": base.K, "L": base.L, "W": base.W,
+            "higher_is_better": False, "data": "synthetic", "sweep": out}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------
 # the CUDA path
 # ----------------------------------------------------------------------------
 def main():
@@ -308,6 +443,12 @@ def main():
                     help="use only this many layers (small cases for profiler captures)")
     ap.add_argument("--aggregate", default="max", choices=["max", "mean"],
                     help="aggregation over the observation rows (mean: Table 2's ablation)")
+    ap.add_argument("--rm-sweep", default=None,
+                    help="comma-separated R:M splits (Table 1): time the step for each")
+    ap.add_argument("--budget", type=int, default=2048, help="K for --rm-sweep")
+    ap.add_argument("--fps-sweep", default=None,
+                    help="comma-separated history lengths: time Continual FPS against naive "
+                         "FPS over each whole history instead of the step")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -322,6 +463,12 @@ def main():
 
     if args.impl == "reference":
         run_reference(args, wl, rank, world)
+        return
+    if args.fps_sweep:
+        fps_sweep(args, wl)
+        return
+    if args.rm_sweep:
+        rm_sweep(args, wl)
         return
 
     from kv_cache_compression_bkv_b200 import bkv

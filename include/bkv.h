@@ -133,6 +133,21 @@ bkv_status bkv_compact(const bkv_cache_desc *src, const void *k_src,
                        const bkv_cache_desc *dst, void *k_dst, void *v_dst,
                        void *stream);
 
+/* Compaction in place: the same result as bkv_compact with the cache as both
+ * source and destination, without a second cache (SURVEY's "ordered chunked
+ * in-place gather"; the page evicts rows but says nothing of buffers).  For
+ * every (layer, KV head) r and i < n_keep, in increasing i:
+ *   k[r][i][:] = k[r][idx[r][i]][:],  v likewise.
+ *   idx  device, int32 [Ly*Hkv][n_keep]; every idx[r][i] must satisfy
+ *        i <= idx[r][i] < capacity, which any ascending list of distinct
+ *        positions does (bkv_select_topk's output, for one).  A row breaking
+ *        this is skipped and reported as BKV_ERR_DEVICE_ASSERT by
+ *        bkv_read_device_status; rows already in place are not copied.
+ *   v may be NULL to compact only the keys.  Rows are at most 32 KB.
+ * Requires 0 <= n_keep <= capacity. */
+bkv_status bkv_compact_inplace(const bkv_cache_desc *desc, void *k, void *v,
+                               const int32_t *idx, int64_t n_keep, void *stream);
+
 /* Continual farthest-point sampling of the beacon queries (Fig. 7).
  * For every (layer, query head): the union U = [beacons_in rows
  * 0..n_beacons_in-1; window rows 0..W-1 (oldest first)] is sampled greedily in
@@ -166,7 +181,9 @@ typedef struct {
   void *beacons_out;           /* device, [Ly][Hq][M][d]; required when W > 0 */
   float scale;                 /* 0: 1/sqrt(head_dim) */
   bkv_cache_desc dst_cache;    /* destination geometry, capacity >= min(K, L) */
-  void *k_dst, *v_dst;         /* device, destination cache */
+  void *k_dst, *v_dst;         /* device, destination cache; k_dst == k and
+                                  v_dst == v (with dst_cache == cache)
+                                  compacts in place */
   float *scores_out;           /* device, optional f32 [Ly][Hkv][L] */
   int32_t *idx_out;            /* device, optional int32 [Ly][Hkv][min(K, L)] */
   void *workspace;

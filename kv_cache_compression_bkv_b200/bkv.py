@@ -25,7 +25,7 @@ STATUS = {0: "BKV_OK", 1: "BKV_ERR_INVALID_ARG", 2: "BKV_ERR_UNSUPPORTED",
           6: "BKV_ERR_DEVICE_ASSERT"}
 EXPORTS = ("bkv_workspace_size", "bkv_score", "bkv_select_topk", "bkv_compact",
            "bkv_update_beacons", "bkv_compress_step", "bkv_read_device_status",
-           "bkv_status_string", "bkv_score_noalloc", "bkv_score_mean")
+           "bkv_status_string", "bkv_score_noalloc", "bkv_score_mean", "bkv_compact_inplace")
 SCORE_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -71,6 +71,7 @@ def _load() -> ctypes.CDLL:
         "bkv_score": ([D, P, I64, P, I32, P, I32, I32, F, P, P, SZ, P], ctypes.c_int),
         "bkv_select_topk": ([P, I32, I64, I64, P, P, SZ, P], ctypes.c_int),
         "bkv_compact": ([D, P, P, P, I64, D, P, P, P], ctypes.c_int),
+        "bkv_compact_inplace": ([D, P, P, P, I64, P], ctypes.c_int),
         "bkv_update_beacons": ([D, P, I32, I32, P, I32, P, ctypes.POINTER(I32), P, SZ, P],
                                ctypes.c_int),
         "bkv_compress_step": ([ctypes.POINTER(StepArgs), ctypes.POINTER(I32),
@@ -186,6 +187,13 @@ def bkv_compact(src: Geometry, k_src, v_src, idx, n_keep: int, dst: Geometry, k_
     _check(LIB.bkv_compact(ctypes.byref(ds), _ptr(k_src), _ptr(v_src), _ptr(idx), n_keep,
                            ctypes.byref(dd), _ptr(k_dst), _ptr(v_dst), _stream(stream)),
            "bkv_compact")
+
+
+def bkv_compact_inplace(geom: Geometry, k, v, idx, n_keep: int, stream=None) -> None:
+    """bkv_compact with the cache as source and destination (idx[r][i] >= i)."""
+    d = geom.desc()
+    _check(LIB.bkv_compact_inplace(ctypes.byref(d), _ptr(k), _ptr(v), _ptr(idx), n_keep,
+                                   _stream(stream)), "bkv_compact_inplace")
 
 
 def bkv_update_beacons(geom: Geometry, beacons_in, n_beacons_in: int, M: int, window, W: int,

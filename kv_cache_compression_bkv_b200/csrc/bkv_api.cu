@@ -262,6 +262,28 @@ bkv_status bkv_compact(const bkv_cache_desc *src, const void *k_src, const void 
   return launch_compact(a, static_cast<cudaStream_t>(stream));
 }
 
+bkv_status bkv_compact_inplace(const bkv_cache_desc *desc, void *k, void *v, const int32_t *idx,
+                               int64_t n_keep, void *stream) {
+  bkv_status st = check_desc(desc);
+  if (st != BKV_OK) return st;
+  if (!k || n_keep < 0 || n_keep > desc->capacity) return BKV_ERR_INVALID_ARG;
+  if (n_keep > 0 && !idx) return BKV_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v) || (reinterpret_cast<uintptr_t>(idx) & 3u))
+    return BKV_ERR_INVALID_ARG;
+  if (v && overlaps(k, cache_bytes(desc), v, cache_bytes(desc))) return BKV_ERR_INVALID_ARG;
+  CompactArgs a;
+  a.k_src = static_cast<const uint8_t *>(k);
+  a.v_src = static_cast<const uint8_t *>(v);
+  a.k_dst = static_cast<uint8_t *>(k);
+  a.v_dst = static_cast<uint8_t *>(v);
+  a.idx = idx;
+  a.n_heads = desc->n_layers * desc->n_kv_heads;
+  a.n_keep = n_keep;
+  a.src_cap = a.dst_cap = desc->capacity;
+  a.row_bytes = static_cast<int>(desc->head_dim * elem_size(desc->dtype));
+  return launch_compact_inplace(a, static_cast<cudaStream_t>(stream));
+}
+
 bkv_status bkv_update_beacons(const bkv_cache_desc *desc, const void *beacons_in,
                               int32_t n_beacons_in, int32_t M, const void *window, int32_t W,
                               void *beacons_out, int32_t *n_beacons_out, void *workspace,
@@ -324,9 +346,12 @@ bkv_status bkv_compress_step(const bkv_step_args *a, int32_t *n_beacons_out, int
       !aligned16(a->v) || !aligned16(a->scores_out) || !aligned16(a->idx_out))
     return BKV_ERR_INVALID_ARG;
   const size_t sb = cache_bytes(d), db = cache_bytes(dd);
-  if (overlaps(a->k_dst, db, a->k, sb) || overlaps(a->k_dst, db, a->v, sb) ||
-      overlaps(a->v_dst, db, a->k, sb) || overlaps(a->v_dst, db, a->v, sb) ||
-      overlaps(a->k_dst, db, a->v_dst, db))
+  // in place: the destination is exactly the source cache
+  const bool in_place = a->k_dst == a->k && a->v_dst == a->v && dd->capacity == d->capacity;
+  if (in_place ? overlaps(a->k, sb, a->v, sb)
+               : (overlaps(a->k_dst, db, a->k, sb) || overlaps(a->k_dst, db, a->v, sb) ||
+                  overlaps(a->v_dst, db, a->k, sb) || overlaps(a->v_dst, db, a->v, sb) ||
+                  overlaps(a->k_dst, db, a->v_dst, db)))
     return BKV_ERR_INVALID_ARG;
 
   FpsGeom f{d->n_layers, d->n_q_heads, d->head_dim, d->dtype, a->n_beacons_in, a->M, a->W,
@@ -410,7 +435,12 @@ bkv_status bkv_compress_step(const bkv_step_args *a, int32_t *n_beacons_out, int
   c.src_cap = d->capacity;
   c.dst_cap = dd->capacity;
   c.row_bytes = static_cast<int>(d->head_dim * elem_size(d->dtype));
-  st = launch_compact(c, s);
+  if (in_place) {
+    // nothing to move when every row is kept
+    st = copy_all ? BKV_OK : launch_compact_inplace(c, s);
+  } else {
+    st = launch_compact(c, s);
+  }
   if (st != BKV_OK) return st;
   if (!mark(5)) return BKV_ERR_CUDA;
   if (n_beacons_out) *n_beacons_out = nb_used;
@@ -424,6 +454,7 @@ bkv_status bkv_read_device_status(void *stream, int32_t *where_out) {
   int code = take_status_score_tc(s, &where);
   if (code == 0) code = take_status_select(s, &where);
   if (code == 0) code = take_status_fps_tc(s, &where);
+  if (code == 0) code = take_status_compact(s, &where);
   if (code < 0) return BKV_ERR_CUDA;
   if (where_out) *where_out = code ? where : 0;
   if (code == 0) return BKV_OK;

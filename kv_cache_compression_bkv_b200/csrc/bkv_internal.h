@@ -92,6 +92,8 @@ struct CompactArgs {
   int row_bytes;               // multiple of 16
 };
 bkv_status launch_compact(const CompactArgs &a, cudaStream_t stream);
+// In place: k_dst/v_dst (== the source) with dst_cap; idx[i] >= i required.
+bkv_status launch_compact_inplace(const CompactArgs &a, cudaStream_t stream);
 
 // ---- fps.cu
 struct FpsGeom {
@@ -101,10 +103,13 @@ struct FpsGeom {
 };
 size_t fps_workspace_bytes(const FpsGeom &g);
 bool fps_supported(const FpsGeom &g);
-// fps_tc.cu: bf16, head_dim 128, the union of a query head in shared memory
+// fps_tc.cu: bf16, head_dim 128.  A union whose distance array does not fit
+// in shared memory keeps it in the workspace: fps_tc_workspace_bytes (0 when
+// it fits) covers one slice per CTA of the persistent grid.
 bool fps_tc_supported(const FpsGeom &g);
+size_t fps_tc_workspace_bytes(const FpsGeom &g);
 bkv_status launch_fps_tc(const FpsGeom &g, const void *beacons_in, const void *window,
-                         void *beacons_out, cudaStream_t stream);
+                         void *beacons_out, void *ws, size_t ws_bytes, cudaStream_t stream);
 bkv_status launch_fps(const FpsGeom &g, const void *beacons_in, const void *window,
                       void *beacons_out, void *ws, size_t ws_bytes, cudaStream_t stream);
 
@@ -126,5 +131,6 @@ bool ensure_smem_limit(Kernel kernel, int bytes, int *done_flags /* [64] */) {
 int take_status_score_tc(cudaStream_t, int *);
 int take_status_select(cudaStream_t, int *);
 int take_status_fps_tc(cudaStream_t, int *);
+int take_status_compact(cudaStream_t, int *);
 
 }  // namespace bkv

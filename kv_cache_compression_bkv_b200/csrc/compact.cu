@@ -6,11 +6,24 @@
 // every row is read and written by full, aligned 32-byte sectors.  Each thread
 // keeps several rows' loads in flight before storing (kUnroll) so that enough
 // bytes are outstanding per SM to cover HBM latency.
+//
+// In place (the destination is the source cache): row i takes row idx_i with
+// idx_i >= i, which holds for any ascending list of kept positions.  One CTA
+// per (head, K or V) walks its rows in chunks in increasing i; a chunk
+// is read whole into registers, the CTA synchronises, then it is written.
+// A row read by chunk c lies at or past the chunk's first row, so it is
+// either in chunk c (written only after the barrier) or in a later chunk
+// (written only after chunk c's reads have returned); rows written by chunk c
+// lie before every row a later chunk reads.  Rows already in place are
+// skipped.  A chunk is at most 32 KB (128 rows of 256 bytes).
 #include <cuda_runtime.h>
 
 #include <algorithm>
 
+#include "bkv_device_status.cuh"
 #include "bkv_internal.h"
+
+BKV_DEFINE_STATUS_ACCESSOR(take_status_compact)
 
 namespace bkv {
 namespace {
@@ -66,7 +79,54 @@ __global__ void __launch_bounds__(kThreads) compact_kernel(const CompactArgs a) 
   }
 }
 
+constexpr int kInplaceThreads = 256;
+constexpr int kInplacePer = 8;  // 16-byte pieces per thread and chunk
+
+__global__ void __launch_bounds__(kInplaceThreads) compact_inplace_kernel(const CompactArgs a) {
+  const int head = blockIdx.x;
+  uint8_t *base = (blockIdx.y == 0 ? a.k_dst : a.v_dst) + static_cast<size_t>(head) * a.dst_cap * a.row_bytes;
+  const int32_t *idx = a.idx + static_cast<size_t>(head) * a.n_keep;
+  const int chunks = a.row_bytes >> 4;  // 16-byte pieces per row
+  const int rows = kInplacePer * kInplaceThreads / chunks;  // rows per chunk
+  const int per_chunk = rows * chunks;
+  for (long long i0 = 0; i0 < a.n_keep; i0 += rows) {
+    uint4 v[kInplacePer];
+    long long dst[kInplacePer];
+#pragma unroll
+    for (int u = 0; u < kInplacePer; ++u) {
+      const int e = threadIdx.x + u * kInplaceThreads;
+      dst[u] = -1;
+      if (e >= per_chunk) continue;
+      const long long i = i0 + e / chunks;
+      if (i >= a.n_keep) continue;
+      const int c = e % chunks;
+      const long long src = idx[i];
+      if (src < i || src >= a.dst_cap) {
+        if (c == 0) record_device_status(BKV_DEV_ASSERT, 501);
+        continue;
+      }
+      if (src == i) continue;  // already in place
+      // L2-coherent load: this kernel writes the same buffer
+      v[u] = __ldcg(reinterpret_cast<const uint4 *>(base + src * a.row_bytes + c * 16));
+      dst[u] = i * a.row_bytes + c * 16;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < kInplacePer; ++u)
+      if (dst[u] >= 0) __stcg(reinterpret_cast<uint4 *>(base + dst[u]), v[u]);
+  }
+}
+
 }  // namespace
+
+bkv_status launch_compact_inplace(const CompactArgs &a, cudaStream_t stream) {
+  if (a.n_keep == 0 || a.n_heads == 0) return BKV_OK;
+  if (a.row_bytes < 16 || a.row_bytes > 16 * kInplacePer * kInplaceThreads) return BKV_ERR_UNSUPPORTED;
+  dim3 grid(static_cast<unsigned>(a.n_heads), a.v_dst != nullptr ? 2u : 1u);
+  if (a.k_dst == nullptr) return BKV_ERR_INVALID_ARG;
+  compact_inplace_kernel<<<grid, kInplaceThreads, 0, stream>>>(a);
+  return cudaGetLastError() == cudaSuccess ? BKV_OK : BKV_ERR_CUDA;
+}
 
 bkv_status launch_compact(const CompactArgs &a, cudaStream_t stream) {
   const long long total = static_cast<long long>(a.n_heads) * a.n_keep * (a.row_bytes >> 4);

@@ -301,7 +301,9 @@ bkv_status launch_dim(const FpsGeom &g, const void *bin, const void *win, void *
 
 }  // namespace
 
-size_t fps_workspace_bytes(const FpsGeom &) { return 0; }
+size_t fps_workspace_bytes(const FpsGeom &g) {
+  return fps_tc_supported(g) ? fps_tc_workspace_bytes(g) : 0;
+}
 
 namespace {
 bool fps_simt_supported(const FpsGeom &g) {
@@ -312,12 +314,13 @@ bool fps_simt_supported(const FpsGeom &g) {
 
 bool fps_supported(const FpsGeom &g) { return fps_tc_supported(g) || fps_simt_supported(g); }
 
-// bf16 unions that fit in shared memory take the tensor-core kernel
-// (fps_tc.cu); f32 inputs and larger unions take the CUDA-core kernel above.
+// bf16 queries with head_dim 128 take the tensor-core kernel (fps_tc.cu);
+// f32 inputs and other head sizes take the CUDA-core kernel above.
 bkv_status launch_fps(const FpsGeom &g, const void *beacons_in, const void *window,
-                      void *beacons_out, void *, size_t, cudaStream_t stream) {
+                      void *beacons_out, void *ws, size_t ws_bytes, cudaStream_t stream) {
   if (g.n_pick <= 0) return BKV_OK;
-  if (fps_tc_supported(g)) return launch_fps_tc(g, beacons_in, window, beacons_out, stream);
+  if (fps_tc_supported(g))
+    return launch_fps_tc(g, beacons_in, window, beacons_out, ws, ws_bytes, stream);
   if (!fps_simt_supported(g)) return BKV_ERR_UNSUPPORTED;
   if (g.dtype == BKV_BF16)
     return launch_dim<__nv_bfloat16>(g, beacons_in, window, beacons_out, stream);

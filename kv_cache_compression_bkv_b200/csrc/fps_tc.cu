@@ -15,7 +15,13 @@
 // two sums may differ in their last bit, which can only reorder picks whose
 // distances agree to about 1e-7.
 //
-// The grid is persistent: one CTA per SM loops over the query heads.
+// While a round selects, the first tiles of its coming pass are already
+// loaded into the ring.  After the seed pass a ring stage is released by the
+// MMA's commit alone.
+//
+// The grid is persistent: one CTA per SM loops over the query heads.  The
+// distance and inverse-norm arrays live in shared memory, or for a union too
+// large for it in the caller's workspace (one slice per CTA).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -140,7 +146,9 @@ __device__ void distance_pass(const Layout &s, const CUtensorMap *bmap, const CU
             umma_f16(tmem + a * 64, ad, bd, idesc, (kb | kk) != 0);
           }
         }
-        umma_commit(empty0 + 8 * st);
+        // the seed pass's epilogue still reads the staged tile (the norms)
+        // and releases the stage itself
+        if (!first) umma_commit(empty0 + 8 * st);
         umma_commit(tfull0 + 8 * a);
       }
     }
@@ -204,7 +212,7 @@ __device__ void distance_pass(const Layout &s, const CUtensorMap *bmap, const CU
         }
         named_barrier_sync(2 + wg, 128);
       }
-      if (ok && warp == 4 + 4 * wg && lane == 0) mbar_arrive(empty0 + 8 * st);
+      if (first && ok && warp == 4 + 4 * wg && lane == 0) mbar_arrive(empty0 + 8 * st);
       if (!ok) continue;
       if (!valid) continue;
       float di = first ? 2.f : s.dist[i];
@@ -265,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fps_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__ CUtensorMap wmap,
                   const FpsGeom g, const __nv_bfloat16 *__restrict__ beacons_in,
                   const __nv_bfloat16 *__restrict__ window, __nv_bfloat16 *__restrict__ beacons_out,
-                  int n_qheads) {
+                  int n_qheads, float *__restrict__ gdist) {
   extern __shared__ uint8_t smem_raw[];
   const int n = g.nb_in + g.W;
   const int m = g.n_pick;
@@ -285,7 +293,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   s.cvec = reinterpret_cast<float *>(s.bop + kBBytes);
   s.gram = s.cvec + kCand * kCStride;
   s.whist = reinterpret_cast<uint32_t *>(s.gram + kCand * kCand);
-  s.dist = reinterpret_cast<float *>(s.whist + kWarps * 256);
+  // the distance and inverse-norm arrays: in shared memory, or this CTA's
+  // slice of the workspace for a union too large for it
+  s.dist = gdist ? gdist + static_cast<size_t>(blockIdx.x) * 2 * n
+                 : reinterpret_cast<float *>(s.whist + kWarps * 256);
   s.inv = s.dist + n;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -294,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) {
       mbar_init(smem_u32(&s.bars[i]), 1);
-      mbar_init(smem_u32(&s.bars[3 + i]), 2);  // the MMA's commit + the epilogue
+      mbar_init(smem_u32(&s.bars[3 + i]), 1);  // the MMA's commit (the epilogue's in the seed pass)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(smem_u32(&s.bars[6 + a]), 1);
@@ -509,18 +520,41 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-size_t fps_tc_smem_bytes(const FpsGeom &g) {
-  return static_cast<size_t>(kFixedBytes) + 8 * (static_cast<size_t>(g.nb_in) + g.W);
+namespace {
+
+// The persistent grid never exceeds this many CTAs (the workspace holds one
+// distance slice per CTA when the arrays live there).
+constexpr int kMaxCtas = 148;
+
+size_t union_array_bytes(const FpsGeom &g) { return 8 * (static_cast<size_t>(g.nb_in) + g.W); }
+
+bool arrays_in_smem(const FpsGeom &g) {
+  return static_cast<size_t>(kFixedBytes) + union_array_bytes(g) <= static_cast<size_t>(kSmemLimit);
+}
+
+size_t smem_bytes(const FpsGeom &g) {
+  return static_cast<size_t>(kFixedBytes) + (arrays_in_smem(g) ? union_array_bytes(g) : 0);
+}
+
+int fps_tc_grid(const FpsGeom &g) { return std::min(g.n_layers * g.n_q_heads, kMaxCtas); }
+
+}  // namespace
+
+size_t fps_tc_workspace_bytes(const FpsGeom &g) {
+  return arrays_in_smem(g) ? 0 : static_cast<size_t>(fps_tc_grid(g)) * union_array_bytes(g);
 }
 
 bool fps_tc_supported(const FpsGeom &g) {
   return g.dtype == BKV_BF16 && g.head_dim == kDim &&
-         fps_tc_smem_bytes(g) <= static_cast<size_t>(kSmemLimit) &&
          static_cast<long long>(g.n_layers) * g.n_q_heads * std::max(g.M, g.W) < (1LL << 31) - 256;
 }
 
 bkv_status launch_fps_tc(const FpsGeom &g, const void *beacons_in, const void *window,
-                         void *beacons_out, cudaStream_t stream) {
+                         void *beacons_out, void *ws, size_t ws_bytes, cudaStream_t stream) {
+  const size_t ws_need = fps_tc_workspace_bytes(g);
+  if (ws_need > 0 && (ws == nullptr || ws_bytes < ws_need ||
+                      (reinterpret_cast<uintptr_t>(ws) & 15u) != 0))
+    return BKV_ERR_WORKSPACE;
   const int n_qheads = g.n_layers * g.n_q_heads;
   // Tensor maps over every head's beacon slots and window rows.  A map needs
   // a non-empty tensor: an absent part (no beacons, or no window) points at
@@ -536,16 +570,16 @@ bkv_status launch_fps_tc(const FpsGeom &g, const void *beacons_in, const void *w
       !make_bf16_rows_map(&wmap, wsrc, wrows, kTileRows))
     return BKV_ERR_CUDA;
   static int attr_done[64];
-  const int smem = static_cast<int>(fps_tc_smem_bytes(g));
+  const int smem = static_cast<int>(smem_bytes(g));
   if (!ensure_smem_limit(fps_tc_kernel, kSmemLimit, attr_done)) return BKV_ERR_CUDA;
-  int sms = 148, dev = 0;
+  int sms = kMaxCtas, dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int grid = std::max(1, std::min(n_qheads, sms));
+  const int grid = std::max(1, std::min(fps_tc_grid(g), sms));
   fps_tc_kernel<<<grid, kThreads, smem, stream>>>(
       bmap, wmap, g, static_cast<const __nv_bfloat16 *>(beacons_in),
       static_cast<const __nv_bfloat16 *>(window), static_cast<__nv_bfloat16 *>(beacons_out),
-      n_qheads);
+      n_qheads, ws_need > 0 ? static_cast<float *>(ws) : nullptr);
   return cudaGetLastError() == cudaSuccess ? BKV_OK : BKV_ERR_CUDA;
 }
 

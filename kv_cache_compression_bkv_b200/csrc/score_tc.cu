@@ -298,22 +298,19 @@ __global__ void __launch_bounds__(kP1Threads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
+      if (key_base + 64 > L) {  // the ragged end of the keys
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        float (&cur)[32] = c ? vb : va;
-        const long long k0 = key_base + c * 32;
-        if (k0 + 32 > L) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (k0 + i >= L) cur[i] = -INFINITY;
+        for (int i = 0; i < 32; ++i) {
+          if (key_base + i >= L) va[i] = -INFINITY;
+          if (key_base + 32 + i >= L) vb[i] = -INFINITY;
         }
-        const float mz = max32(cur) * kz;
-        if (mz > m) {
-          ssum *= ex2_approx(m - mz);
-          m = mz;
-        }
-        if (m != -INFINITY) ssum += chunk_exp_sum(cur, kz, m);
       }
+      // one running-max update per 64 columns, then 32 independent exp pairs
+      const float mz = fmaxf(max32(va), max32(vb)) * kz;
+      const float m_new = fmaxf(m, mz);
+      ssum = m_new == -INFINITY ? 0.f : ssum * ex2_approx(m - m_new);
+      m = m_new;
+      if (m != -INFINITY) ssum += chunk_exp_sum(va, kz, m) + chunk_exp_sum(vb, kz, m);
     }
     // combine the four column quarters of each row; the exchange reuses the
     // key stages, free once the last tile's MMAs have completed

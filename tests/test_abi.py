@@ -127,6 +127,20 @@ def test_compact_rejects():
     assert call(dst=ctypes.byref(desc(cap=256, dt=bkv.BKV_F32))) == INVALID
 
 
+def test_compact_inplace_rejects():
+    f = LIB.bkv_compact_inplace
+    d = desc(cap=1024)
+    big = 1 << 30
+    assert f(ctypes.byref(d), A, A + big, A + 2 * big, 1025, S) == INVALID  # beyond capacity
+    assert f(ctypes.byref(d), A, A + big, A + 2 * big, -1, S) == INVALID
+    assert f(ctypes.byref(d), None, A + big, A + 2 * big, 10, S) == INVALID
+    assert f(ctypes.byref(d), A, A + big, None, 10, S) == INVALID
+    assert f(ctypes.byref(d), A + 8, A + big, A + 2 * big, 10, S) == INVALID  # misaligned
+    assert f(ctypes.byref(d), A, A + big, A + 2 * big + 2, 10, S) == INVALID
+    assert f(ctypes.byref(d), A, A + 64, A + 2 * big, 10, S) == INVALID   # K and V overlap
+    assert f(None, A, A + big, A + 2 * big, 10, S) == INVALID
+
+
 def test_update_beacons_rejects():
     f = LIB.bkv_update_beacons
     d = desc()
@@ -148,7 +162,10 @@ def test_update_beacons_rejects():
     assert call(bout=0) == INVALID
     assert call(bout=A + 64) == INVALID                 # overlaps beacons_in
     assert call(bout=A + big + 128) == INVALID          # overlaps window
-    assert call(W=100000) == UNSUPPORTED                # distances do not fit shared memory
+    # a bf16 union this large keeps its distances in the workspace
+    assert call(W=100000) == WORKSPACE
+    # the f32 kernel keeps them in shared memory only
+    assert call(d=ctypes.byref(desc(dt=bkv.BKV_F32)), W=100000) == UNSUPPORTED
     assert n.value == -7                                # outputs untouched
 
 
@@ -183,7 +200,9 @@ def step_args(**kw):
     (dict(idx_out=A + 2), INVALID),                # misaligned
     (dict(workspace_bytes=4096), WORKSPACE),
     (dict(workspace=None), WORKSPACE),
-    (dict(W=100000), UNSUPPORTED),
+    (dict(W=100000, cache=desc(cap=1024, dt=bkv.BKV_F32),
+          dst_cache=desc(cap=512, dt=bkv.BKV_F32)), UNSUPPORTED),  # f32 union too large
+    (dict(W=100000, workspace_bytes=1 << 20), WORKSPACE),  # bf16: needs workspace slices
     (dict(aggregate=2), INVALID),                  # neither max nor mean
     (dict(aggregate=-1), INVALID),
 ])

@@ -137,9 +137,11 @@ FPS_CASES = {
     "window_only_one": lambda: small(W=1, M=4, n_beacons_in=0, R=1),
     "ragged_tiles": lambda: small(W=333, M=40, n_beacons_in=37),
     "many_rounds": lambda: small(n_q_heads=2, n_kv_heads=1, W=1200, M=128, n_beacons_in=100),
-    # a union too large for the shared-memory distance array of the
-    # tensor-core kernel: the CUDA-core kernel handles it
+    # unions too large for the shared-memory distance arrays: the tensor-core
+    # kernel keeps them in the workspace (one slice per CTA)
     "large_union": lambda: small(n_q_heads=2, n_kv_heads=1, W=9000, M=32, n_beacons_in=32),
+    # naive FPS (Fig. 7's baseline): the whole query history, no beacons
+    "naive_history": lambda: small(n_q_heads=4, n_kv_heads=1, W=20000, M=48, n_beacons_in=0),
 }
 
 
@@ -151,8 +153,10 @@ def test_update_beacons(case, dev):
     g = bkv.geometry_of(inp.k, wl.n_q_heads)
     bin_, win = inp.beacons.to(dev), inp.window.to(dev)
     bout = torch.zeros_like(bin_)
+    ws = torch.empty(max(1, bkv.bkv_workspace_size(g, 1, 0, wl.M, wl.W, 1)), dtype=torch.uint8,
+                     device=dev)
     n = bkv.bkv_update_beacons(g, bin_ if wl.beacons_in else None, wl.beacons_in, wl.M, win,
-                               wl.W, bout)
+                               wl.W, bout, ws)
     torch.cuda.synchronize()
     assert n == min(wl.M, wl.beacons_in + wl.W)
     out_raw = raw(bout)
@@ -292,3 +296,90 @@ def test_full_size_sampled_mean(dev):
     assert n_exact >= 1, "every sampled head hit an FPS near-tie"
     sums = out["scores"].double().sum(-1)
     assert bool(((sums - 1.0).abs() < 1e-3).all()), sums.flatten()[:8]
+
+
+def _ascending_positions(rng, cap, n_keep, mode):
+    """Kept positions in [0, cap), ascending, with the shapes compaction meets."""
+    if mode == "prefix_kept":       # the first rows stay, then a sparse tail
+        head = np.arange(n_keep // 3)
+        rest = np.sort(rng.choice(np.arange(n_keep // 3, cap), n_keep - head.size, replace=False))
+        return np.concatenate([head, rest])
+    if mode == "tail":              # only the newest rows survive
+        return np.arange(cap - n_keep, cap)
+    return np.sort(rng.choice(cap, n_keep, replace=False))
+
+
+@pytest.mark.parametrize("dtype,d,cap,n_keep,mode", [
+    ("bf16", 128, 1000, 300, "random"),
+    ("bf16", 128, 4096, 1537, "prefix_kept"),
+    ("bf16", 128, 777, 777, "random"),        # every row kept: nothing moves
+    ("bf16", 128, 5000, 129, "tail"),
+    ("f32", 128, 2000, 1000, "random"),       # 512-byte rows: 64-row chunks
+    ("f32", 24, 999, 400, "prefix_kept"),     # 96-byte rows: chunks of 341 rows
+])
+def test_compact_inplace(dtype, d, cap, n_keep, mode, dev):
+    """In-place compaction equals the out-of-place gather, byte for byte."""
+    bkv = _lib()
+    rng = np.random.default_rng(cap + n_keep)
+    Ly, Hkv = 2, 3
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    k0 = torch.randn(Ly, Hkv, cap, d, generator=torch.Generator().manual_seed(1)).to(tdt)
+    v0 = torch.randn(Ly, Hkv, cap, d, generator=torch.Generator().manual_seed(2)).to(tdt)
+    idx = np.stack([_ascending_positions(rng, cap, n_keep, mode) for _ in range(Ly * Hkv)])
+    idx_t = torch.from_numpy(idx.astype(np.int32)).to(dev)
+    k, v = k0.to(dev), v0.to(dev)
+    g = bkv.Geometry(Ly, Hkv, Hkv, d, cap, tdt)
+    bkv.bkv_compact_inplace(g, k, v, idx_t, n_keep)
+    torch.cuda.synchronize()
+    assert bkv.bkv_read_device_status()[0] == 0
+    kr, vr = raw(k), raw(v)
+    k0r, v0r = raw(k0), raw(v0)
+    for r in range(Ly * Hkv):
+        l, h = divmod(r, Hkv)
+        check_compaction(kr[l, h, :n_keep], k0r[l, h], idx[r], f"in-place K {mode} r{r}")
+        check_compaction(vr[l, h, :n_keep], v0r[l, h], idx[r], f"in-place V {mode} r{r}")
+        # rows past n_keep are left as they were or hold moved-from data; the
+        # kept prefix is all that is defined
+
+
+def test_compact_inplace_reports_a_backward_index(dev):
+    """A position below its slot is skipped and reported, not followed."""
+    bkv = _lib()
+    cap, n_keep, d = 512, 200, 128
+    k = torch.randn(1, 1, cap, d, device=dev).to(torch.bfloat16)
+    before = raw(k)
+    idx = torch.arange(n_keep, dtype=torch.int32) + 5
+    idx[150] = 3                                   # 3 < 150: breaks idx[i] >= i
+    g = bkv.Geometry(1, 1, 1, d, cap, torch.bfloat16)
+    bkv.bkv_compact_inplace(g, k, None, idx.to(dev), n_keep)
+    st, where = bkv.bkv_read_device_status()
+    assert st == 6 and where == 501                # BKV_ERR_DEVICE_ASSERT
+    after = raw(k)
+    good = [i for i in range(n_keep) if i != 150]
+    assert np.array_equal(after[0, 0, good], before[0, 0, np.array(good) + 5])
+
+
+@pytest.mark.parametrize("case", ["bf16_fps", "no_window", "keep_all"])
+def test_compress_step_in_place(case, dev):
+    """The step with the source cache as destination gives the out-of-place result."""
+    bkv, synth = _lib(), _synth()
+    wl = STEP_CASES[case]()
+    inp = synth.make_step_inputs(wl, seed=6)
+    out, nb = _run_step(wl, inp, dev)
+    g = bkv.geometry_of(inp.k, wl.n_q_heads)
+    t = {n: getattr(inp, n).to(dev) for n in ("k", "v", "recent", "beacons", "window")}
+    keep = min(wl.K, wl.L)
+    bout = torch.zeros_like(t["beacons"])
+    idx = torch.empty(wl.n_layers, wl.n_kv_heads, keep, dtype=torch.int32, device=dev)
+    ws = torch.empty(bkv.bkv_workspace_size(g, wl.L, wl.R, wl.M, wl.W, wl.K), dtype=torch.uint8,
+                     device=dev)
+    nb2, nl = bkv.bkv_compress_step(
+        g, t["k"], t["v"], wl.L, wl.K, t["recent"] if wl.R else None, wl.R,
+        t["beacons"] if wl.beacons_in else None, wl.beacons_in, wl.M,
+        t["window"] if wl.W else None, wl.W, bout, 0.0, g, t["k"], t["v"], None, idx, ws)
+    torch.cuda.synchronize()
+    assert bkv.bkv_read_device_status()[0] == 0
+    assert (nb2, nl) == (nb, keep)
+    assert torch.equal(idx, out["idx"])
+    assert np.array_equal(raw(t["k"])[:, :, :keep], raw(out["kd"]))
+    assert np.array_equal(raw(t["v"])[:, :, :keep], raw(out["vd"]))
