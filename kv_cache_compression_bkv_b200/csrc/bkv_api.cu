@@ -455,6 +455,7 @@ bkv_status bkv_read_device_status(void *stream, int32_t *where_out) {
   if (code == 0) code = take_status_select(s, &where);
   if (code == 0) code = take_status_fps_tc(s, &where);
   if (code == 0) code = take_status_compact(s, &where);
+  if (code == 0) code = take_status_fps(s, &where);
   if (code < 0) return BKV_ERR_CUDA;
   if (where_out) *where_out = code ? where : 0;
   if (code == 0) return BKV_OK;

@@ -132,5 +132,6 @@ int take_status_score_tc(cudaStream_t, int *);
 int take_status_select(cudaStream_t, int *);
 int take_status_fps_tc(cudaStream_t, int *);
 int take_status_compact(cudaStream_t, int *);
+int take_status_fps(cudaStream_t, int *);
 
 }  // namespace bkv

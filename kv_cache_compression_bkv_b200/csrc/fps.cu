@@ -28,8 +28,11 @@
 
 #include <algorithm>
 
+#include "bkv_device_status.cuh"
 #include "bkv_internal.h"
 #include "fps_common.cuh"
+
+BKV_DEFINE_STATUS_ACCESSOR(take_status_fps)
 
 namespace bkv {
 namespace {
@@ -252,6 +255,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncthreads();
     const int np = s.scal[4];
+    if (np == 0) {
+      // only distances that are not numbers (NaN input rows) can stop the
+      // replay before its first pick; report instead of looping
+      if (tid == 0) record_device_status(BKV_DEV_ASSERT, 406);
+      break;
+    }
     // this round's picks: outputs, vectors, inverse norms
     for (int e = tid; e < np * d; e += kThreads) {
       const int k = e / d, t = e - k * d;

@@ -50,12 +50,16 @@ constexpr int kStages = 3;
 constexpr int kTileBytes = kTileRows * kDim * 2;  // 32 KB
 constexpr int kBBlock = kCand * 128;              // one 64-element K block of the picks
 constexpr int kBBytes = 2 * kBBlock;              // 16 KB
-constexpr int kCStride = kDim + 4;
+constexpr int kCRows = 128;                       // candidate operand rows (64 + zero rows)
+constexpr int kCBlock = kCRows * 128;             // one 64-element K block of the candidates
+constexpr int kCBytes = 2 * kCBlock;              // 32 KB
 constexpr int kSmallBytes = 4096;
 constexpr int kFixedBytes = kSmallBytes + 1024 + kStages * kTileBytes + kBBytes +
-                            kCand * kCStride * 4 + kCand * kCand * 4 + kWarps * 256 * 4;
+                            kCBytes + kCand * kCand * 4 + kWarps * 256 * 4;
 constexpr int kSmemLimit = 232448;
-constexpr uint32_t kTmemCols = 128;  // two accumulators of up to 64 columns
+// two accumulators of up to 64 columns, then the candidates' Gram block
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kGramCol = 128;
 constexpr int kAbort = 15;           // index of the abort flag in scal[]
 
 enum { kWhereProd = 401, kWhereMma = 402, kWhereEpi = 403, kWhereDrain = 404 };
@@ -71,7 +75,8 @@ struct Layout {
   float *pinv;      // [kCand]
   uint8_t *stages;  // [kStages][kTileBytes]
   uint8_t *bop;     // picks, K-major 128-byte swizzle: [2][kCand rows][128 B]
-  float *cvec;      // [kCand][kCStride]
+  uint8_t *cop;     // candidates, K-major 128-byte swizzle: [2][kCRows rows][128 B];
+                    // rows kCand.. stay zero (the Gram MMA has M = 128)
   float *gram;      // [kCand][kCand]
   uint32_t *whist;  // [kWarps][256] per-warp histograms of the selection
   float *dist;      // [n]
@@ -253,16 +258,17 @@ __device__ void distance_pass(const Layout &s, const CUtensorMap *bmap, const CU
 }
 
 // The picks of this round into the B operand (rows padded with zeros to a
-// multiple of 16) and the output beacons.
+// multiple of 16) and the output beacons: the seed's row from global memory,
+// a round's picks from the staged candidate rows.
 __device__ void stage_picks(const Layout &s, const Head &h, __nv_bfloat16 *out, int picked,
-                            int np) {
+                            int np, bool seed) {
   const int npad = (np + 15) & ~15;
   for (int e = threadIdx.x; e < npad * 16; e += kThreads) {
     const int k = e >> 4, c16 = e & 15, kb = c16 >> 3, c = c16 & 7;
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
     if (k < np) {
-      const __nv_bfloat16 *src = h.point(s.cidx[s.pick[k]]) + c16 * 8;
-      v = *reinterpret_cast<const uint4 *>(src);
+      v = seed ? *reinterpret_cast<const uint4 *>(h.point(s.cidx[s.pick[k]]) + c16 * 8)
+               : *reinterpret_cast<const uint4 *>(s.cop + kb * kCBlock + sw128_offset(s.pick[k], c));
       *reinterpret_cast<uint4 *>(out + static_cast<size_t>(picked + k) * kDim + c16 * 8) = v;
     }
     *reinterpret_cast<uint4 *>(s.bop + kb * kBBlock + sw128_offset(k, c)) = v;
@@ -290,8 +296,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t big = (raw_base + kSmallBytes + 1023u) & ~1023u;
   s.stages = smem_raw + (big - raw_base);
   s.bop = s.stages + kStages * kTileBytes;
-  s.cvec = reinterpret_cast<float *>(s.bop + kBBytes);
-  s.gram = s.cvec + kCand * kCStride;
+  s.cop = s.bop + kBBytes;
+  s.gram = reinterpret_cast<float *>(s.cop + kCBytes);
   s.whist = reinterpret_cast<uint32_t *>(s.gram + kCand * kCand);
   // the distance and inverse-norm arrays: in shared memory, or this CTA's
   // slice of the workspace for a union too large for it
@@ -312,6 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&s.bars[8 + a]), 4);  // one arrive per warp of its warpgroup
     }
     mbar_init(smem_u32(&s.bars[10]), 1);
+    mbar_init(smem_u32(&s.bars[11]), 1);  // the Gram block's MMA
     fence_barrier_init();
     prefetch_tensormap(&bmap);
     prefetch_tensormap(&wmap);
@@ -321,11 +328,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(smem_u32(s.tmem_slot), kTmemCols);
     tmem_relinquish();
   }
+  // the candidate operand's padding rows are zero for good
+  for (int e = tid; e < 2 * (kCRows - kCand) * 8; e += kThreads) {
+    const int kb = e / ((kCRows - kCand) * 8), rem = e - kb * (kCRows - kCand) * 8;
+    const int r = kCand + (rem >> 3), c = rem & 7;
+    *reinterpret_cast<uint4 *>(s.cop + kb * kCBlock + sw128_offset(r, c)) = make_uint4(0u, 0u, 0u, 0u);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *s.tmem_slot;
   uint32_t seq = 0;
+  uint32_t gram_phase = 0;
+  bool stuck = false;  // uniform: set by every thread from the same shared value
 
   for (int qh = blockIdx.x; qh < n_qheads; qh += gridDim.x) {
     Head h{beacons_in + static_cast<size_t>(qh) * g.M * kDim,
@@ -345,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (tid > 0 && tid < 16) s.pinv[tid] = __int_as_float(0x7fc00000);
     __syncthreads();
-    stage_picks(s, h, out, 0, 1);
+    stage_picks(s, h, out, 0, 1, true);
     fence_proxy_async_smem();
     __syncthreads();
     distance_pass(s, &bmap, &wmap, tmem, qh, g, n_btiles, n_tiles, seq, 1, true, 0);
@@ -400,47 +415,55 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       __syncthreads();
-      for (int e = tid; e < nc * (kDim / 8); e += kThreads) {
-        const int a = e >> 4, t = (e & 15) * 8;
-        float u[8];
-        load8(h.point(s.cidx[a]) + t, u);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) s.cvec[a * kCStride + t + j] = u[j];
+      // the candidates' rows into the swizzled operand (rows past nc keep
+      // whatever an earlier round left; their Gram entries are never read)
+      for (int e = tid; e < nc * 16; e += kThreads) {
+        const int a = e >> 4, c16 = e & 15, kb = c16 >> 3, c = c16 & 7;
+        *reinterpret_cast<uint4 *>(s.cop + kb * kCBlock + sw128_offset(a, c)) =
+            *reinterpret_cast<const uint4 *>(h.point(s.cidx[a]) + c16 * 8);
       }
+      fence_proxy_async_smem();
+      tc_fence_before();
       __syncthreads();
-      // Gram block, 4 x 4 dot products per thread (a = ta + 16 r, b = tb + 16 r'):
-      // each loaded 8-element slice feeds four dot products, and the lanes of
-      // a phase read rows in distinct banks
-      if (tid < 256) {
-        const int ta = tid & 15, tb = tid >> 4;
-        float2 acc[4][4];
+      // Gram block on the tensor cores: D[a][b] = cand_a . cand_b, M = 128
+      // (rows a >= kCand are the zero padding), N = kCand, K = 128, the same
+      // f32 accumulation of exact bf16 products as the distance pass
+      if (warp == 1 && lane == 0) {
+        tc_fence_after();
+        const uint32_t idesc = idesc_bf16_f32(kCRows, kCand);
+        const uint32_t c_base = smem_u32(s.cop);
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
+        for (int kb = 0; kb < 2; ++kb) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) acc[r][q] = make_float2(0.f, 0.f);
-#pragma unroll 2
-        for (int t = 0; t < kDim; t += 8) {
-          float u[4][8], w[4][8];
-#pragma unroll
-          for (int r = 0; r < 4; ++r) {
-            load8(s.cvec + (ta + 16 * r) * kCStride + t, u[r]);
-            load8(s.cvec + (tb + 16 * r) * kCStride + t, w[r]);
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = smem_desc_k_sw128(c_base + kb * kCBlock + kk * 32);
+            umma_f16(tmem + kGramCol, ad, ad, idesc, (kb | kk) != 0);
           }
-#pragma unroll
-          for (int r = 0; r < 4; ++r)
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-#pragma unroll
-              for (int j = 0; j < 8; j += 2)
-                acc[r][q] = __ffma2_rn(make_float2(u[r][j], u[r][j + 1]),
-                                       make_float2(w[q][j], w[q][j + 1]), acc[r][q]);
         }
-#pragma unroll
-        for (int r = 0; r < 4; ++r)
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            s.gram[(tb + 16 * q) * kCand + ta + 16 * r] = __fadd_rn(acc[r][q].x, acc[r][q].y);
+        umma_commit(smem_u32(&s.bars[11]));
       }
+      if (warp == 4 || warp == 5) {
+        // TMEM lane = candidate a: warp 4 reads rows 0..31, warp 5 rows 32..63
+        if (mbar_wait_warp(smem_u32(&s.bars[11]), gram_phase & 1, kWhereEpi)) {
+          tc_fence_after();
+          const uint32_t taddr = tmem + (static_cast<uint32_t>((warp - 4) * 32) << 16) + kGramCol;
+          float *row = s.gram + ((warp - 4) * 32 + lane) * kCand;
+#pragma unroll 1
+          for (int half = 0; half < 2; ++half) {
+            float x[32];
+            tmem_ld_32x32b_x32(taddr + half * 32, x);
+            tmem_ld_wait_regs(x);
+#pragma unroll
+            for (int b = 0; b < 32; b += 4)
+              *reinterpret_cast<float4 *>(row + half * 32 + b) =
+                  make_float4(x[b], x[b + 1], x[b + 2], x[b + 3]);
+          }
+        } else {
+          s.scal[kAbort] = 1;
+        }
+        tc_fence_before();
+      }
+      ++gram_phase;
       __syncthreads();
       // replay the greedy choice among the candidates (warp 0, two per lane).
       // The argmax in (distance desc, index asc) order takes two warp
@@ -482,9 +505,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncthreads();
       const int np = s.scal[4];
+      if (np == 0) {
+        // only distances that are not numbers (NaN input rows) can stop the
+        // replay before its first pick; report and stop instead of looping
+        if (tid == 0) record_device_status(BKV_DEV_ASSERT, 405);
+        stuck = true;
+        seq += pre;  // the coming pass's first tiles are in flight: drain them
+        break;
+      }
       if (tid < ((np + 15) & ~15))
         s.pinv[tid] = tid < np ? s.inv[s.cidx[s.pick[tid]]] : __int_as_float(0x7fc00000);
-      stage_picks(s, h, out, picked, np);
+      stage_picks(s, h, out, picked, np, false);
       __syncthreads();
       if (tid < np) s.dist[s.cidx[s.pick[tid]]] = -1.f;
       fence_proxy_async_smem();
@@ -495,7 +526,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (s.scal[kAbort]) break;
       picked += np;
     }
-    if (s.scal[kAbort]) break;
+    if (s.scal[kAbort] || stuck) break;
   }
 
   // drain: every TMA load and MMA issued by this CTA has completed before the
