@@ -63,7 +63,12 @@ __device__ __forceinline__ bool before(float da, int ia, float db, int ib) {
 // which would otherwise pile every key into one or two bins); each warp counts
 // into its own histogram.  Then every key above the threshold and the
 // lowest-index keys equal to it are emitted.
-// Scratch: whist[kThreads / 32 * 256], hist[256], scal[>= 8].
+// Once the bin still to be resolved holds at most kRankMax keys, the
+// remaining digit passes are replaced by ranking those keys against each
+// other (key desc, index asc).
+// Scratch: whist[kThreads / 32 * 256] (>= 2 * kRankMax words), hist[256], scal[>= 8].
+constexpr int kRankMax = 256;
+
 template <int kThreads>
 __device__ void select_best(const float *dist, int n, int n_live, int want, uint32_t *whist,
                             uint32_t *hist, int *scal, int *cidx, float *cdist) {
@@ -103,6 +108,7 @@ __device__ void select_best(const float *dist, int n, int n_live, int want, uint
   int krem = want;
   int n_eq = n_live;  // live keys matching the prefix
   for (; hi > 0; hi -= 8) {
+    if (n_eq <= kRankMax) break;  // few enough to rank directly
     const int lo = hi > 8 ? hi - 8 : 0;
     uint32_t *mine = whist + warp * 256;
     for (int b = lane; b < 256; b += 32) mine[b] = 0;
@@ -170,6 +176,61 @@ __device__ void select_best(const float *dist, int n, int n_live, int want, uint
         if (pos < want) {
           cidx[pos] = i;
           cdist[pos] = dist[i];
+        }
+      }
+    }
+    return;
+  }
+  if (hi > 0) {
+    // the bin (key & mask) == prefix holds n_eq <= kRankMax keys, of which
+    // the krem best are kept, with every key above the bin.  Keys above are
+    // emitted as found; the bin's keys are listed, then each is kept when
+    // fewer than krem listed keys come before it in (key desc, index asc).
+    static_assert(kThreads / 32 * 256 >= 2 * kRankMax, "rank list does not fit");
+    uint32_t *lkey = whist;
+    int *lidx = reinterpret_cast<int *>(whist + kRankMax);
+    if (tid == 0) scal[3] = 0;
+    __syncthreads();
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    for (int base = 0; base < n; base += kThreads) {
+      const int i = base + tid;
+      const uint32_t key = i < n ? dist_key(dist[i]) : 0u;
+      const bool live = key != 0u;
+      const bool above = live && (key & mask) > prefix;
+      const bool inbin = live && (key & mask) == prefix;
+      const uint32_t ba = __ballot_sync(0xffffffffu, above);
+      const uint32_t bb = __ballot_sync(0xffffffffu, inbin);
+      int pa = 0, pb = 0;
+      if (lane == 0) {
+        if (ba) pa = atomicAdd(&scal[2], __popc(ba));
+        if (bb) pb = atomicAdd(&scal[3], __popc(bb));
+      }
+      pa = __shfl_sync(0xffffffffu, pa, 0) + __popc(ba & lt_mask);
+      pb = __shfl_sync(0xffffffffu, pb, 0) + __popc(bb & lt_mask);
+      if (above && pa < want) {
+        cidx[pa] = i;
+        cdist[pa] = dist[i];
+      }
+      if (inbin && pb < kRankMax) {
+        lkey[pb] = key;
+        lidx[pb] = i;
+      }
+    }
+    __syncthreads();
+    const int listed = min(scal[3], kRankMax);
+    for (int e = tid; e < listed; e += kThreads) {
+      const uint32_t ke = lkey[e];
+      const int ie = lidx[e];
+      int rank = 0;
+      for (int f = 0; f < listed; ++f) {
+        const uint32_t kf = lkey[f];
+        rank += (kf > ke || (kf == ke && lidx[f] < ie)) ? 1 : 0;
+      }
+      if (rank < krem) {
+        const int pos = atomicAdd(&scal[2], 1);
+        if (pos < want) {
+          cidx[pos] = ie;
+          cdist[pos] = dist[ie];
         }
       }
     }
