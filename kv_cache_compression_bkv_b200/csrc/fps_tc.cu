@@ -41,16 +41,16 @@ namespace {
 using namespace sm100;
 using namespace fpsk;
 
-constexpr int kThreads = 384;  // warp 0 TMA, warp 1 MMA, warps 4..11 distance epilogue
+constexpr int kThreads = 384;  // warp 0 TMA, warps 1-2 MMA, warps 4..11 distance epilogue
 constexpr int kWarps = kThreads / 32;
 constexpr int kCand = 64;      // candidates per round (T)
 constexpr int kDim = 128;
 constexpr int kTileRows = 128;
-constexpr int kStages = 3;
+constexpr int kStages = 4;  // even tiles use stages 0 and 2, odd tiles 1 and 3
 constexpr int kTileBytes = kTileRows * kDim * 2;  // 32 KB
 constexpr int kBBlock = kCand * 128;              // one 64-element K block of the picks
 constexpr int kBBytes = 2 * kBBlock;              // 16 KB
-constexpr int kCRows = 128;                       // candidate operand rows (64 + zero rows)
+constexpr int kCRows = kCand;                     // candidate operand rows
 constexpr int kCBlock = kCRows * 128;             // one 64-element K block of the candidates
 constexpr int kCBytes = 2 * kCBlock;              // 32 KB
 constexpr int kSmallBytes = 4096;
@@ -64,8 +64,13 @@ constexpr int kAbort = 15;           // index of the abort flag in scal[]
 
 enum { kWhereProd = 401, kWhereMma = 402, kWhereEpi = 403, kWhereDrain = 404 };
 
+// Barriers: full[4] empty[4] tfull[2] tempty[2], the two MMA threads' drain
+// barriers, the Gram block's.
+constexpr int kBarFull = 0, kBarEmpty = 4, kBarTfull = 8, kBarTempty = 10, kBarDone = 12,
+              kBarGram = 14;
+
 struct Layout {
-  uint64_t *bars;   // full[3] empty[3] tfull[2] tempty[2] done
+  uint64_t *bars;   // see kBarFull ..
   uint32_t *tmem_slot;
   int *scal;        // [16]
   uint32_t *hist;   // [256]
@@ -75,8 +80,7 @@ struct Layout {
   float *pinv;      // [kCand]
   uint8_t *stages;  // [kStages][kTileBytes]
   uint8_t *bop;     // picks, K-major 128-byte swizzle: [2][kCand rows][128 B]
-  uint8_t *cop;     // candidates, K-major 128-byte swizzle: [2][kCRows rows][128 B];
-                    // rows kCand.. stay zero (the Gram MMA has M = 128)
+  uint8_t *cop;     // candidates, K-major 128-byte swizzle: [2][kCRows rows][128 B]
   float *gram;      // [kCand][kCand]
   uint32_t *whist;  // [kWarps][256] per-warp histograms of the selection
   float *dist;      // [n]
@@ -104,7 +108,7 @@ __device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
 __device__ bool issue_tiles(const Layout &s, const CUtensorMap *bmap, const CUtensorMap *wmap,
                             int qh, const FpsGeom &g, int n_btiles, uint32_t seq, int j0,
                             int j1) {
-  const uint32_t full0 = smem_u32(&s.bars[0]), empty0 = smem_u32(&s.bars[3]);
+  const uint32_t full0 = smem_u32(&s.bars[kBarFull]), empty0 = smem_u32(&s.bars[kBarEmpty]);
   for (int j = j0; j < j1; ++j) {
     const uint32_t q = seq + j, st = q % kStages;
     if (!mbar_wait(empty0 + 8 * st, ((q / kStages) & 1) ^ 1, kWhereProd)) return false;
@@ -122,19 +126,24 @@ __device__ void distance_pass(const Layout &s, const CUtensorMap *bmap, const CU
                               uint32_t tmem, int qh, const FpsGeom &g, int n_btiles, int n_tiles,
                               uint32_t seq, int np, bool first, int prefetched) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t full0 = smem_u32(&s.bars[0]), empty0 = smem_u32(&s.bars[3]);
-  const uint32_t tfull0 = smem_u32(&s.bars[6]), tempty0 = smem_u32(&s.bars[8]);
+  const uint32_t full0 = smem_u32(&s.bars[kBarFull]), empty0 = smem_u32(&s.bars[kBarEmpty]);
+  const uint32_t tfull0 = smem_u32(&s.bars[kBarTfull]), tempty0 = smem_u32(&s.bars[kBarTempty]);
   if (warp == 0) {
     if (lane == 0 &&
         !issue_tiles(s, bmap, wmap, qh, g, n_btiles, seq, prefetched, n_tiles))
       s.scal[kAbort] = 1;
-  } else if (warp == 1) {
+  } else if (warp == 1 || warp == 2) {
+    // two MMA threads, one per accumulator: warp 1 takes the even tiles of
+    // the sequence (stages 0, 2, accumulator 0), warp 2 the odd ones, so the
+    // issue latencies of their tcgen05 instructions and barrier waits overlap
     if (lane == 0) {
       const int npad = (np + 15) & ~15;
       const uint32_t idesc = idesc_bf16_f32(kTileRows, npad);
       const uint32_t b_base = smem_u32(s.bop);
+      const uint32_t mine = static_cast<uint32_t>(warp - 1);
       for (int j = 0; j < n_tiles; ++j) {
         const uint32_t q = seq + j, st = q % kStages, a = q & 1;
+        if (a != mine) continue;
         if (!mbar_wait(full0 + 8 * st, (q / kStages) & 1, kWhereMma) ||
             !mbar_wait(tempty0 + 8 * a, ((q >> 1) & 1) ^ 1, kWhereMma)) {
           s.scal[kAbort] = 1;
@@ -151,9 +160,7 @@ __device__ void distance_pass(const Layout &s, const CUtensorMap *bmap, const CU
             umma_f16(tmem + a * 64, ad, bd, idesc, (kb | kk) != 0);
           }
         }
-        // the seed pass's epilogue still reads the staged tile (the norms)
-        // and releases the stage itself
-        if (!first) umma_commit(empty0 + 8 * st);
+        // the epilogue releases the stage once it has seen this commit
         umma_commit(tfull0 + 8 * a);
       }
     }
@@ -181,7 +188,11 @@ __device__ void distance_pass(const Layout &s, const CUtensorMap *bmap, const CU
         tmem_reg_fence(v1);
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(tempty0 + 8 * a);
+        if (lane == 0) {
+          mbar_arrive(tempty0 + 8 * a);
+          // the MMA has completed, so it no longer reads the staged tile
+          if (!first && warp == 4 + 4 * wg) mbar_arrive(empty0 + 8 * (q % kStages));
+        }
       }
       int i;
       bool valid;
@@ -310,15 +321,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_tiles = n_btiles + (g.W + kTileRows - 1) / kTileRows;
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(smem_u32(&s.bars[i]), 1);
-      mbar_init(smem_u32(&s.bars[3 + i]), 1);  // the MMA's commit (the epilogue's in the seed pass)
+      mbar_init(smem_u32(&s.bars[kBarFull + i]), 1);
+      mbar_init(smem_u32(&s.bars[kBarEmpty + i]), 1);  // one epilogue thread
     }
     for (int a = 0; a < 2; ++a) {
-      mbar_init(smem_u32(&s.bars[6 + a]), 1);
-      mbar_init(smem_u32(&s.bars[8 + a]), 4);  // one arrive per warp of its warpgroup
+      mbar_init(smem_u32(&s.bars[kBarTfull + a]), 1);
+      mbar_init(smem_u32(&s.bars[kBarTempty + a]), 4);  // one arrive per warp of its warpgroup
+      mbar_init(smem_u32(&s.bars[kBarDone + a]), 1);
     }
-    mbar_init(smem_u32(&s.bars[10]), 1);
-    mbar_init(smem_u32(&s.bars[11]), 1);  // the Gram block's MMA
+    mbar_init(smem_u32(&s.bars[kBarGram]), 1);  // the Gram block's MMA
     fence_barrier_init();
     prefetch_tensormap(&bmap);
     prefetch_tensormap(&wmap);
@@ -327,12 +338,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     tmem_alloc(smem_u32(s.tmem_slot), kTmemCols);
     tmem_relinquish();
-  }
-  // the candidate operand's padding rows are zero for good
-  for (int e = tid; e < 2 * (kCRows - kCand) * 8; e += kThreads) {
-    const int kb = e / ((kCRows - kCand) * 8), rem = e - kb * (kCRows - kCand) * 8;
-    const int r = kCand + (rem >> 3), c = rem & 7;
-    *reinterpret_cast<uint4 *>(s.cop + kb * kCBlock + sw128_offset(r, c)) = make_uint4(0u, 0u, 0u, 0u);
   }
   tc_fence_before();
   __syncthreads();
@@ -425,12 +430,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       __syncthreads();
-      // Gram block on the tensor cores: D[a][b] = cand_a . cand_b, M = 128
-      // (rows a >= kCand are the zero padding), N = kCand, K = 128, the same
-      // f32 accumulation of exact bf16 products as the distance pass
+      // Gram block on the tensor cores: D[a][b] = cand_a . cand_b, N = kCand,
+      // K = 128, the same f32 accumulation of exact bf16 products as the
+      // distance pass.  M = 128: rows a >= kCand of A run on into the next
+      // 8 KB of shared memory (the other K block, then the Gram buffer), and
+      // those rows of D are never read.
       if (warp == 1 && lane == 0) {
         tc_fence_after();
-        const uint32_t idesc = idesc_bf16_f32(kCRows, kCand);
+        const uint32_t idesc = idesc_bf16_f32(128, kCand);
         const uint32_t c_base = smem_u32(s.cop);
 #pragma unroll
         for (int kb = 0; kb < 2; ++kb) {
@@ -440,11 +447,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma_f16(tmem + kGramCol, ad, ad, idesc, (kb | kk) != 0);
           }
         }
-        umma_commit(smem_u32(&s.bars[11]));
+        umma_commit(smem_u32(&s.bars[kBarGram]));
       }
       if (warp == 4 || warp == 5) {
         // TMEM lane = candidate a: warp 4 reads rows 0..31, warp 5 rows 32..63
-        if (mbar_wait_warp(smem_u32(&s.bars[11]), gram_phase & 1, kWhereEpi)) {
+        if (mbar_wait_warp(smem_u32(&s.bars[kBarGram]), gram_phase & 1, kWhereEpi)) {
           tc_fence_after();
           const uint32_t taddr = tmem + (static_cast<uint32_t>((warp - 4) * 32) << 16) + kGramCol;
           float *row = s.gram + ((warp - 4) * 32 + lane) * kCand;
@@ -534,11 +541,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0 && seq > 0) {
     const uint32_t first = seq > kStages ? seq - kStages : 0;
     for (uint32_t q = first; q < seq; ++q)
-      mbar_wait(smem_u32(&s.bars[q % kStages]), (q / kStages) & 1, kWhereDrain);
+      mbar_wait(smem_u32(&s.bars[kBarFull + q % kStages]), (q / kStages) & 1, kWhereDrain);
   }
-  if (warp == 1 && lane == 0) {
-    umma_commit(smem_u32(&s.bars[10]));
-    mbar_wait(smem_u32(&s.bars[10]), 0, kWhereDrain);
+  if ((warp == 1 || warp == 2) && lane == 0) {
+    umma_commit(smem_u32(&s.bars[kBarDone + warp - 1]));
+    mbar_wait(smem_u32(&s.bars[kBarDone + warp - 1]), 0, kWhereDrain);
   }
   tc_fence_before();
   __syncthreads();
