@@ -25,7 +25,8 @@ void finish_score_geom(ScoreGeom *g) {
 
 size_t score_workspace_bytes(const ScoreGeom &g) {
   const size_t c = align_up(static_cast<size_t>(g.n_heads()) * g.n_obs_pad * sizeof(float), kAlign);
-  const size_t y = align_up(static_cast<size_t>(g.n_groups) * g.n_heads() *
+  const int groups = std::max(g.n_groups, mean_grouping(g).n_groups);
+  const size_t y = align_up(static_cast<size_t>(groups) * g.n_heads() *
                                 static_cast<size_t>(g.L) * sizeof(float),
                             kAlign);
   return c + y;
@@ -127,7 +128,8 @@ bkv_status run_score(const ScoreGeom &g, int dtype, const void *k, const void *r
   if (dtype == BKV_BF16) {
     st = launch_score_rowstats_tc(g, k, recent, beacons, w.c, s);
     if (st != BKV_OK) return st;
-    return launch_score_colmax_tc(g, k, recent, beacons, w.c, w.ypart, mean, s);
+    return launch_score_colmax_tc(mean ? mean_grouping(g) : g, k, recent, beacons, w.c, w.ypart,
+                                  mean, s);
   }
   st = launch_score_rowstats_simt(g, static_cast<const float *>(k),
                                   static_cast<const float *>(recent),
@@ -138,10 +140,11 @@ bkv_status run_score(const ScoreGeom &g, int dtype, const void *k, const void *r
                                   static_cast<const float *>(beacons), w.c, w.ypart, mean, s);
 }
 
-SelectInput score_select_input(const ScoreGeom &g, const ScoreWorkspace &w, bool mean) {
+SelectInput score_select_input(const ScoreGeom &g, int dtype, const ScoreWorkspace &w,
+                               bool mean) {
   SelectInput in;
   in.src = w.ypart;
-  in.n_parts = g.n_groups;
+  in.n_parts = mean && dtype == BKV_BF16 ? mean_grouping(g).n_groups : g.n_groups;
   in.part_stride = static_cast<size_t>(g.n_heads()) * static_cast<size_t>(g.L);
   in.mean = mean ? 1 : 0;
   in.inv_count = 1.0f / static_cast<float>(g.n_obs);
@@ -163,7 +166,8 @@ bkv_status score_entry(const bkv_cache_desc *desc, const void *k, int64_t L,
   const ScoreWorkspace w = carve_score_workspace(g, workspace);
   st = run_score(g, desc->dtype, k, recent_q, beacons, w, mean, s);
   if (st != BKV_OK) return st;
-  return launch_finalize_scores(score_select_input(g, w, mean), g.n_heads(), L, scores, s);
+  return launch_finalize_scores(score_select_input(g, desc->dtype, w, mean), g.n_heads(), L,
+                                scores, s);
 }
 
 }  // namespace
@@ -392,7 +396,8 @@ bkv_status bkv_compress_step(const bkv_step_args *a, int32_t *n_beacons_out, int
       st = launch_score_rowstats_tc(g, a->k, a->recent_q, bq, w.c, s);
       if (st != BKV_OK) return st;
       if (!mark(2)) return BKV_ERR_CUDA;
-      st = launch_score_colmax_tc(g, a->k, a->recent_q, bq, w.c, w.ypart, mean, s);
+      st = launch_score_colmax_tc(mean ? mean_grouping(g) : g, a->k, a->recent_q, bq, w.c, w.ypart,
+                                  mean, s);
     } else {
       st = launch_score_rowstats_simt(g, static_cast<const float *>(a->k),
                                       static_cast<const float *>(a->recent_q),
@@ -408,7 +413,7 @@ bkv_status bkv_compress_step(const bkv_step_args *a, int32_t *n_beacons_out, int
     return BKV_ERR_CUDA;
   }
   if (!mark(3)) return BKV_ERR_CUDA;
-  const SelectInput in = score_select_input(g, w, mean);
+  const SelectInput in = score_select_input(g, d->dtype, w, mean);
   const bool copy_all = keep >= a->L;
   if (!copy_all) {
     st = launch_select_topk(in, g.n_heads(), a->L, keep, idx, a->scores_out, sel_ws, sel_b, s);

@@ -34,11 +34,22 @@ struct ScoreGeom {
 // Fill the derived fields of a ScoreGeom (n_obs, padding, groups).
 void finish_score_geom(ScoreGeom *g);
 
+// The grouping of the tensor-core mean aggregation: groups of at most 256
+// observation rows (the max aggregation's are up to 512).
+inline ScoreGeom mean_grouping(const ScoreGeom &g) {
+  ScoreGeom m = g;
+  m.n_groups = (g.n_obs + 255) / 256;
+  const int per = (g.n_obs + m.n_groups - 1) / m.n_groups;
+  m.rows_per_group = (per + 15) / 16 * 16;
+  return m;
+}
+
 // Workspace sections of the scoring passes.
 struct ScoreWorkspace {
   float *c;      // [n_heads][n_obs_pad]  row normalisers (natural log units)
-  float *ypart;  // [n_groups][n_heads][L] per group of rows: max of (x - c)
-                 // (max aggregation) or sum of exp(x - c) (mean aggregation)
+  float *ypart;  // [groups][n_heads][L] per group of rows: max of (x - c)
+                 // (max aggregation) or sum of exp(x - c) (mean aggregation);
+                 // sized for the mean's (finer) grouping
 };
 size_t score_workspace_bytes(const ScoreGeom &g);
 ScoreWorkspace carve_score_workspace(const ScoreGeom &g, void *ws);

@@ -170,7 +170,7 @@ __device__ __forceinline__ void load_obs_rows_sw128(uint8_t *dst, int nrows, int
 constexpr int kP1Rows = 128;
 constexpr int kP1Keys = 256;
 constexpr int kP1Stages = 3;
-constexpr int kP1EpiWarps = 16;  // 4 warpgroups, 64 of the 256 columns each
+constexpr int kP1EpiWarps = 16;  // 4 warpgroups: 2 per tile parity, 128 of 256 columns each
 constexpr int kP1Threads = 128 + 32 * kP1EpiWarps;  // warp 0 TMA, warp 1 MMA, 4.. epilogue
 constexpr int kP1ABytes = kP1Rows * kRowBytes;     // 32 KB
 constexpr int kP1StageBytes = kP1Keys * kRowBytes; // 64 KB
@@ -209,7 +209,7 @@ __global__ void __launch_bounds__(kP1Threads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull0 + 8 * a, 1);
-      mbar_init(tempty0 + 8 * a, kP1EpiWarps);  // one arrive per epilogue warp
+      mbar_init(tempty0 + 8 * a, kP1EpiWarps / 2);  // one arrive per warp reading it
     }
     mbar_init(done, 1);
     fence_barrier_init();
@@ -273,47 +273,58 @@ __global__ void __launch_bounds__(kP1Threads, 1)
       mbar_wait(done, 0, kWhereP1Drain);
     }
   } else if (warp >= 4) {
-    // ---- epilogue: four warpgroups, each owning 64 of the 256 columns of a
-    // tile; TMEM lane = observation row, so every thread keeps its row's
-    // online max and sum of 2^(x log2 e) over its columns
+    // ---- epilogue: four warpgroups; warpgroups 0-1 take the even tiles
+    // (accumulator 0) and 2-3 the odd ones, each 128 of the 256 columns in
+    // two blocks of 64, so the two pairs read TMEM at different times and
+    // each covers the other's load latency.  TMEM lane = observation row:
+    // every thread keeps its row's online max and sum of 2^(x log2 e) over
+    // its columns
     const int wg = (warp - 4) >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const float kz = g.scale * kLog2e;
     float m = -INFINITY, ssum = 0.f;
     bool ok = true;
-    for (int t = 0; t < n_tiles && ok; ++t) {
+    for (int t = wg >> 1; t < n_tiles && ok; t += 2) {
       const int acc = t & 1;
       if (!mbar_wait_warp(tfull0 + 8 * acc, (t >> 1) & 1, kWhereP1Epi)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) +
-                             acc * kP1Keys + wg * 64;
-      const long long key_base = static_cast<long long>(t) * kP1Keys + wg * 64;
-      float va[32], vb[32];
-      tmem_ld_32x32b_x32(taddr, va);
-      tmem_ld_32x32b_x32(taddr + 32, vb);
-      tmem_ld_wait_regs(va);
-      tmem_reg_fence(vb);
-      // the accumulator buffer is free as soon as both loads have landed
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
-      if (key_base + 64 > L) {  // the ragged end of the keys
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          if (key_base + i >= L) va[i] = -INFINITY;
-          if (key_base + 32 + i >= L) vb[i] = -INFINITY;
+#pragma unroll 1
+      for (int b = 0; b < 2; ++b) {
+        const int col = (wg & 1) * 128 + b * 64;
+        const uint32_t taddr =
+            tmem + (static_cast<uint32_t>(quarter * 32) << 16) + acc * kP1Keys + col;
+        const long long key_base = static_cast<long long>(t) * kP1Keys + col;
+        float va[32], vb[32];
+        tmem_ld_32x32b_x32(taddr, va);
+        tmem_ld_32x32b_x32(taddr + 32, vb);
+        tmem_ld_wait_regs(va);
+        tmem_reg_fence(vb);
+        if (b == 1) {
+          // the accumulator is free once this warp's last loads have landed
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
         }
+        if (key_base + 64 > L) {  // the ragged end of the keys
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            if (key_base + i >= L) va[i] = -INFINITY;
+            if (key_base + 32 + i >= L) vb[i] = -INFINITY;
+          }
+        }
+        // one running-max update per 64 columns, then 32 independent exp pairs
+        const float mz = fmaxf(max32(va), max32(vb)) * kz;
+        const float m_new = fmaxf(m, mz);
+        ssum = m_new == -INFINITY ? 0.f : ssum * ex2_approx(m - m_new);
+        m = m_new;
+        if (m != -INFINITY) ssum += chunk_exp_sum(va, kz, m) + chunk_exp_sum(vb, kz, m);
       }
-      // one running-max update per 64 columns, then 32 independent exp pairs
-      const float mz = fmaxf(max32(va), max32(vb)) * kz;
-      const float m_new = fmaxf(m, mz);
-      ssum = m_new == -INFINITY ? 0.f : ssum * ex2_approx(m - m_new);
-      m = m_new;
-      if (m != -INFINITY) ssum += chunk_exp_sum(va, kz, m) + chunk_exp_sum(vb, kz, m);
     }
-    // combine the four column quarters of each row; the exchange reuses the
-    // key stages, free once the last tile's MMAs have completed
+    // combine the four warpgroups' partial sums of each row; the exchange
+    // reuses the key stages, free once every tile's MMAs have completed --
+    // which the warpgroup of the last tile has seen, so all wait for it
+    named_barrier_sync(1, 32 * kP1EpiWarps);
     float *xchg = reinterpret_cast<float *>(sB);  // [3][128][2]
     if (wg > 0) {
       xchg[((wg - 1) * kP1Rows + row) * 2] = m;
@@ -349,9 +360,12 @@ __global__ void __launch_bounds__(kP1Threads, 1)
 }
 
 // ------------------------------------------------------------------ pass 2
-// Max aggregation: two epilogue warpgroups, one per column sub-chunk.  Mean
-// aggregation (an exp per element instead of a max) splits each sub-chunk's
-// 32-column pieces between two warpgroups, four in all.
+// Max aggregation: two epilogue warpgroups, one per column sub-chunk of up to
+// 256 observation rows.  Mean aggregation (an exp per element instead of a
+// max) takes groups of at most 256 rows, so that a tile's accumulator fills
+// half of TMEM and the MMA can run one tile ahead of the exps: four epilogue
+// warpgroups, two on the even tiles (TMEM columns 0..255) and two on the odd
+// ones (256..511), each pair splitting the columns in halves.
 constexpr int kP2Keys = 128;
 constexpr int kP2TileBytes = kP2Keys * kRowBytes;  // 32 KB
 constexpr int kP2ExtraRowBytes = 32;              // the extra K=16 step, 32-byte swizzle
@@ -421,7 +435,7 @@ __global__ void __launch_bounds__(p2_threads(kMean), 1)
     }
     for (int u = 0; u < 2; ++u) {
       mbar_init(tfull0 + 8 * u, 1);
-      mbar_init(tempty0 + 8 * u, 4 * kSplit);  // one arrive per warp reading it
+      mbar_init(tempty0 + 8 * u, kMean ? 8 : 4);  // one arrive per warp reading it
     }
     mbar_init(done, 1);
     fence_barrier_init();
@@ -495,9 +509,13 @@ __global__ void __launch_bounds__(p2_threads(kMean), 1)
         if (!mbar_wait(full0 + 8 * s, (it / n_stages) & 1, kWhereP2Mma)) break;
         const uint32_t a_base = smem_u32(sK + s * kP2TileBytes);
         for (int u = 0; u < n_sub; ++u) {
-          if (!mbar_wait(tempty0 + 8 * u, (it & 1) ^ 1, kWhereP2Mma)) { ok = false; break; }
+          // max: one accumulator per sub-chunk; mean (one sub-chunk): one per
+          // tile parity
+          const int buf = kMean ? (it & 1) : u;
+          const uint32_t par = kMean ? (((it >> 1) & 1) ^ 1) : ((it & 1) ^ 1);
+          if (!mbar_wait(tempty0 + 8 * buf, par, kWhereP2Mma)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t d = tmem + u * 256;
+          const uint32_t d = tmem + buf * 256;
           const uint32_t b_rows = q_base + u * N0 * kKbBytes;
           const uint32_t idesc = u == 0 ? idesc0 : idesc1;
 #pragma unroll
@@ -511,14 +529,85 @@ __global__ void __launch_bounds__(p2_threads(kMean), 1)
           }
           umma_f16(d, smem_desc_k_sw32(smem_u32(sXk)),
                    smem_desc_k_sw32(smem_u32(sXq) + u * N0 * kP2ExtraRowBytes), idesc, 1u);
-          umma_commit(tfull0 + 8 * u);
+          umma_commit(tfull0 + 8 * buf);
         }
         umma_commit(empty0 + 8 * s);
       }
       umma_commit(done);
       mbar_wait(done, 0, kWhereP2Drain);
     }
-  } else if (warp >= 4) {
+  } else if (kMean && warp >= 4) {
+    // Warpgroup e takes the tiles of parity e >> 1 and the column half e & 1
+    // of the group's rows (rows_pad <= 256, one sub-chunk); per key (TMEM
+    // lane) it sums exp(scale * acc) over its columns, releases the
+    // accumulator after its last TMEM load, and the two halves' sums meet in
+    // shared memory.
+    const int e = (warp - 4) >> 2;
+    const int par = e >> 1, h = e & 1;
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;  // key within the tile
+    const float kz = g.scale * kLog2e;
+    float *yout = ypart + (static_cast<size_t>(gi) * g.n_heads() + head) * static_cast<size_t>(L);
+    const int c0 = h * 128, c1 = min(N0, c0 + 128);
+    const int n32 = c1 > c0 ? (c1 - c0) >> 5 : 0;
+    const bool tail16 = c1 > c0 && ((c1 - c0) & 16) != 0;  // N0 is a multiple of 16
+    bool ok = true;  // warp-uniform; after a timeout only the barriers remain
+    for (int it = par; it < n_tiles; it += 2) {
+      const int buf = it & 1;  // == par
+      float y = 0.f;
+      if (ok && !mbar_wait_warp(tfull0 + 8 * buf, (it >> 1) & 1, kWhereP2Epi)) ok = false;
+      if (ok) {
+        tc_fence_after();
+        const uint32_t taddr =
+            tmem + (static_cast<uint32_t>(quarter * 32) << 16) + buf * 256 + c0;
+        bool released = false;
+        auto release = [&]() {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(tempty0 + 8 * buf);
+          released = true;
+        };
+        // two TMEM loads in flight; the accumulator is handed back as soon as
+        // the last of this warp's loads has landed
+        float va[32], vb[32];
+        int i = 0;
+        if (n32 > 0) {
+          tmem_ld_32x32b_x32(taddr, va);
+          tmem_ld_wait_regs(va);
+          if (n32 == 1 && !tail16) release();
+        }
+#pragma unroll 1
+        for (; i + 2 <= n32; i += 2) {
+          tmem_ld_32x32b_x32(taddr + (i + 1) * 32, vb);
+          y += chunk_exp_sum(va, kz, 0.f);
+          tmem_ld_wait_regs(vb);
+          if (i + 2 == n32 && !tail16) release();
+          if (i + 2 < n32) tmem_ld_32x32b_x32(taddr + (i + 2) * 32, va);
+          y += chunk_exp_sum(vb, kz, 0.f);
+          if (i + 2 < n32) {
+            tmem_ld_wait_regs(va);
+            if (i + 3 == n32 && !tail16) release();
+          }
+        }
+        if (i < n32) y += chunk_exp_sum(va, kz, 0.f);
+        if (tail16) {
+          float v[16];
+          tmem_ld_32x32b_x16(taddr + n32 * 32, v);
+          tmem_ld_wait_regs(v);
+          release();
+          y += chunk_exp_sum(v, kz, 0.f);
+        }
+        if (!released) release();  // a half with no columns
+      }
+      float *slot = ybuf + (par * 2 + ((it >> 1) & 1)) * 128;
+      if (h == 1) slot[row] = y;
+      named_barrier_sync(1 + par, 256);
+      if (h == 0 && ok) {
+        const long long j = static_cast<long long>(t0 + it) * kP2Keys + row;
+        if (j < L) yout[j] = y + slot[row];
+      }
+    }
+  } else if (!kMean && warp >= 4) {
     // Warpgroup e = u * kSplit + h reads column sub-chunk u, its 32-column
     // pieces h, h + kSplit, ...; per key (TMEM lane) it reduces
     // acc = q . k - c_o / scale over them: the max (max aggregation) or the
