@@ -4,20 +4,23 @@
 // Same exact speculative rounds as fps.cu (select the T+1 best unselected
 // points; Gram block of the T candidates; replay the greedy choice among
 // them while the best one provably beats every other point; lower all
-// distances by the round's picks), with T = 64 and a different distance pass:
-// the union [beacons; window] of a query head is streamed by TMA in tiles of
-// 128 points (128-byte swizzle, no multicast) into a 3-stage ring, one thread
-// issues D[128 points][N] = tile . picks^T (M=128, N = picks rounded up to 16,
-// K = 128) into a double-buffered TMEM accumulator, and four epilogue warps
-// (TMEM lane = point) turn the dot products into cosine distances and lower
-// the shared-memory distance array.  The candidates' Gram block is formed on
-// the CUDA cores in f32; bf16 products are exact in f32 on either path, the
-// two sums may differ in their last bit, which can only reorder picks whose
-// distances agree to about 1e-7.
-//
+// distances by the round's picks), with T = 64 and the contractions on the
+// tensor cores:
+//   * the distance pass streams the union [beacons; window] of a query head
+//     by TMA in tiles of 128 points (128-byte swizzle, no multicast) through a
+//     4-stage ring and forms D[128 points][N] = tile . picks^T (M = 128, N =
+//     picks rounded up to 16, K = 128) in one of two TMEM accumulators.  Two
+//     threads issue the MMAs, warp 1 for the even tiles of the sequence
+//     (stages 0 and 2, accumulator 0) and warp 2 for the odd ones, so their
+//     instruction latencies overlap and every stage and accumulator keeps a
+//     single consumer.  Two epilogue warpgroups (TMEM lane = point) turn the
+//     dot products into cosine distances and lower the distance array;
+//   * the candidates' rows are staged in the MMA's swizzled layout and one
+//     M = 128 x N = 64 MMA forms their Gram block, the same f32 sums of exact
+//     bf16 products as the distance pass.
 // While a round selects, the first tiles of its coming pass are already
-// loaded into the ring.  After the seed pass a ring stage is released by the
-// MMA's commit alone.
+// loaded into the ring.  After the seed pass (whose epilogue also reads the
+// staged tiles for the norms) a stage is released by the MMA's commit.
 //
 // The grid is persistent: one CTA per SM loops over the query heads.  The
 // distance and inverse-norm arrays live in shared memory, or for a union too
@@ -160,7 +163,9 @@ __device__ void distance_pass(const Layout &s, const CUtensorMap *bmap, const CU
             umma_f16(tmem + a * 64, ad, bd, idesc, (kb | kk) != 0);
           }
         }
-        // the epilogue releases the stage once it has seen this commit
+        // the stage is free once these MMAs complete (in the seed pass the
+        // epilogue still reads it for the norms and releases it itself)
+        if (!first) umma_commit(empty0 + 8 * st);
         umma_commit(tfull0 + 8 * a);
       }
     }
@@ -188,11 +193,7 @@ __device__ void distance_pass(const Layout &s, const CUtensorMap *bmap, const CU
         tmem_reg_fence(v1);
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(tempty0 + 8 * a);
-          // the MMA has completed, so it no longer reads the staged tile
-          if (!first && warp == 4 + 4 * wg) mbar_arrive(empty0 + 8 * (q % kStages));
-        }
+        if (lane == 0) mbar_arrive(tempty0 + 8 * a);
       }
       int i;
       bool valid;
@@ -322,7 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) {
       mbar_init(smem_u32(&s.bars[kBarFull + i]), 1);
-      mbar_init(smem_u32(&s.bars[kBarEmpty + i]), 1);  // one epilogue thread
+      mbar_init(smem_u32(&s.bars[kBarEmpty + i]), 1);  // the MMA's commit (seed pass: the epilogue)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(smem_u32(&s.bars[kBarTfull + a]), 1);
