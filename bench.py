@@ -504,11 +504,12 @@ def main():
                      device=dev)
     stream = torch.cuda.current_stream()
 
-    def step(events=None, t=devt):
+    def step(events=None, t=devt, o=None, st=None):
+        o = o or {"kd": kd, "vd": vd, "bout": bout, "idx": idx}
         return bkv.bkv_compress_step(g, t["k"], t["v"], wl.L, wl.K, t["recent"], wl.R,
                                      t["beacons"], wl.beacons_in, wl.M,
-                                     t["window"] if wl.W else None, wl.W, bout, 0.0, dstg, kd,
-                                     vd, None, idx, ws, stream, events,
+                                     t["window"] if wl.W else None, wl.W, o["bout"], 0.0, dstg,
+                                     o["kd"], o["vd"], None, o["idx"], ws, st or stream, events,
                                      aggregate=args.aggregate)
 
     for _ in range(args.warmup):
@@ -549,27 +550,52 @@ def main():
     entries = wl.n_layers * wl.n_kv_heads * wl.L
     value = weak_scaling_value(entries, world, ms)
 
-    # ---- end to end: pinned host inputs in, compacted cache out, every step
+    # ---- end to end: pinned host inputs in, compacted cache out, every step.
+    # Steps are pipelined over three streams as a serving loop would: step
+    # i+1's inputs upload (into the other of two device input sets) while
+    # step i computes and step i-1's outputs download (from the other of two
+    # output sets); each step's copies and compute still all happen.
     e2e_steps = args.e2e_steps or max(3, min(args.steps, 10))
-    out_host = {"kd": torch.empty_like(kd, device="cpu").pin_memory(),
-                "vd": torch.empty_like(vd, device="cpu").pin_memory(),
-                "bout": torch.empty_like(bout, device="cpu").pin_memory(),
-                "idx": torch.empty_like(idx, device="cpu").pin_memory()}
+    outs = [{"kd": kd, "vd": vd, "bout": bout, "idx": idx},
+            {"kd": torch.empty_like(kd), "vd": torch.empty_like(vd),
+             "bout": torch.empty_like(bout), "idx": torch.empty_like(idx)}]
+    ins = [devt, {n: torch.empty_like(devt[n]) for n in names}]
+    out_host = {n: torch.empty_like(kd if n in ("kd", "vd") else outs[0][n],
+                                    device="cpu").pin_memory()
+                for n in ("kd", "vd", "bout", "idx")}
     h2d = sum(host[n].numel() * host[n].element_size() for n in names if n != "window" or wl.W)
     d2h = sum(t.numel() * t.element_size() for t in out_host.values())
+    s_up, s_down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(e2e_steps)]
+    ev_done = [torch.cuda.Event() for _ in range(e2e_steps)]
+    ev_out = [torch.cuda.Event() for _ in range(e2e_steps)]
     barrier()
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(e2e_steps):
-        for n in names:
-            devt[n].copy_(host[n], non_blocking=True)
-        step()
-        out_host["kd"].copy_(kd, non_blocking=True)
-        out_host["vd"].copy_(vd, non_blocking=True)
-        out_host["bout"].copy_(bout, non_blocking=True)
-        out_host["idx"].copy_(idx, non_blocking=True)
+    s_up.wait_stream(stream)
+    s_down.wait_stream(stream)
+    for i in range(e2e_steps):
+        b = i & 1
+        with torch.cuda.stream(s_up):
+            if i >= 2:
+                s_up.wait_event(ev_done[i - 2])  # input set b is free again
+            for n in names:
+                if n != "window" or wl.W:
+                    ins[b][n].copy_(host[n], non_blocking=True)
+            ev_in[i].record(s_up)
+        stream.wait_event(ev_in[i])
+        if i >= 2:
+            stream.wait_event(ev_out[i - 2])  # output set b has been read back
+        step(t=ins[b], o=outs[b], st=stream)
+        ev_done[i].record(stream)
+        with torch.cuda.stream(s_down):
+            s_down.wait_event(ev_done[i])
+            for n in ("kd", "vd", "bout", "idx"):
+                out_host[n].copy_(outs[b][n], non_blocking=True)
+            ev_out[i].record(s_down)
+    stream.wait_stream(s_down)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()

@@ -69,11 +69,16 @@ __device__ __forceinline__ bool before(float da, int ia, float db, int ib) {
 // Scratch: whist[kThreads / 32 * 256] (>= 2 * kRankMax words), hist[256], scal[>= 8].
 constexpr int kRankMax = 256;
 
+// With have_range, scal[6] and scal[7] already hold (as unsigned) a lower
+// bound of the live keys' minimum and their maximum, and the first pass over
+// the keys is skipped.
 template <int kThreads>
 __device__ void select_best(const float *dist, int n, int n_live, int want, uint32_t *whist,
-                            uint32_t *hist, int *scal, int *cidx, float *cdist) {
+                            uint32_t *hist, int *scal, int *cidx, float *cdist,
+                            bool have_range = false) {
   constexpr int kWarps = kThreads / 32;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (!have_range) {
   // common prefix of the live keys
   uint32_t kmin = 0xffffffffu, kmax = 0u;
   for (int i = tid; i < n; i += kThreads) {
@@ -100,6 +105,7 @@ __device__ void select_best(const float *dist, int n, int n_live, int want, uint
     scal[7] = static_cast<int>(b);
   }
   __syncthreads();
+  }
   const uint32_t gmin = static_cast<uint32_t>(scal[7]) == 0u ? 0u : static_cast<uint32_t>(scal[6]);
   const uint32_t diff = gmin ^ static_cast<uint32_t>(scal[7]);
   int hi = diff == 0u ? 0 : 32 - __clz(diff);  // bits [hi, 32) are shared

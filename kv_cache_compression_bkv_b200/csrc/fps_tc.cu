@@ -231,40 +231,50 @@ __device__ void distance_pass(const Layout &s, const CUtensorMap *bmap, const CU
       }
       if (first && ok && warp == 4 + 4 * wg && lane == 0) mbar_arrive(empty0 + 8 * st);
       if (!ok) continue;
-      if (!valid) continue;
-      float di = first ? 2.f : s.dist[i];
-      if (di < 0.f) continue;  // already selected
-      // x_k = 1 - dot_k * inv_i * inv_k, as cos_dist computes it; padded
-      // picks carry a NaN inverse norm, which min ignores
-      const float inv_i = s.inv[i];
-      const float2 ninv = make_float2(-inv_i, -inv_i);
-      float mn = INFINITY;
-#pragma unroll
-      for (int k = 0; k < 32; k += 4) {
-        if (k < npad) {
-          const float4 pv = *reinterpret_cast<const float4 *>(s.pinv + k);
-          const float2 x0 = __ffma2_rn(__fmul2_rn(make_float2(v0[k], v0[k + 1]), ninv),
-                                       make_float2(pv.x, pv.y), make_float2(1.f, 1.f));
-          const float2 x1 = __ffma2_rn(__fmul2_rn(make_float2(v0[k + 2], v0[k + 3]), ninv),
-                                       make_float2(pv.z, pv.w), make_float2(1.f, 1.f));
-          mn = fminf(mn, fminf(fminf(x0.x, x0.y), fminf(x1.x, x1.y)));
-        }
-      }
-      if (npad > 32) {
+      const float di = !valid ? -1.f : first ? 2.f : s.dist[i];
+      // the range of the new keys, which the next selection starts from
+      uint32_t kmn = 0xffffffffu, kmx = 0u;
+      if (di >= 0.f) {  // a point not yet selected
+        // x_k = 1 - dot_k * inv_i * inv_k, as cos_dist computes it; padded
+        // picks carry a NaN inverse norm, which min ignores
+        const float inv_i = s.inv[i];
+        const float2 ninv = make_float2(-inv_i, -inv_i);
+        float mn = INFINITY;
 #pragma unroll
         for (int k = 0; k < 32; k += 4) {
-          if (k + 32 < npad) {
-            const float4 pv = *reinterpret_cast<const float4 *>(s.pinv + 32 + k);
-            const float2 x0 = __ffma2_rn(__fmul2_rn(make_float2(v1[k], v1[k + 1]), ninv),
+          if (k < npad) {
+            const float4 pv = *reinterpret_cast<const float4 *>(s.pinv + k);
+            const float2 x0 = __ffma2_rn(__fmul2_rn(make_float2(v0[k], v0[k + 1]), ninv),
                                          make_float2(pv.x, pv.y), make_float2(1.f, 1.f));
-            const float2 x1 = __ffma2_rn(__fmul2_rn(make_float2(v1[k + 2], v1[k + 3]), ninv),
+            const float2 x1 = __ffma2_rn(__fmul2_rn(make_float2(v0[k + 2], v0[k + 3]), ninv),
                                          make_float2(pv.z, pv.w), make_float2(1.f, 1.f));
             mn = fminf(mn, fminf(fminf(x0.x, x0.y), fminf(x1.x, x1.y)));
           }
         }
+        if (npad > 32) {
+#pragma unroll
+          for (int k = 0; k < 32; k += 4) {
+            if (k + 32 < npad) {
+              const float4 pv = *reinterpret_cast<const float4 *>(s.pinv + 32 + k);
+              const float2 x0 = __ffma2_rn(__fmul2_rn(make_float2(v1[k], v1[k + 1]), ninv),
+                                           make_float2(pv.x, pv.y), make_float2(1.f, 1.f));
+              const float2 x1 = __ffma2_rn(__fmul2_rn(make_float2(v1[k + 2], v1[k + 3]), ninv),
+                                           make_float2(pv.z, pv.w), make_float2(1.f, 1.f));
+              mn = fminf(mn, fminf(fminf(x0.x, x0.y), fminf(x1.x, x1.y)));
+            }
+          }
+        }
+        // min(di, clamp(x, 0, 2)) == max(min(di, x), 0) for di in [0, 2]
+        const float nd = fmaxf(fminf(di, mn), 0.f);
+        s.dist[i] = nd;
+        kmn = kmx = dist_key(nd);
       }
-      // min(di, clamp(x, 0, 2)) == max(min(di, x), 0) for di in [0, 2]
-      s.dist[i] = fmaxf(fminf(di, mn), 0.f);
+      kmn = __reduce_min_sync(0xffffffffu, kmn);
+      kmx = __reduce_max_sync(0xffffffffu, kmx);
+      if (lane == 0) {
+        atomicMin(reinterpret_cast<unsigned int *>(&s.scal[6]), kmn);
+        atomicMax(reinterpret_cast<unsigned int *>(&s.scal[7]), kmx);
+      }
     }
   }
 }
@@ -365,6 +375,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       s.pinv[0] = ss > 0.f ? 1.0f / sqrtf(ss) : 0.f;
     }
     if (tid > 0 && tid < 16) s.pinv[tid] = __int_as_float(0x7fc00000);
+    if (tid == 0) {  // the seed pass gathers the range of its keys (the seed's
+      s.scal[6] = -1;  // own 0 among them: a lower bound is all it needs)
+      s.scal[7] = 0;
+    }
     __syncthreads();
     stage_picks(s, h, out, 0, 1, true);
     fence_proxy_async_smem();
@@ -387,7 +401,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int pre = min(kStages, n_tiles);
       if (tid == 0 && !issue_tiles(s, &bmap, &wmap, qh, g, n_btiles, seq, 0, pre))
         s.scal[kAbort] = 1;
-      select_best<kThreads>(s.dist, n, unsel, want, s.whist, s.hist, s.scal, s.cidx, s.cdist);
+      select_best<kThreads>(s.dist, n, unsel, want, s.whist, s.hist, s.scal, s.cidx, s.cdist,
+                            true);  // the pass left the key range in scal[6..7]
       __syncthreads();
       // the candidates need no order; only the bound (the last of the kCand+1
       // selected in (distance desc, index asc) order) moves to slot kCand
@@ -526,6 +541,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       stage_picks(s, h, out, picked, np, false);
       __syncthreads();
       if (tid < np) s.dist[s.cidx[s.pick[tid]]] = -1.f;
+      if (tid == 0) {  // the coming pass gathers the range of its new keys
+        s.scal[6] = -1;
+        s.scal[7] = 0;
+      }
       fence_proxy_async_smem();
       __syncthreads();
       distance_pass(s, &bmap, &wmap, tmem, qh, g, n_btiles, n_tiles, seq, np, false, pre);
