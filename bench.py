@@ -233,6 +233,8 @@ def workload_config(wl, args) -> dict:
            "M": wl.M, "K": wl.K, "W": wl.W}
     if args.aggregate != "max":
         cfg["aggregate"] = args.aggregate
+    if getattr(args, "in_place", False):
+        cfg["compaction"] = "in place"
     return cfg
 
 
@@ -443,6 +445,9 @@ def main():
                     help="use only this many layers (small cases for profiler captures)")
     ap.add_argument("--aggregate", default="max", choices=["max", "mean"],
                     help="aggregation over the observation rows (mean: Table 2's ablation)")
+    ap.add_argument("--in-place", action="store_true",
+                    help="compact into the scored cache itself (bkv_compress_step with "
+                         "k_dst == k)")
     ap.add_argument("--rm-sweep", default=None,
                     help="comma-separated R:M splits (Table 1): time the step for each")
     ap.add_argument("--budget", type=int, default=2048, help="K for --rm-sweep")
@@ -496,8 +501,15 @@ def main():
     devt = {n: torch.empty_like(host[n], device=dev) for n in names}
     for n in names:
         devt[n].copy_(host[n])
-    kd = torch.empty(wl.n_layers, wl.n_kv_heads, keep, wl.head_dim, dtype=inp.k.dtype, device=dev)
-    vd = torch.empty_like(kd)
+    if args.in_place:
+        # the step compacts the cache it scored (each timed step then sees the
+        # previous step's result: the same work on other data)
+        dstg = g
+        kd, vd = devt["k"][:, :, :keep], devt["v"][:, :, :keep]
+    else:
+        kd = torch.empty(wl.n_layers, wl.n_kv_heads, keep, wl.head_dim, dtype=inp.k.dtype,
+                         device=dev)
+        vd = torch.empty_like(kd)
     bout = torch.empty_like(devt["beacons"])
     idx = torch.empty(wl.n_layers, wl.n_kv_heads, keep, dtype=torch.int32, device=dev)
     ws = torch.empty(bkv.bkv_workspace_size(g, wl.L, wl.R, wl.M, wl.W, wl.K), dtype=torch.uint8,
@@ -556,12 +568,16 @@ def main():
     # step i computes and step i-1's outputs download (from the other of two
     # output sets); each step's copies and compute still all happen.
     e2e_steps = args.e2e_steps or max(3, min(args.steps, 10))
-    outs = [{"kd": kd, "vd": vd, "bout": bout, "idx": idx},
-            {"kd": torch.empty_like(kd), "vd": torch.empty_like(vd),
-             "bout": torch.empty_like(bout), "idx": torch.empty_like(idx)}]
     ins = [devt, {n: torch.empty_like(devt[n]) for n in names}]
-    out_host = {n: torch.empty_like(kd if n in ("kd", "vd") else outs[0][n],
-                                    device="cpu").pin_memory()
+    if args.in_place:
+        outs = [{"kd": ins[b]["k"][:, :, :keep], "vd": ins[b]["v"][:, :, :keep],
+                 "bout": bout if b == 0 else torch.empty_like(bout),
+                 "idx": idx if b == 0 else torch.empty_like(idx)} for b in range(2)]
+    else:
+        outs = [{"kd": kd, "vd": vd, "bout": bout, "idx": idx},
+                {"kd": torch.empty_like(kd), "vd": torch.empty_like(vd),
+                 "bout": torch.empty_like(bout), "idx": torch.empty_like(idx)}]
+    out_host = {n: torch.empty(outs[0][n].shape, dtype=outs[0][n].dtype).pin_memory()
                 for n in ("kd", "vd", "bout", "idx")}
     h2d = sum(host[n].numel() * host[n].element_size() for n in names if n != "window" or wl.W)
     d2h = sum(t.numel() * t.element_size() for t in out_host.values())
@@ -610,7 +626,7 @@ def main():
     wm = work_model(wl)
     # the captured counters are those of the default configuration
     traffic = (load_traffic() if args.workload == "qwen3_14b" and not args.layers
-               and args.aggregate == "max" else {})
+               and args.aggregate == "max" and not args.in_place else {})
     phases = {}
     for p in PHASES:
         m = wm[p]
