@@ -134,8 +134,9 @@ bkv_status bkv_compact(const bkv_cache_desc *src, const void *k_src,
                        void *stream);
 
 /* Compaction in place: the same result as bkv_compact with the cache as both
- * source and destination, without a second cache (SURVEY's "ordered chunked
- * in-place gather"; the page evicts rows but says nothing of buffers).  For
+ * source and destination, without a second cache (an ordered, chunked gather
+ * within one buffer; the BeaconKV page evicts rows, Fig. 5(a), but says
+ * nothing of buffers).  For
  * every (layer, KV head) r and i < n_keep, in increasing i:
  *   k[r][i][:] = k[r][idx[r][i]][:],  v likewise.
  *   idx  device, int32 [Ly*Hkv][n_keep]; every idx[r][i] must satisfy

@@ -55,7 +55,7 @@ constexpr int kBBlock = kCand * 128;              // one 64-element K block of t
 constexpr int kBBytes = 2 * kBBlock;              // 16 KB
 constexpr int kCRows = kCand;                     // candidate operand rows
 constexpr int kCBlock = kCRows * 128;             // one 64-element K block of the candidates
-constexpr int kCBytes = 2 * kCBlock;              // 32 KB
+constexpr int kCBytes = 2 * kCBlock;              // 16 KB
 constexpr int kSmallBytes = 4096;
 constexpr int kFixedBytes = kSmallBytes + 1024 + kStages * kTileBytes + kBBytes +
                             kCBytes + kCand * kCand * 4 + kWarps * 256 * 4;
@@ -102,10 +102,6 @@ __device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-// One distance pass over every tile of the head: producer (warp 0), MMA
-// issuer (warp 1) and epilogue (warps 4..7) run their own loops; `seq` is the
-// number of tiles all passes so far have moved through the ring, so every
-// role derives the same stage and phase for each tile.
 // Issue the TMA loads of tiles [j0, j1) of the pass that starts at `seq`
 // (producer thread only).  Returns false after a timeout.
 __device__ bool issue_tiles(const Layout &s, const CUtensorMap *bmap, const CUtensorMap *wmap,
@@ -125,6 +121,11 @@ __device__ bool issue_tiles(const Layout &s, const CUtensorMap *bmap, const CUte
   return true;
 }
 
+// One distance pass over every tile of the head: the producer (warp 0), the
+// two MMA threads (warps 1 and 2) and the epilogue warpgroups (warps 4..11)
+// run their own loops; `seq` is the number of tiles all passes so far have
+// moved through the ring, so every role derives the same stage, accumulator
+// and barrier phase for each tile.
 __device__ void distance_pass(const Layout &s, const CUtensorMap *bmap, const CUtensorMap *wmap,
                               uint32_t tmem, int qh, const FpsGeom &g, int n_btiles, int n_tiles,
                               uint32_t seq, int np, bool first, int prefetched) {
