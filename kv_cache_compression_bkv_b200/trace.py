@@ -7,6 +7,7 @@ window), scores the cache with the recent and beacon queries, keeps the
 budget K and compacts into the other of two cache buffers.  The decode step
 itself is not simulated: the keys, values and queries of each interval come
 from the seeded trace generator (synth.trace_*) and are appended in one copy.
+With in_place the step compacts into the cache it scored (one cache buffer).
 """
 from __future__ import annotations
 
@@ -34,6 +35,7 @@ class TraceRun:
     seed: int
     device: torch.device
     layers: int | None = None      # use only the first `layers` layers
+    in_place: bool = False         # compact into the cache itself (one cache buffer)
     events: list[TraceEvent] = field(default_factory=list)
 
     def __post_init__(self):
@@ -53,7 +55,10 @@ class TraceRun:
                 self.queries[l, q] = synth.trace_queries(tr, self.seed, l, q).to(dt)
         dev = self.device
         self.cache = [(torch.zeros(Ly, Hkv, self.cap, d, dtype=dt, device=dev),
-                       torch.zeros(Ly, Hkv, self.cap, d, dtype=dt, device=dev)) for _ in range(2)]
+                       torch.zeros(Ly, Hkv, self.cap, d, dtype=dt, device=dev))
+                      for _ in range(1 if self.in_place else 2)]
+        if self.in_place:  # source and destination are the same buffers
+            self.cache.append(self.cache[0])
         self.beacons = [torch.zeros(Ly, Hq, tr.M, d, dtype=dt, device=dev) for _ in range(2)]
         self.window = torch.empty(Ly, Hq, tr.interval, d, dtype=dt, device=dev)
         self.recent = torch.empty(Ly, Hq, tr.R, d, dtype=dt, device=dev)

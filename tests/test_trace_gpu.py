@@ -21,14 +21,15 @@ from parity_helpers import check_fps, check_topk, f64, picks_from_rows, raw
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
 
-def test_qwen3_4b_trace_follows_the_oracle_trace():
+@pytest.mark.parametrize("in_place", [False, True])
+def test_qwen3_4b_trace_follows_the_oracle_trace(in_place):
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA device")
     from kv_cache_compression_bkv_b200 import synth
     from kv_cache_compression_bkv_b200.trace import TraceRun
 
     tr = synth.TRACES["qwen3_4b_trace"]
-    run = TraceRun(tr, seed=0, device=torch.device("cuda:0"), layers=1)
+    run = TraceRun(tr, seed=0, device=torch.device("cuda:0"), layers=1, in_place=in_place)
     G, Hkv, I, K, M, R = tr.group, tr.n_kv_heads, tr.interval, tr.K, tr.M, tr.R
     keys_raw = raw(run.keys[0])          # [Hkv, steps, d]
     vals_raw = raw(run.values[0])
