@@ -78,18 +78,27 @@ __device__ __forceinline__ float max32(const float (&v)[32]) {
   return max3f(b, c, e);
 }
 
-// 2^x on the FMA pipe, for a pair of x <= 0: Cody-Waite reduction x = j + f
-// with j = rint(x) (by adding 1.5 * 2^23) and f in [-0.5, 0.5]; a cubic
-// p(f) ~ 2^f (coefficients from fit_exp2_poly.py, max relative error 7.6e-5);
-// then 2^j is added into p's exponent field.  x is clamped at -126, so the
-// smallest result is about 1e-38 instead of 0.
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
-  x.x = fmaxf(x.x, -126.f);
-  x.y = fmaxf(x.y, -126.f);
-  const float2 t = __fadd2_rn(x, make_float2(kMagic, kMagic));
-  const float2 j = __fadd2_rn(t, make_float2(-kMagic, -kMagic));
-  const float2 f = __ffma2_rn(j, make_float2(-1.f, -1.f), x);
+// Saturating FMA: min(max(a * b + c, 0), 1) (NaN gives 0).
+__device__ __forceinline__ float fma_sat(float a, float b, float c) {
+  float r;
+  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^(v * kz - m) on the FMA pipe, for a pair.  One saturating FMA per element
+// maps x = v * kz - m from [-126, 128] onto y = (x + 126) / 254 in [0, 1], so
+// that x below the range gives about 2^-126, x above it (and m = -inf) about
+// 2^127, and NaN 2^-126; then Cody-Waite reduction of x' = 254 y - 126 =
+// j + f, j = rint(x') by adding 1.5 * 2^23, f in [-0.5, 0.5]; a cubic p(f) ~
+// 2^f (coefficients from fit_exp2_poly.py, max relative error 7.6e-5); and
+// 2^j added into p's exponent field, which stays in [0, 254].  `a` = kz / 254
+// and `b` = (126 - m) / 254 are the mapping's coefficients.
+__device__ __forceinline__ float2 exp2_poly2(float vx, float vy, float a, float b) {
+  constexpr float kBase = 12582912.0f - 126.f;  // 1.5 * 2^23 - 126, exact
+  const float2 y = make_float2(fma_sat(vx, a, b), fma_sat(vy, a, b));
+  const float2 t = __ffma2_rn(y, make_float2(254.f, 254.f), make_float2(kBase, kBase));
+  const float2 u = __ffma2_rn(t, make_float2(-1.f, -1.f), make_float2(kBase, kBase));
+  const float2 f = __ffma2_rn(y, make_float2(254.f, 254.f), u);
   float2 p = __ffma2_rn(f, make_float2(0.05517051f, 0.05517051f),
                         make_float2(0.24260840f, 0.24260840f));
   p = __ffma2_rn(p, f, make_float2(0.69326091f, 0.69326091f));
@@ -100,23 +109,27 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
 }
 
 // Sum of 2^(v[i] * kz - m) over one chunk of N (32 or 16) columns.  About
-// 7 of every 16 pairs go through exp2_poly2 (FMA pipe), the rest through
-// ex2.approx (MUFU), so that both pipes share the load.
-constexpr int kPolyPairs = 7;
+// 5 of every 16 pairs go through exp2_poly2 (FMA pipe), the rest through
+// ex2.approx (MUFU), so that both pipes share the load (measured best of 0 to
+// 8 on the 14B-shaped step).  An element with v * kz - m above 128 (or
+// m = -inf) makes the sum exceed 2^126 or inf/NaN.
+constexpr int kPolyPairs = 5;
 template <int N>
 __device__ __forceinline__ float chunk_exp_sum(const float (&v)[N], float kz, float m) {
   constexpr int kPoly = (kPolyPairs * N + 16) / 32;
+  constexpr float kInv254 = 1.f / 254.f;
+  const float a = kz * kInv254, b = fmaf(-m, kInv254, 126.f * kInv254);
   const float2 kz2 = make_float2(kz, kz), nm2 = make_float2(-m, -m);
   float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
   for (int p = 0; p < N / 2; ++p) {
-    const float2 a = __ffma2_rn(make_float2(v[2 * p], v[2 * p + 1]), kz2, nm2);
     float2 e;
     if (p < kPoly) {
-      e = exp2_poly2(a);
+      e = exp2_poly2(v[2 * p], v[2 * p + 1], a, b);
     } else {
-      e.x = ex2_approx(a.x);
-      e.y = ex2_approx(a.y);
+      const float2 x = __ffma2_rn(make_float2(v[2 * p], v[2 * p + 1]), kz2, nm2);
+      e.x = ex2_approx(x.x);
+      e.y = ex2_approx(x.y);
     }
     acc = __fadd2_rn(acc, e);
   }
@@ -277,8 +290,8 @@ __global__ void __launch_bounds__(kP1Threads, 1)
     // (accumulator 0) and 2-3 the odd ones, each 128 of the 256 columns in
     // two blocks of 64, so the two pairs read TMEM at different times and
     // each covers the other's load latency.  TMEM lane = observation row:
-    // every thread keeps its row's online max and sum of 2^(x log2 e) over
-    // its columns
+    // every thread keeps its row's reference m and the sum of
+    // 2^(x log2 e - m) over its columns
     const int wg = (warp - 4) >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
@@ -313,12 +326,19 @@ __global__ void __launch_bounds__(kP1Threads, 1)
             if (key_base + 32 + i >= L) vb[i] = -INFINITY;
           }
         }
-        // one running-max update per 64 columns, then 32 independent exp pairs
-        const float mz = fmaxf(max32(va), max32(vb)) * kz;
-        const float m_new = fmaxf(m, mz);
-        ssum = m_new == -INFINITY ? 0.f : ssum * ex2_approx(m - m_new);
-        m = m_new;
-        if (m != -INFINITY) ssum += chunk_exp_sum(va, kz, m) + chunk_exp_sum(vb, kz, m);
+        // the exps of the 64 columns are taken against the row's reference m
+        // (not yet its running max); only when a sum exceeds 2^64 -- the
+        // first columns of the row (m = -inf), or a column more than 64 above
+        // m in log2 units -- does m move up to this block's max and the block
+        // is summed again.  Every value summed stays below 2^64.
+        float bs = chunk_exp_sum(va, kz, m) + chunk_exp_sum(vb, kz, m);
+        if (!(bs <= 0x1p64f)) {
+          const float m_new = fmaxf(m, fmaxf(max32(va), max32(vb)) * kz);
+          ssum = m_new == -INFINITY ? 0.f : ssum * ex2_approx(m - m_new);
+          m = m_new;
+          bs = m == -INFINITY ? 0.f : chunk_exp_sum(va, kz, m) + chunk_exp_sum(vb, kz, m);
+        }
+        ssum += bs;
       }
     }
     // combine the four warpgroups' partial sums of each row; the exchange
