@@ -55,14 +55,45 @@ SCORE_CASES = {
     "exact_tiles": lambda: small(n_q_heads=8, n_kv_heads=1, R=32, M=32, n_beacons_in=32,
                                  L=4096, K=1024, capacity=4096),
     "big_norms": lambda: small(big_key_frac=0.05, big_key_norm=40.0, L=2000, K=500),
+    "rising_logits": lambda: small(L=1000, K=200),
 }
+
+
+def _rising_logits(inp):
+    """Keys whose first channel climbs from 0 to 400 along the cache, with a
+    spike of 800 at 80% of it, and queries whose first channel runs from -1
+    to 4 over the rows: the logits of the leaning rows climb by ~200 log2
+    units (a spike ~400 up), so the row statistics move their reference in
+    mid-row, past the 2^64 and 2^128 marks; the rows at -1 see the logits
+    fall as far (their exps underflow)."""
+    gen = torch.Generator().manual_seed(123)
+    L = inp.wl.L
+    ramp = torch.linspace(0.0, 400.0, L)
+    ramp[int(0.8 * L)] = 800.0
+    k = 0.5 * torch.randn(inp.k[:, :, :L].shape, generator=gen)
+    k[..., 0] += ramp
+    inp.k[:, :, :L] = k.to(inp.k.dtype)
+    for t in (inp.recent, inp.beacons):
+        q = 0.5 * torch.randn(t.shape, generator=gen)
+        q[..., 0] = torch.linspace(-1.0, 4.0, t.shape[2])
+        t.copy_(q.to(t.dtype))
+
+
+INPUT_HOOKS = {"rising_logits": _rising_logits}
+
+
+def score_inputs(case, wl, seed):
+    inp = _synth().make_step_inputs(wl, seed=seed)
+    if case in INPUT_HOOKS:
+        INPUT_HOOKS[case](inp)
+    return inp
 
 
 @pytest.mark.parametrize("case", sorted(SCORE_CASES))
 def test_score_select_compact(case, dev):
     bkv, synth = _lib(), _synth()
     wl = SCORE_CASES[case]()
-    inp = synth.make_step_inputs(wl, seed=11)
+    inp = score_inputs(case, wl, seed=11)
     g = bkv.geometry_of(inp.k, wl.n_q_heads)
     k, v = inp.k.to(dev), inp.v.to(dev)
     rq, bq = inp.recent.to(dev), inp.beacons.to(dev)
@@ -102,7 +133,7 @@ def test_score_mean(case, dev):
     top-K on those scores; the mean of softmax rows sums to 1 over the keys."""
     bkv, synth = _lib(), _synth()
     wl = SCORE_CASES[case]()
-    inp = synth.make_step_inputs(wl, seed=12)
+    inp = score_inputs(case, wl, seed=12)
     g = bkv.geometry_of(inp.k, wl.n_q_heads)
     k = inp.k.to(dev)
     rq, bq = inp.recent.to(dev), inp.beacons.to(dev)
