@@ -9,8 +9,9 @@
 //
 //   pass 1 (row statistics)   D[o][j] = Q_blk . K_tile^T, M = 128 observation
 //     rows, N = 256 keys.  TMEM lane = observation row, so each epilogue
-//     thread owns one row and keeps an online (max, sum of exp2) over the
-//     columns it reads; no cross-thread reduction per element.
+//     thread owns one row and keeps a (reference, sum of exp2) pair over the
+//     columns it reads -- the reference moves up only when a block's sum
+//     shows a key far above it; no cross-thread reduction per element.
 //   pass 2 (column max)       D[j][o] = K_tile . Q_grp^T - c_o / scale, M = 128
 //     keys, N = up to 2 x 256 observation rows.  The subtraction is one more
 //     K=16 step of the same MMA: every key carries a block (1, 1, 1, 0, ...)
