@@ -102,7 +102,16 @@ def work_model(wl):
         "step_flop": contraction,
         "step_bytes": float(H) * (L * d * es + n_obs * d * es + 2 * 4 * L + 2 * 4 * K
                                   + 4 * K * d * es),
+        # the row normalisers need one exp per logit
+        "step_exps": float(H) * n_obs * L,
     }
+
+
+def mufu_bound_s(wm, peaks):
+    """The exps of the step on the MUFU units alone (16 ex2 per clock per SM,
+    148 SMs, the max SM clock): a third bound beside the tensor and HBM ones,
+    which the row statistics beat by taking part of the exps on the FMA pipe."""
+    return wm["step_exps"] / (16 * 148 * peaks["sm_max_mhz"] * 1e6)
 
 
 def peak_for(bound, peaks):
@@ -667,6 +676,7 @@ def main():
         "step_us": ms * 1e3,
         "pct_roofline": 100.0 * t_roof / (ms / 1e3),
         "t_roof_us": t_roof * 1e6,
+        "t_mufu_us": mufu_bound_s(wm, peaks) * 1e6,
         "roofline": roofline,
         "phases": phases,
         "cpu_baseline": cpu,
