@@ -41,6 +41,8 @@ def pin_closed_forms(lib):
         s = oracle.max_aggregate(x, c, _lib=lib)
         np.testing.assert_allclose(c, case["c"], rtol=0, atol=1e-12, err_msg=case["name"])
         np.testing.assert_allclose(s, case["s"], rtol=0, atol=1e-12, err_msg=case["name"])
+        sm = oracle.mean_aggregate(x, c, _lib=lib)
+        np.testing.assert_allclose(sm, case["s_mean"], rtol=0, atol=1e-12, err_msg=case["name"])
         for K, want in case["topk"].items():
             got = oracle.select_topk(np.array(case["s"]), int(K), _lib=lib)
             assert got.tolist() == want, (case["name"], K, got.tolist(), want)

@@ -22,6 +22,9 @@ MUTANTS = {
     "aggregate_min": ("if (p > best) best = p;", "if (p < best || o == 0) best = p;"),
     "aggregate_row_index": ("double p = exp(x[o * L + j] - c[o]);", "double p = exp(x[o * L + j] - c[0]);"),
     "mean_drop_divide": ("s[j] = sum / (double)n_obs;", "s[j] = sum;"),
+    "mean_divide_by_keys": ("s[j] = sum / (double)n_obs;", "s[j] = sum / (double)L;"),
+    "mean_row_index": ("for (int64_t o = 0; o < n_obs; ++o) sum += exp(x[o * L + j] - c[o]);",
+                       "for (int64_t o = 0; o < n_obs; ++o) sum += exp(x[o * L + j] - c[0]);"),
     "topk_tie_high": ("return (x->j < y->j) ? -1 : (x->j > y->j);", "return (x->j > y->j) ? -1 : (x->j < y->j);"),
     "topk_no_ascending_sort": ("qsort(idx, (size_t)keep, sizeof(int32_t), oracle_cmp_int_asc);", ""),
     "topk_ascending_scores": ("if (x->s > y->s) return -1;\n  if (x->s < y->s) return 1;", "if (x->s < y->s) return -1;\n  if (x->s > y->s) return 1;"),
