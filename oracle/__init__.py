@@ -15,6 +15,14 @@ steps are composed.
 
 Inputs arrive as numpy arrays of any float dtype; they are converted to
 float64, which is exact for bfloat16 and float32 values.
+
+Pins (tests/oracle_pins.py): the C functions by closed forms, library
+routines and brute force; the composition here (observation_set, score_head,
+newest_rows, ring_rows, update_beacons_head, compress_head) by the
+hand-derived whole step of tests/golden/closed_forms.json, brute-force greedy
+FPS over the [beacons; window] union, and a history written into a ring one
+row at a time.  tests/test_oracle_mutants.py plants plausible mistakes in
+both and checks that each fails a pin.
 """
 from __future__ import annotations
 
@@ -206,6 +214,26 @@ def observation_set(recent, beacons, n_beacons: int):
 
 def default_scale(d: int) -> float:
     return 1.0 / np.sqrt(float(d))
+
+
+def newest_rows(rows, n: int):
+    """The n newest rows of a query history listed oldest first ([..., T, d]).
+
+    The recent queries of Fig. 5(a)/(b) are the R newest decode queries; with
+    the window of Fig. 7 listed oldest first they are its last R rows.
+    """
+    rows = np.asarray(rows)
+    T = rows.shape[-2]
+    return rows[..., T - n:T, :]
+
+
+def ring_rows(ring, head: int, n: int):
+    """The n newest rows, oldest first, of a ring buffer [..., cap, d] whose
+    next write goes to slot ``head`` (so the newest row sits at head - 1)."""
+    ring = np.asarray(ring)
+    cap = ring.shape[-2]
+    idx = [(head - n + i) % cap for i in range(n)]
+    return ring[..., idx, :]
 
 
 def score_head(k, recent, beacons, n_beacons: int, scale: float | None = None,

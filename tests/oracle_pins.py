@@ -204,3 +204,72 @@ def pin_fps_replay(lib):
 ALL_PINS = [pin_closed_forms, pin_logits_matmul, pin_softmax, pin_score_head_composition,
             pin_topk_full_sort, pin_compact_bytes, pin_fps_bruteforce, pin_fps_special_sets,
             pin_fps_replay]
+
+
+# --------------------------------------------------------------------------
+# Pins of the composition (oracle/__init__.py): each takes the oracle module
+# itself (or a mutated copy of it, see test_oracle_mutants.py).
+# --------------------------------------------------------------------------
+def pin_step_golden(mod):
+    """The hand-derived whole step of tests/golden/closed_forms.json: Continual
+    FPS over [stored beacons; window] (Fig. 7), then scores from the recent
+    query and the updated beacons (Fig. 5(b)), max aggregation and top-K
+    (Fig. 5(c)), compaction (Fig. 5(a))."""
+    for case in _golden()["step_cases"]:
+        b = np.array(case["beacons"])
+        w = np.array(case["window"])
+        k = np.array(case["k"])
+        v = np.array(case["v"])
+        recent = mod.newest_rows(w, case["R"])
+        for K, want in case["topk"].items():
+            r = mod.compress_head(k, v, recent, b, case["n_beacons"], w, case["M"], int(K),
+                                  scale=case["scale"])
+            assert [p.tolist() for p in r["picks"]] == case["picks"], (case["name"], r["picks"])
+            np.testing.assert_array_equal(r["beacons"], np.array(case["new_beacons"]))
+            assert r["n_beacons"] == case["M"]
+            np.testing.assert_allclose(r["scores"], case["s"], rtol=0, atol=1e-12,
+                                       err_msg=case["name"])
+            assert r["idx"].tolist() == want, (case["name"], K, r["idx"].tolist())
+            np.testing.assert_array_equal(r["k"], k[want])
+            np.testing.assert_array_equal(r["v"], v[want])
+
+
+def pin_update_beacons_composition(mod):
+    """Continual FPS over the stored beacons (slots past n_beacons ignored),
+    then the window oldest first, against brute-force greedy on that union."""
+    rng = np.random.default_rng(9)
+    for trial in range(40):
+        d = int(rng.integers(2, 5))
+        M = int(rng.integers(1, 6))
+        nb = int(rng.integers(0, M + 1))
+        W = int(rng.integers(0 if nb else 1, 5))
+        beacons = rng.standard_normal((M, d))
+        beacons[nb:] = rng.standard_normal((M - nb, d)) * 50.0   # stale slots
+        window = rng.standard_normal((W, d))
+        if trial % 4 == 0 and W and nb:
+            window[W - 1] = beacons[0] * 2.0   # a query in a beacon's direction
+        newb, sel = mod.update_beacons_head(beacons, nb, window, M)
+        U = np.concatenate([beacons[:nb], window])
+        want = _fps_brute(U, M)
+        assert sel.tolist() == want, (trial, sel.tolist(), want)
+        np.testing.assert_array_equal(newb, U[want])
+
+
+def pin_ring_rows(mod):
+    """The newest n rows of a ring buffer, oldest first, against a history
+    written into the ring one row at a time."""
+    rng = np.random.default_rng(10)
+    for cap, T, n in [(8, 5, 3), (8, 8, 8), (8, 13, 5), (5, 27, 5), (6, 6, 0), (7, 100, 1)]:
+        hist = rng.standard_normal((T, 3))
+        ring = np.zeros((cap, 3))
+        head = 0
+        for t in range(T):
+            ring[head] = hist[t]
+            head = (head + 1) % cap
+        got = mod.ring_rows(ring, head, n)
+        want = np.stack([hist[t] for t in range(T - n, T)]) if n else np.zeros((0, 3))
+        np.testing.assert_array_equal(got, want)
+        np.testing.assert_array_equal(mod.newest_rows(hist, n), want)
+
+
+COMPOSITION_PINS = [pin_step_golden, pin_update_beacons_composition, pin_ring_rows]

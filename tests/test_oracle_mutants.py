@@ -2,16 +2,21 @@
 
 Each mutant is a one-line textual change to a temporary copy of
 oracle/bkv_oracle.c (a dropped term, a flipped sign or comparison, a wrong
-index, a lost sort), compiled on the CPU.  The real oracle is untouched.
+index, a lost sort), compiled on the CPU, or of the composition in
+oracle/__init__.py (the order of the FPS union, the stale beacon slots, the
+beacons used for scoring, which end of the history the recent queries come
+from), imported from a temporary directory.  The real oracle is untouched.
 """
+import importlib.util
 import os
 import shutil
 import subprocess
+import sys
 
 import pytest
 
 import oracle
-from oracle_pins import ALL_PINS
+from oracle_pins import ALL_PINS, COMPOSITION_PINS
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "bkv_oracle.c")
 
@@ -55,3 +60,50 @@ def test_mutant_fails_a_pin(name, tmp_path):
         except AssertionError:
             failed.append(pin.__name__)
     assert failed, f"mutant {name} passed every pin"
+
+
+PY_SRC = os.path.join(os.path.dirname(oracle.__file__), "__init__.py")
+
+PY_MUTANTS = {
+    # Fig. 7: the union lists the current beacons first, then the window
+    "union_window_first": ("U = np.concatenate([b, w], axis=0) if w.size else b",
+                           "U = np.concatenate([w, b], axis=0) if w.size else b"),
+    # only the first n_beacons slots hold beacons
+    "union_all_slots": ("b = np.asarray(beacons)[:n_beacons]", "b = np.asarray(beacons)"),
+    # scoring uses the beacons after the update, not the stored ones
+    "score_old_beacons": ("s, c = score_head(k_rows, recent, beacons_used, n_used, scale,",
+                          "s, c = score_head(k_rows, recent, beacons, n_beacons, scale,"),
+    # the recent queries are the newest rows of the history
+    "recent_oldest_rows": ("return rows[..., T - n:T, :]", "return rows[..., 0:n, :]"),
+    # the observation set holds every query head's recent rows
+    "obs_drops_recent": ("        parts.append(recent[g])\n", ""),
+    # a ring's newest row sits just before the write position
+    "ring_off_by_one": ("idx = [(head - n + i) % cap for i in range(n)]",
+                        "idx = [(head - n + i + 1) % cap for i in range(n)]"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(PY_MUTANTS))
+def test_composition_mutant_fails_a_pin(name, tmp_path):
+    before, after = PY_MUTANTS[name]
+    text = open(PY_SRC).read()
+    assert text.count(before) == 1, f"mutation site for {name} not unique/present"
+    pkg = tmp_path / f"oracle_mut_{name}"
+    pkg.mkdir()
+    (pkg / "__init__.py").write_text(text.replace(before, after))
+    shutil.copy(SRC, pkg / "bkv_oracle.c")
+    spec = importlib.util.spec_from_file_location(pkg.name, pkg / "__init__.py",
+                                                  submodule_search_locations=[str(pkg)])
+    mod = importlib.util.module_from_spec(spec)
+    sys.modules[pkg.name] = mod
+    try:
+        spec.loader.exec_module(mod)
+        failed = []
+        for pin in COMPOSITION_PINS:
+            try:
+                pin(mod)
+            except AssertionError:
+                failed.append(pin.__name__)
+    finally:
+        sys.modules.pop(pkg.name, None)
+    assert failed, f"composition mutant {name} passed every pin"
