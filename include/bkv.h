@@ -131,7 +131,10 @@ bkv_status bkv_select_topk(const float *scores, int32_t n_rows, int64_t L,
  *   k_dst[r][i][:] = k_src[r][idx[r][i]][:],  v_dst likewise (byte copies).
  *   src/dst   geometry of the source and destination caches: same layers,
  *             heads, head_dim and dtype; dst->capacity >= n_keep
- *   idx       device, int32 [Ly*Hkv][n_keep], each in [0, src->capacity)
+ *   idx       device, int32 [Ly*Hkv][n_keep], each in [0, src->capacity); a
+ *             position outside that range is not read: its destination row is
+ *             left as it was and BKV_ERR_DEVICE_ASSERT is reported by
+ *             bkv_read_device_status
  * The destination must not overlap the source.  Either pair (k_src, k_dst) or
  * (v_src, v_dst) may be NULL/NULL to copy only the other. */
 bkv_status bkv_compact(const bkv_cache_desc *src, const void *k_src,
@@ -230,7 +233,9 @@ bkv_status bkv_compress_step(const bkv_step_args *args, int32_t *n_beacons_out,
  * holds until the process exits.
  *   - The first call on each device looks up the array's device address with
  *     that device current (cudaGetSymbolAddress); make that first call before
- *     any stream capture.
+ *     any stream capture.  The address is looked up again when the device's
+ *     context has changed since (after a cudaDeviceReset, for one), so make
+ *     the first call after a reset before any capture as well.
  *   - A problem whose scratch does not fit the array (at most
  *     bkv_workspace_size(desc, L, R, n_beacons, 0, 1) bytes are needed) is
  *     rejected with BKV_ERR_WORKSPACE before anything is launched.

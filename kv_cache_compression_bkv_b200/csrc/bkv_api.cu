@@ -5,6 +5,7 @@
 // rejected call leaves the outputs untouched.  Nothing here allocates device
 // memory: scratch space comes from the caller's workspace.
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <cmath>
@@ -44,6 +45,15 @@ ScoreWorkspace carve_score_workspace(const ScoreGeom &g, void *ws) {
 namespace {
 
 constexpr long long kMaxRows = (1LL << 31) - 1;
+
+// A host-side NVTX range (visible to a profiler that records NVTX, a no-op
+// otherwise) around the enqueueing of one phase of the step.
+struct PhaseRange {
+  explicit PhaseRange(const char *name) { nvtxRangePushA(name); }
+  ~PhaseRange() { nvtxRangePop(); }
+  PhaseRange(const PhaseRange &) = delete;
+  PhaseRange &operator=(const PhaseRange &) = delete;
+};
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -384,14 +394,17 @@ bkv_status bkv_compress_step(const bkv_step_args *a, int32_t *n_beacons_out, int
     if (!a->phase_events || !a->phase_events[i]) return true;
     return cudaEventRecord(static_cast<cudaEvent_t>(a->phase_events[i]), s) == cudaSuccess;
   };
+  PhaseRange step_range("bkv_compress_step");
   if (!mark(0)) return BKV_ERR_CUDA;
   if (update) {
+    PhaseRange r("bkv continual FPS");
     st = launch_fps(f, a->beacons_in, a->window, a->beacons_out, fps_ws, fps_b, s);
     if (st != BKV_OK) return st;
   }
   if (!mark(1)) return BKV_ERR_CUDA;
   const void *bq = nb_used > 0 ? score_beacons : nullptr;
   if (need_scores) {
+    PhaseRange r("bkv scoring");
     if (d->dtype == BKV_BF16) {
       st = launch_score_rowstats_tc(g, a->k, a->recent_q, bq, w.c, s);
       if (st != BKV_OK) return st;
@@ -415,20 +428,24 @@ bkv_status bkv_compress_step(const bkv_step_args *a, int32_t *n_beacons_out, int
   if (!mark(3)) return BKV_ERR_CUDA;
   const SelectInput in = score_select_input(g, d->dtype, w, mean);
   const bool copy_all = keep >= a->L;
-  if (!copy_all) {
-    st = launch_select_topk(in, g.n_heads(), a->L, keep, idx, a->scores_out, sel_ws, sel_b, s);
-    if (st != BKV_OK) return st;
-  } else {
-    if (a->scores_out) {
-      st = launch_finalize_scores(in, g.n_heads(), a->L, a->scores_out, s);
+  {
+    PhaseRange r("bkv top-K");
+    if (!copy_all) {
+      st = launch_select_topk(in, g.n_heads(), a->L, keep, idx, a->scores_out, sel_ws, sel_b, s);
       if (st != BKV_OK) return st;
-    }
-    if (a->idx_out) {
-      st = launch_iota_rows(a->idx_out, g.n_heads(), keep, s);
-      if (st != BKV_OK) return st;
+    } else {
+      if (a->scores_out) {
+        st = launch_finalize_scores(in, g.n_heads(), a->L, a->scores_out, s);
+        if (st != BKV_OK) return st;
+      }
+      if (a->idx_out) {
+        st = launch_iota_rows(a->idx_out, g.n_heads(), keep, s);
+        if (st != BKV_OK) return st;
+      }
     }
   }
   if (!mark(4)) return BKV_ERR_CUDA;
+  PhaseRange compact_range("bkv compaction");
   CompactArgs c;
   c.k_src = static_cast<const uint8_t *>(a->k);
   c.v_src = static_cast<const uint8_t *>(a->v);

@@ -1,7 +1,9 @@
 // compact.cu -- eviction of the unselected KV pairs (BeaconKV abstract and
 // Fig. 5(a)): the kept K and V rows are gathered into a dense new cache.
 //
-// A pure byte copy, bound by HBM bandwidth.  Each thread moves 16-byte
+// A pure byte copy, bound by HBM bandwidth.  A kept position outside the
+// source cache is never followed: its row is skipped and reported as a failed
+// device-side check.  Each thread moves 16-byte
 // vectors; consecutive threads cover consecutive 16-byte chunks of a row, so
 // every row is read and written by full, aligned 32-byte sectors.  Each thread
 // keeps several rows' loads in flight before storing (kUnroll) so that enough
@@ -64,6 +66,12 @@ __global__ void __launch_bounds__(kThreads) compact_kernel(const CompactArgs a) 
         const long long h = row / a.n_keep;
         const long long i = row - h * a.n_keep;
         const long long src_row = a.idx ? static_cast<long long>(a.idx[row]) : i;
+        if (src_row < 0 || src_row >= a.src_cap) {
+          // a position outside the source cache: report it and leave the
+          // destination row as it is rather than read out of bounds
+          if (c == 0) record_device_status(BKV_DEV_ASSERT, 502);
+          continue;
+        }
         const long long src_off = (h * a.src_cap + src_row) * a.row_bytes + c * 16;
         dst_off[u] = (h * a.dst_cap + i) * a.row_bytes + c * 16;
         if (kHasK) kv[u] = ld_stream(reinterpret_cast<const uint4 *>(a.k_src + src_off));

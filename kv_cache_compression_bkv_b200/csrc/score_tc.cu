@@ -38,6 +38,7 @@
 
 #include "bkv_internal.h"
 #include "sm100.cuh"
+#include "tma_host.h"
 
 BKV_DEFINE_STATUS_ACCESSOR(take_status_score_tc)
 
@@ -89,11 +90,13 @@ __device__ __forceinline__ float fma_sat(float a, float b, float c) {
 // 2^(v * kz - m) on the FMA pipe, for a pair.  One saturating FMA per element
 // maps x = v * kz - m from [-126, 128] onto y = (x + 126) / 254 in [0, 1], so
 // that x below the range gives about 2^-126, x above it (and m = -inf) about
-// 2^127, and NaN 2^-126; then Cody-Waite reduction of x' = 254 y - 126 =
-// j + f, j = rint(x') by adding 1.5 * 2^23, f in [-0.5, 0.5]; a cubic p(f) ~
-// 2^f (coefficients from fit_exp2_poly.py, max relative error 7.6e-5); and
-// 2^j added into p's exponent field, which stays in [0, 254].  `a` = kz / 254
-// and `b` = (126 - m) / 254 are the mapping's coefficients.
+// 2^128 (p(0) * 2^128, finite and just under FLT_MAX: two such terms overflow
+// a sum to inf), and NaN 2^-126; then Cody-Waite reduction of x' = 254 y -
+// 126 = j + f, j = rint(x') by adding 1.5 * 2^23, f in [-0.5, 0.5]; a cubic
+// p(f) ~ 2^f (coefficients from a Lawson-weighted least-squares fit, max
+// relative error 7.6e-5; tests/fit_exp2_poly.py); and 2^j added into p's
+// exponent field, which stays in [0, 254].  `a` = kz / 254 and `b` =
+// (126 - m) / 254 are the mapping's coefficients.
 __device__ __forceinline__ float2 exp2_poly2(float vx, float vy, float a, float b) {
   constexpr float kBase = 12582912.0f - 126.f;  // 1.5 * 2^23 - 126, exact
   const float2 y = make_float2(fma_sat(vx, a, b), fma_sat(vy, a, b));
@@ -729,24 +732,10 @@ __global__ void __launch_bounds__(p2_threads(kMean), 1)
 }
 
 // ------------------------------------------------------------------ host
-PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void *p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
 // Tensor map of the whole key cache as a 2-D bf16 array
 // [n_layers * n_kv_heads * cap rows][128], boxes of 64 x box_rows, 128 B swizzle.
 bool make_key_map(CUtensorMap *map, const void *k, const ScoreGeom &g, int box_rows) {
-  auto encode = get_encode_fn();
+  auto encode = tensor_map_encoder();
   if (!encode) return false;
   const cuuint64_t rows = static_cast<cuuint64_t>(g.n_heads()) * static_cast<cuuint64_t>(g.cap);
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(kDim), rows};

@@ -1,4 +1,6 @@
-"""Fit the cubic used by score_tc.cu to evaluate 2^f on the FMA pipe.
+"""Fit the cubic that kv_cache_compression_bkv_b200/csrc/score_tc.cu uses to
+evaluate 2^f on the FMA pipe (test infrastructure: test_exp2_route.py checks
+the kernel's constants against this fit and emulates its route).
 
 Method: Cody-Waite range reduction x = j + f with j = rint(x) and f in
 [-0.5, 0.5], then a polynomial p(f) ~ 2^f.  The coefficients below come from a

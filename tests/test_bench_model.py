@@ -19,8 +19,11 @@ def test_work_model_14b():
     assert wm["step_bytes"] == pytest.approx(4.876e9, rel=1e-3)
     assert wm["step_exps"] == pytest.approx(n_obs * L * H)
     assert wm["compact"]["work"] == pytest.approx(4 * K * d * 2 * H)
-    # FPS: M picks against M' + W union points of d channels, per query head
-    assert wm["fps"]["work"] == pytest.approx(1600 * 128 * (128 + 4096) * 128)
+    # FPS: M picks against M' + W union points of d channels, per query head,
+    # as FMAs and (tensor cores) as 2 FLOP each
+    assert wm["fps_fma"] == pytest.approx(1600 * 128 * (128 + 4096) * 128)
+    assert wm["fps"]["work"] == pytest.approx(2 * 1600 * 128 * (128 + 4096) * 128)
+    assert wm["fps"]["bound"] == "tensor" and wm["fps"]["unit"] == "FLOP"
 
 
 def test_mufu_bound_14b():

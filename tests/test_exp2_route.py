@@ -12,11 +12,12 @@ import numpy as np
 import pytest
 
 CSRC = pathlib.Path(__file__).resolve().parents[1] / "kv_cache_compression_bkv_b200" / "csrc"
+HERE = pathlib.Path(__file__).resolve().parent
 KZ = np.float32(0.08838835 * 1.4426950408889634)  # (1/sqrt(128)) * log2(e)
 
 
 def _fit_module():
-    spec = importlib.util.spec_from_file_location("fit_exp2_poly", CSRC / "fit_exp2_poly.py")
+    spec = importlib.util.spec_from_file_location("fit_exp2_poly", HERE / "fit_exp2_poly.py")
     mod = importlib.util.module_from_spec(spec)
     spec.loader.exec_module(mod)
     return mod
@@ -72,3 +73,19 @@ def test_above_the_range_shows_in_the_sum(fit):
     v = np.linspace(-1e6, 1e6, 1001).astype(np.float32)
     r = fit.exp2_route(v, KZ, -np.inf, c).astype(np.float64)
     assert np.all(r > 2.0 ** 64)
+
+
+def test_saturated_top_is_just_under_float_max(fit):
+    """At the top of the mapped range (x >= 128, or a reference of -inf) the
+    saturating map gives y = 1, f = 0 and an exponent of 2^128 inserted into
+    p(0): about 2^128, finite and just below FLT_MAX -- so two such terms in a
+    sum overflow to inf, which the row statistics treat like any sum above
+    2^64 (the block is summed again against a new reference)."""
+    c = _kernel_coeffs()
+    for m in (0.0, 40.0, -np.inf):
+        v = np.array([1e30, 3e4, (200.0 + (0 if np.isinf(m) else m)) / KZ], dtype=np.float32)
+        r = fit.exp2_route(v, KZ, m, c)
+        assert np.all(np.isfinite(r)), r
+        rr = r.astype(np.float64)
+        assert np.all(rr > 2.0 ** 127.99) and np.all(rr <= np.finfo(np.float32).max)
+        assert np.isinf(np.float32(r[0]) + np.float32(r[1]))
