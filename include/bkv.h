@@ -33,7 +33,10 @@
  *   - Errors: argument checks run on the host before anything is launched; a
  *     failing check returns BKV_ERR_INVALID_ARG / _UNSUPPORTED / _WORKSPACE and
  *     leaves every output untouched.  A failed launch returns BKV_ERR_CUDA.
- *     No exception, abort or exit crosses this interface.
+ *     No exception, abort or exit crosses this interface.  For tests of these
+ *     paths, a non-empty environment variable BKV_INJECT_LAUNCH_FAILURE (not
+ *     "0"), set before the library's first launch, makes every kernel launch
+ *     fail with BKV_ERR_CUDA before anything is enqueued.
  *   - Layouts are dense and row-major.  A cache tensor is
  *     [n_layers][n_kv_heads][capacity][head_dim]; query tensors are
  *     [n_layers][n_q_heads][rows][head_dim] in the cache's dtype.  Every base
@@ -206,6 +209,16 @@ typedef struct {
    * records its event at once. */
   void **phase_events;
   int32_t aggregate;           /* bkv_aggregate; 0 (a zeroed struct) = max */
+  /* Optional decode-side query ring (Fig. 7's "newest window" as the decode
+   * loop keeps it): NULL, or device [Ly][Hq][ring_cap][d] in which the decode
+   * step writes its t-th query (t = 0, 1, ...) of every query head to slot
+   * t mod ring_cap.  With a ring, recent_q and window must be NULL: the R
+   * recent queries are the ring's newest R rows and the window its newest W
+   * rows (oldest first), read in place where the ring wraps.
+   * Requires W <= ring_cap, R <= ring_cap, ring_pos >= max(W, R). */
+  const void *query_ring;
+  int64_t ring_cap;            /* slots per query head */
+  int64_t ring_pos;            /* queries written so far (the next slot is ring_pos mod ring_cap) */
 } bkv_step_args;
 
 #define BKV_STEP_EVENTS 6
@@ -256,6 +269,20 @@ bkv_status bkv_score_noalloc(const bkv_cache_desc *desc, const void *k,
  * returns the first code recorded since the previous call (BKV_OK if none),
  * clears it, and stores an internal location tag in *where_out (optional). */
 bkv_status bkv_read_device_status(void *stream, int32_t *where_out);
+
+/* Diagnostic of the bounded device-side waits; the paper has no counterpart.
+ * Launches one warp on `stream` that waits -- through the same bounded wait
+ * routine the kernels use -- on an mbarrier that nothing ever arrives on,
+ * with a wall-clock limit of limit_ns instead of the kernels' 0.5 s.  The
+ * wait gives up, records BKV_ERR_TIMEOUT with location tag 901 for
+ * bkv_read_device_status, and the kernel exits normally: no TMA load or MMA
+ * is in flight, so nothing is left behind and later calls run as usual.
+ *   limit_ns  1000 .. 100000000 (1 us .. 100 ms)
+ *   outcome   device, int32, 4-byte aligned: 0 when the wait gave up, 1 if
+ *             it was satisfied (it cannot be)
+ * Errors: BKV_ERR_INVALID_ARG for a limit out of range or a null or
+ * misaligned outcome (nothing launched); BKV_ERR_CUDA if the launch fails. */
+bkv_status bkv_selftest_wait_timeout(int64_t limit_ns, int32_t *outcome, void *stream);
 
 /* Static text for a status code. */
 const char *bkv_status_string(bkv_status status);

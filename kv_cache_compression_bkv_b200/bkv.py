@@ -25,7 +25,8 @@ STATUS = {0: "BKV_OK", 1: "BKV_ERR_INVALID_ARG", 2: "BKV_ERR_UNSUPPORTED",
           6: "BKV_ERR_DEVICE_ASSERT"}
 EXPORTS = ("bkv_workspace_size", "bkv_score", "bkv_select_topk", "bkv_compact",
            "bkv_update_beacons", "bkv_compress_step", "bkv_read_device_status",
-           "bkv_status_string", "bkv_score_noalloc", "bkv_score_mean", "bkv_compact_inplace")
+           "bkv_status_string", "bkv_score_noalloc", "bkv_score_mean", "bkv_compact_inplace",
+           "bkv_selftest_wait_timeout")
 SCORE_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -53,7 +54,9 @@ class StepArgs(ctypes.Structure):
                 ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
                 ("stream", ctypes.c_void_p),
                 ("phase_events", ctypes.POINTER(ctypes.c_void_p)),
-                ("aggregate", ctypes.c_int32)]
+                ("aggregate", ctypes.c_int32),
+                ("query_ring", ctypes.c_void_p), ("ring_cap", ctypes.c_int64),
+                ("ring_pos", ctypes.c_int64)]
 
 STEP_EVENTS = 6
 
@@ -80,6 +83,7 @@ def _load() -> ctypes.CDLL:
         "bkv_status_string": ([ctypes.c_int], ctypes.c_char_p),
         "bkv_score_noalloc": ([D, P, I64, P, I32, P, I32, I32, F, P, P], ctypes.c_int),
         "bkv_score_mean": ([D, P, I64, P, I32, P, I32, I32, F, P, P, SZ, P], ctypes.c_int),
+        "bkv_selftest_wait_timeout": ([I64, P, P], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -212,11 +216,14 @@ def bkv_compress_step(geom: Geometry, k, v, L: int, K: int, recent_q, R: int, be
                       n_beacons_in: int, M: int, window, W: int, beacons_out, scale: float,
                       dst: Geometry, k_dst, v_dst, scores_out=None, idx_out=None,
                       workspace=None, stream=None, phase_events=None,
-                      aggregate: str = "max") -> tuple[int, int]:
+                      aggregate: str = "max", query_ring=None, ring_pos: int = 0) -> tuple[int, int]:
     """One whole compression step; returns (beacons valid after, new cache length).
 
     phase_events: optional list of STEP_EVENTS torch.cuda.Event (timing enabled)
     recorded at the step's phase boundaries.  aggregate: "max" or "mean".
+    query_ring: optional decode-side ring [layers, q_heads, cap, d] holding query
+    t in slot t % cap, with ring_pos queries written; recent_q and window must
+    then be None (the recent rows and the window are the ring's newest R and W).
     """
     a = StepArgs()
     a.cache = geom.desc()
@@ -234,6 +241,10 @@ def bkv_compress_step(geom: Geometry, k, v, L: int, K: int, recent_q, R: int, be
     a.workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     a.stream = _stream(stream)
     a.aggregate = AGGREGATE[aggregate]
+    if query_ring is not None:
+        a.query_ring = _ptr(query_ring)
+        a.ring_cap = query_ring.shape[2]
+        a.ring_pos = ring_pos
     if phase_events is not None:
         if len(phase_events) != STEP_EVENTS:
             raise ValueError(f"phase_events needs {STEP_EVENTS} events")
@@ -244,6 +255,12 @@ def bkv_compress_step(geom: Geometry, k, v, L: int, K: int, recent_q, R: int, be
     _check(LIB.bkv_compress_step(ctypes.byref(a), ctypes.byref(nb), ctypes.byref(nl)),
            "bkv_compress_step")
     return nb.value, nl.value
+
+
+def bkv_selftest_wait_timeout(limit_ns: int, outcome, stream=None) -> None:
+    """Make one bounded device-side wait give up on purpose (diagnostic)."""
+    _check(LIB.bkv_selftest_wait_timeout(limit_ns, _ptr(outcome), _stream(stream)),
+           "bkv_selftest_wait_timeout")
 
 
 def bkv_read_device_status(stream=None) -> tuple[int, int]:

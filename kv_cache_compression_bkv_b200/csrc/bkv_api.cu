@@ -9,11 +9,20 @@
 
 #include <algorithm>
 #include <cmath>
+#include <cstdlib>
 
 #include "bkv_device_status.cuh"
 #include "bkv_internal.h"
 
 namespace bkv {
+
+bool injected_launch_failure() {
+  static const bool on = [] {
+    const char *v = std::getenv("BKV_INJECT_LAUNCH_FAILURE");
+    return v != nullptr && v[0] != '\0' && !(v[0] == '0' && v[1] == '\0');
+  }();
+  return on;
+}
 
 void finish_score_geom(ScoreGeom *g) {
   g->group = g->n_q_heads / g->n_kv_heads;
@@ -96,9 +105,14 @@ size_t query_bytes(const bkv_cache_desc *d, long long rows) {
          d->head_dim * elem_size(d->dtype);
 }
 
+// recent_cap / recent_start: where recent row i of a query head lives (row
+// (recent_start + i) mod recent_cap of its block); a dense [R][d] block is
+// cap R, start 0.
 ScoreGeom make_score_geom(const bkv_cache_desc *d, long long L, int R, int nb, int M,
-                          float scale) {
+                          float scale, long long recent_cap = -1, long long recent_start = 0) {
   ScoreGeom g{};
+  g.recent_cap = recent_cap < 0 ? R : recent_cap;
+  g.recent_start = recent_start;
   g.n_layers = d->n_layers;
   g.n_q_heads = d->n_q_heads;
   g.n_kv_heads = d->n_kv_heads;
@@ -209,7 +223,7 @@ size_t bkv_workspace_size(const bkv_cache_desc *desc, int64_t L, int32_t R, int3
   const long long keep = std::min<long long>(K, L);
   total += align_up(static_cast<size_t>(g.n_heads()) * keep * sizeof(int32_t), kAlign);
   FpsGeom f{desc->n_layers, desc->n_q_heads, desc->head_dim, desc->dtype, M, M, W,
-            std::min(M, M + W)};
+            std::min(M, M + W), W, 0};
   total += align_up(fps_workspace_bytes(f), kAlign);
   return total;
 }
@@ -316,7 +330,7 @@ bkv_status bkv_update_beacons(const bkv_cache_desc *desc, const void *beacons_in
     return BKV_ERR_INVALID_ARG;
   if (desc->head_dim > 128) return BKV_ERR_UNSUPPORTED;
   FpsGeom f{desc->n_layers, desc->n_q_heads, desc->head_dim, desc->dtype, n_beacons_in, M, W,
-            std::min(M, n_beacons_in + W)};
+            std::min(M, n_beacons_in + W), W, 0};
   if (!fps_supported(f)) return BKV_ERR_UNSUPPORTED;
   if (workspace_bytes < fps_workspace_bytes(f)) return BKV_ERR_WORKSPACE;
   st = launch_fps(f, beacons_in, window, beacons_out, workspace, workspace_bytes,
@@ -328,11 +342,28 @@ bkv_status bkv_update_beacons(const bkv_cache_desc *desc, const void *beacons_in
 bkv_status bkv_compress_step(const bkv_step_args *a, int32_t *n_beacons_out, int64_t *new_len) {
   if (!a) return BKV_ERR_INVALID_ARG;
   const bkv_cache_desc *d = &a->cache;
-  const bool update = a->window != nullptr && a->W > 0;
+  // the recent queries and the window: dense blocks, or the newest rows of a
+  // decode-side query ring (slot of query t: t mod ring_cap)
+  const bool ring = a->query_ring != nullptr;
+  if (ring) {
+    if (a->recent_q || a->window || a->ring_cap < 1 || a->R < 0 || a->W < 0 ||
+        a->R > a->ring_cap || a->W > a->ring_cap || a->ring_pos < std::max<int64_t>(a->R, a->W) ||
+        !aligned16(a->query_ring) ||
+        static_cast<long long>(d->n_layers) * d->n_q_heads * a->ring_cap > kMaxRows)
+      return BKV_ERR_INVALID_ARG;
+  }
+  const void *recent_src = ring ? a->query_ring : a->recent_q;
+  const void *window_src = ring ? a->query_ring : a->window;
+  const long long recent_cap = ring ? a->ring_cap : a->R;
+  const long long recent_start = ring ? (a->ring_pos - a->R) % a->ring_cap : 0;
+  const long long w_cap = ring ? a->ring_cap : a->W;
+  const long long w_start = ring ? (a->ring_pos - a->W) % a->ring_cap : 0;
+  const size_t wbytes = query_bytes(d, w_cap);
+  const bool update = window_src != nullptr && a->W > 0;
   const int nb_used = update ? std::min(a->M, a->n_beacons_in + a->W) : a->n_beacons_in;
   // scoring arguments (the beacons it reads are the updated ones when W > 0)
   const void *score_beacons = update ? a->beacons_out : a->beacons_in;
-  bkv_status st = check_score_args(d, a->k, a->L, a->recent_q, a->R,
+  bkv_status st = check_score_args(d, a->k, a->L, a->R > 0 ? recent_src : nullptr, a->R,
                                    nb_used > 0 ? score_beacons : nullptr, nb_used, a->M);
   if (st != BKV_OK) return st;
   if (a->K < 1 || !a->v || !std::isfinite(a->scale) || a->scale < 0.f) return BKV_ERR_INVALID_ARG;
@@ -342,11 +373,11 @@ bkv_status bkv_compress_step(const bkv_step_args *a, int32_t *n_beacons_out, int
     if (a->n_beacons_in < 0 || a->n_beacons_in > a->M || !a->beacons_out ||
         (a->n_beacons_in > 0 && !a->beacons_in))
       return BKV_ERR_INVALID_ARG;
-    if (!aligned16(a->window) || !aligned16(a->beacons_out)) return BKV_ERR_INVALID_ARG;
-    const size_t bbytes = query_bytes(d, a->M), wbytes = query_bytes(d, a->W);
+    if (!aligned16(window_src) || !aligned16(a->beacons_out)) return BKV_ERR_INVALID_ARG;
+    const size_t bbytes = query_bytes(d, a->M);
     if (overlaps(a->beacons_out, bbytes, a->beacons_in, bbytes) ||
-        overlaps(a->beacons_out, bbytes, a->window, wbytes) ||
-        overlaps(a->beacons_out, bbytes, a->recent_q, query_bytes(d, a->R)))
+        overlaps(a->beacons_out, bbytes, window_src, wbytes) ||
+        overlaps(a->beacons_out, bbytes, recent_src, query_bytes(d, recent_cap)))
       return BKV_ERR_INVALID_ARG;
   }
   st = check_desc(&a->dst_cache);
@@ -369,9 +400,10 @@ bkv_status bkv_compress_step(const bkv_step_args *a, int32_t *n_beacons_out, int
     return BKV_ERR_INVALID_ARG;
 
   FpsGeom f{d->n_layers, d->n_q_heads, d->head_dim, d->dtype, a->n_beacons_in, a->M, a->W,
-            nb_used};
+            nb_used, w_cap, w_start};
   if (update && !fps_supported(f)) return BKV_ERR_UNSUPPORTED;
-  const ScoreGeom g = make_score_geom(d, a->L, a->R, nb_used, a->M, a->scale);
+  const ScoreGeom g = make_score_geom(d, a->L, a->R, nb_used, a->M, a->scale, recent_cap,
+                                      recent_start);
   const bool need_scores = keep < a->L || a->scores_out != nullptr;
   // workspace: [score][select][idx][fps]
   const size_t score_b = need_scores ? score_workspace_bytes(g) : 0;
@@ -398,7 +430,7 @@ bkv_status bkv_compress_step(const bkv_step_args *a, int32_t *n_beacons_out, int
   if (!mark(0)) return BKV_ERR_CUDA;
   if (update) {
     PhaseRange r("bkv continual FPS");
-    st = launch_fps(f, a->beacons_in, a->window, a->beacons_out, fps_ws, fps_b, s);
+    st = launch_fps(f, a->beacons_in, window_src, a->beacons_out, fps_ws, fps_b, s);
     if (st != BKV_OK) return st;
   }
   if (!mark(1)) return BKV_ERR_CUDA;
@@ -406,19 +438,19 @@ bkv_status bkv_compress_step(const bkv_step_args *a, int32_t *n_beacons_out, int
   if (need_scores) {
     PhaseRange r("bkv scoring");
     if (d->dtype == BKV_BF16) {
-      st = launch_score_rowstats_tc(g, a->k, a->recent_q, bq, w.c, s);
+      st = launch_score_rowstats_tc(g, a->k, recent_src, bq, w.c, s);
       if (st != BKV_OK) return st;
       if (!mark(2)) return BKV_ERR_CUDA;
-      st = launch_score_colmax_tc(mean ? mean_grouping(g) : g, a->k, a->recent_q, bq, w.c, w.ypart,
+      st = launch_score_colmax_tc(mean ? mean_grouping(g) : g, a->k, recent_src, bq, w.c, w.ypart,
                                   mean, s);
     } else {
       st = launch_score_rowstats_simt(g, static_cast<const float *>(a->k),
-                                      static_cast<const float *>(a->recent_q),
+                                      static_cast<const float *>(recent_src),
                                       static_cast<const float *>(bq), w.c, s);
       if (st != BKV_OK) return st;
       if (!mark(2)) return BKV_ERR_CUDA;
       st = launch_score_colmax_simt(g, static_cast<const float *>(a->k),
-                                    static_cast<const float *>(a->recent_q),
+                                    static_cast<const float *>(recent_src),
                                     static_cast<const float *>(bq), w.c, w.ypart, mean, s);
     }
     if (st != BKV_OK) return st;
@@ -478,6 +510,7 @@ bkv_status bkv_read_device_status(void *stream, int32_t *where_out) {
   if (code == 0) code = take_status_fps_tc(s, &where);
   if (code == 0) code = take_status_compact(s, &where);
   if (code == 0) code = take_status_fps(s, &where);
+  if (code == 0) code = take_status_selftest(s, &where);
   if (code < 0) return BKV_ERR_CUDA;
   if (where_out) *where_out = code ? where : 0;
   if (code == 0) return BKV_OK;

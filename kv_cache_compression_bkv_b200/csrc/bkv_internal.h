@@ -23,6 +23,10 @@ struct ScoreGeom {
   long long cap;        // rows allocated per (layer, KV head)
   long long L;          // rows scored
   int R, nb, M;         // recent rows, valid beacons, beacon slots
+  // recent row i of a query head is row (recent_start + i) mod recent_cap of
+  // that head's [recent_cap][d] block: a dense [R][d] block (cap R, start 0)
+  // or the newest R rows of a decode-side query ring
+  long long recent_cap, recent_start;
   int n_obs;            // observation rows per KV head
   int n_obs_pad;        // n_obs rounded up to the row-statistics block (128)
   int n_groups;         // observation groups of the aggregation pass
@@ -111,6 +115,10 @@ struct FpsGeom {
   int n_layers, n_q_heads, head_dim, dtype;
   int nb_in, M, W;
   int n_pick;  // min(M, nb_in + W)
+  // window row w of a query head is row (w_start + w) mod w_cap of that
+  // head's [w_cap][d] block: a dense [W][d] block (cap W, start 0) or the
+  // newest W rows of a decode-side query ring
+  long long w_cap, w_start;
 };
 size_t fps_workspace_bytes(const FpsGeom &g);
 bool fps_supported(const FpsGeom &g);
@@ -123,6 +131,14 @@ bkv_status launch_fps_tc(const FpsGeom &g, const void *beacons_in, const void *w
                          void *beacons_out, void *ws, size_t ws_bytes, cudaStream_t stream);
 bkv_status launch_fps(const FpsGeom &g, const void *beacons_in, const void *window,
                       void *beacons_out, void *ws, size_t ws_bytes, cudaStream_t stream);
+
+// Fault injection for the host-side error paths: when the environment
+// variable BKV_INJECT_LAUNCH_FAILURE is set to a non-empty value other than
+// "0" when the library first checks it, every kernel launcher returns
+// BKV_ERR_CUDA instead of launching, as if the launch had failed, so that
+// tests can check that the entry points report it and leave their outputs
+// untouched.  Read once per process.
+bool injected_launch_failure();
 
 // Raise a kernel's dynamic shared-memory limit once per device (the attribute
 // is per device context).  Returns false if the CUDA call fails.
@@ -144,5 +160,6 @@ int take_status_select(cudaStream_t, int *);
 int take_status_fps_tc(cudaStream_t, int *);
 int take_status_compact(cudaStream_t, int *);
 int take_status_fps(cudaStream_t, int *);
+int take_status_selftest(cudaStream_t, int *);
 
 }  // namespace bkv

@@ -128,6 +128,7 @@ __global__ void __launch_bounds__(kInplaceThreads) compact_inplace_kernel(const 
 }  // namespace
 
 bkv_status launch_compact_inplace(const CompactArgs &a, cudaStream_t stream) {
+  if (injected_launch_failure()) return BKV_ERR_CUDA;
   if (a.n_keep == 0 || a.n_heads == 0) return BKV_OK;
   if (a.row_bytes < 16 || a.row_bytes > 16 * kInplacePer * kInplaceThreads) return BKV_ERR_UNSUPPORTED;
   dim3 grid(static_cast<unsigned>(a.n_heads), a.v_dst != nullptr ? 2u : 1u);
@@ -137,6 +138,7 @@ bkv_status launch_compact_inplace(const CompactArgs &a, cudaStream_t stream) {
 }
 
 bkv_status launch_compact(const CompactArgs &a, cudaStream_t stream) {
+  if (injected_launch_failure()) return BKV_ERR_CUDA;
   const long long total = static_cast<long long>(a.n_heads) * a.n_keep * (a.row_bytes >> 4);
   if (total == 0) return BKV_OK;
   const long long want = (total + kThreads * kUnroll - 1) / (kThreads * kUnroll);

@@ -61,12 +61,16 @@ struct Smem {
   int *scal;         // [8]
 };
 
+// Union point i: beacon i, or window row i - nb, which is row
+// (w_start + i - nb) mod w_cap of the head's window block (dense or a ring).
 template <typename T>
 struct Points {
   const T *B, *Wp;
   int nb, d;
+  long long w_cap, w_start;
   __device__ const T *operator()(int i) const {
-    return i < nb ? B + static_cast<size_t>(i) * d : Wp + static_cast<size_t>(i - nb) * d;
+    return i < nb ? B + static_cast<size_t>(i) * d
+                  : Wp + static_cast<size_t>((w_start + (i - nb)) % w_cap) * d;
   }
 };
 
@@ -140,7 +144,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const size_t qh = blockIdx.x;  // layer * n_q_heads + query head
   Points<T> pt{beacons_in + qh * static_cast<size_t>(g.M) * d,
-               window + qh * static_cast<size_t>(g.W) * d, g.nb_in, d};
+               window + qh * static_cast<size_t>(g.w_cap) * d, g.nb_in, d,
+               g.w_cap > 0 ? g.w_cap : 1, g.w_start};
   T *out = beacons_out + qh * static_cast<size_t>(g.M) * d;
 
   // inverse norms (0 for a zero vector, which makes its distance 1)
@@ -327,6 +332,7 @@ bool fps_supported(const FpsGeom &g) { return fps_tc_supported(g) || fps_simt_su
 // f32 inputs and other head sizes take the CUDA-core kernel above.
 bkv_status launch_fps(const FpsGeom &g, const void *beacons_in, const void *window,
                       void *beacons_out, void *ws, size_t ws_bytes, cudaStream_t stream) {
+  if (injected_launch_failure()) return BKV_ERR_CUDA;
   if (g.n_pick <= 0) return BKV_OK;
   if (fps_tc_supported(g))
     return launch_fps_tc(g, beacons_in, window, beacons_out, ws, ws_bytes, stream);

@@ -1,30 +1,45 @@
 // fps_tc.cu -- Continual farthest-point sampling (BeaconKV, Fig. 7) of bf16
-// queries with head_dim 128, the distance pass of every round on tcgen05.
+// queries with head_dim 128, with the dot products on tcgen05.
 //
-// Same exact speculative rounds as fps.cu (select the T+1 best unselected
-// points; Gram block of the T candidates; replay the greedy choice among
-// them while the best one provably beats every other point; lower all
-// distances by the round's picks), with T = 64 and the contractions on the
-// tensor cores:
-//   * the distance pass streams the union [beacons; window] of a query head
-//     by TMA in tiles of 128 points (128-byte swizzle, no multicast) through a
-//     4-stage ring and forms D[128 points][N] = tile . picks^T (M = 128, N =
-//     picks rounded up to 16, K = 128) in one of two TMEM accumulators.  Two
-//     threads issue the MMAs, warp 1 for the even tiles of the sequence
-//     (stages 0 and 2, accumulator 0) and warp 2 for the odd ones, so their
-//     instruction latencies overlap and every stage and accumulator keeps a
-//     single consumer.  Two epilogue warpgroups (TMEM lane = point) turn the
-//     dot products into cosine distances and lower the distance array;
-//   * the candidates' rows are staged in the MMA's swizzled layout and one
-//     M = 128 x N = 64 MMA forms their Gram block, the same f32 sums of exact
-//     bf16 products as the distance pass.
-// While a round selects, the first tiles of its coming pass are already
-// loaded into the ring.  After the seed pass (whose epilogue also reads the
-// staged tiles for the norms) a stage is released by the MMA's commit.
+// The picks are exactly the greedy sequence (seed U[0]; each further pick is
+// the unselected point farthest in cosine distance from the picked set, ties
+// to the lowest index), found in speculative rounds.  Every point i keeps an
+// upper bound u_i of its distance to the picked set and a stamp t_i: u_i is
+// the exact distance to the first t_i picks (distances only fall as picks are
+// added, so u_i bounds the true distance).  A round
+//   1. selects the T = 128 points with the largest u (histogram of u over
+//      [0, max u] in 256 bins, then the threshold bin ranked exactly), and
+//      the (T+1)-th, whose u bounds every other point's true distance;
+//   2. stages the candidates' rows in the MMA's swizzled layout and forms, in
+//      one tcgen05 commit, their Gram block (M = N = 128) and -- for
+//      candidates whose stamp is behind -- their dots with the picks they
+//      have not seen, so every candidate's distance becomes exact;
+//   3. replays the greedy choice among the candidates with the Gram block
+//      (one warp): the best remaining candidate is the true argmax while it
+//      beats the bound, so it is picked; the round stops at the first one
+//      that does not;
+//   4. writes the candidates' new distances back (exact, stamped) and, in an
+//      eager round, runs a distance pass that brings every point up to date.
+// Rounds are eager (with the pass) until one of them picks at least kSwitch
+// points: from then on only the candidates are refreshed (lazy rounds), which
+// avoids re-streaming the union; a lazy round that certifies no pick falls
+// back to an eager one.  On the clustered queries of the 14B-shaped workload
+// this takes ~5.5 passes over the union per head instead of ~9 (one per
+// round of the all-eager scheme).
+//
+// The distance pass streams the union [beacons; window] of a query head by
+// TMA in tiles of 128 points (128-byte swizzle, no multicast) through a
+// 4-stage ring and forms D[128 points][N] = tile . picks^T (M = 128, K = 128,
+// N = the picks the points have not seen, rounded up to 16) in one of two
+// TMEM accumulators.  Two threads issue the MMAs (warp 1 the even tiles of
+// the sequence, warp 2 the odd ones) so their instruction latencies overlap;
+// two epilogue warpgroups (TMEM lane = point) turn the dots into cosine
+// distances.  Between passes the ring's shared memory holds the round's
+// candidate rows, Gram block and selection scratch.
 //
 // The grid is persistent: one CTA per SM loops over the query heads.  The
-// distance and inverse-norm arrays live in shared memory, or for a union too
-// large for it in the caller's workspace (one slice per CTA).
+// distance, inverse-norm and stamp arrays live in shared memory, or for a
+// union too large for it in the caller's workspace (one slice per CTA).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -44,57 +59,111 @@ namespace {
 using namespace sm100;
 using namespace fpsk;
 
-constexpr int kThreads = 384;  // warp 0 TMA, warps 1-2 MMA, warps 4..11 distance epilogue
+constexpr int kThreads = 384;  // warp 0 TMA, warps 1-2 MMA, warps 4..11 epilogues
 constexpr int kWarps = kThreads / 32;
-constexpr int kCand = 64;      // candidates per round (T)
+constexpr int kCand = 128;     // candidates per round (T)
 constexpr int kDim = 128;
 constexpr int kTileRows = 128;
-constexpr int kStages = 4;  // even tiles use stages 0 and 2, odd tiles 1 and 3
+constexpr int kStages = 4;     // even tiles use stages 0 and 2, odd tiles 1 and 3
 constexpr int kTileBytes = kTileRows * kDim * 2;  // 32 KB
-constexpr int kBBlock = kCand * 128;              // one 64-element K block of the picks
-constexpr int kBBytes = 2 * kBBlock;              // 16 KB
-constexpr int kCRows = kCand;                     // candidate operand rows
-constexpr int kCBlock = kCRows * 128;             // one 64-element K block of the candidates
-constexpr int kCBytes = 2 * kCBlock;              // 16 KB
+constexpr int kMaxPick = 128;                     // beacons per head on this path
+constexpr int kPickRows = kMaxPick + 16;          // picks operand rows (N padding)
+constexpr int kPBlock = kPickRows * 128;          // one 64-element K block of the picks
+constexpr int kCBlock = kCand * 128;              // one 64-element K block of the candidates
+constexpr int kGramStride = kCand + 4;            // floats per Gram row (bank spread)
+constexpr int kListMax = 512;                     // threshold-bin keys ranked directly
+constexpr int kSwitch = 8;                        // picks that end the eager rounds
 constexpr int kSmallBytes = 4096;
-constexpr int kFixedBytes = kSmallBytes + 1024 + kStages * kTileBytes + kBBytes +
-                            kCBytes + kCand * kCand * 4 + kWarps * 256 * 4;
+constexpr int kFixedBytes = kSmallBytes + 1024 + kStages * kTileBytes + 2 * kPBlock;
 constexpr int kSmemLimit = 232448;
-// two accumulators of up to 64 columns, then the candidates' Gram block
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kGramCol = 128;
-constexpr int kAbort = 15;           // index of the abort flag in scal[]
+// TMEM: two pass accumulators of up to 128 columns, the Gram and refresh blocks
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kGramCol = 256, kRefCol = 384;
+// the serial phase's buffers inside the ring (idle between passes)
+constexpr int kGramOff = 0;                        // [kCand][kGramStride] f32
+constexpr int kSelOff = 69632;                     // whist [kWarps][256], list keys/indices
+constexpr int kCopOff = 3 * kTileBytes;            // candidates [2][kCand][128 B]
+static_assert(kGramOff + kCand * kGramStride * 4 <= kSelOff, "Gram block overlaps");
+static_assert(kSelOff + (kWarps * 256 + 2 * kListMax) * 4 <= kCopOff, "selection scratch overlaps");
+static_assert(kCopOff + 2 * kCBlock <= kStages * kTileBytes, "candidates overflow the ring");
+static_assert(kPBlock % 1024 == 0, "picks K blocks must keep 1024-byte atoms");
+
+// scal[] slots
+enum {
+  kSNp = 4,        // picks of the round
+  kSFallback = 5,  // the threshold bin is too large: radix select instead
+  kSKeyMin = 6,    // key range of the last pass (select_best reads 6 and 7)
+  kSKeyMax = 7,
+  kSAbove = 8,     // keys in bins above the threshold bin
+  kSNeed = 9,      // keys wanted from the threshold bin
+  kSBin = 10,      // the threshold bin
+  kSCand = 11,     // candidate counter
+  kSList = 12,     // threshold-bin list counter
+  kSRef = 13,      // lowest stamp among the candidates
+  kSDmax = 14,     // upper bound of every live distance (float bits)
+  kAbort = 15,
+  kSLive = 16,     // live keys counted by the histogram
+  kScalWords = 32
+};
 
 enum { kWhereProd = 401, kWhereMma = 402, kWhereEpi = 403, kWhereDrain = 404 };
 
 // Barriers: full[4] empty[4] tfull[2] tempty[2], the two MMA threads' drain
-// barriers, the Gram block's.
+// barriers, the round's Gram/refresh commit.
 constexpr int kBarFull = 0, kBarEmpty = 4, kBarTfull = 8, kBarTempty = 10, kBarDone = 12,
               kBarGram = 14;
 
 struct Layout {
-  uint64_t *bars;   // see kBarFull ..
+  uint64_t *bars;
   uint32_t *tmem_slot;
-  int *scal;        // [16]
+  int *scal;        // [kScalWords]
   uint32_t *hist;   // [256]
-  int *cidx;        // [kCand + 1]
+  int *cidx;        // [kCand + 1] candidates, then the bound
   float *cdist;     // [kCand + 1]
-  int *pick;        // [kCand]
-  float *pinv;      // [kCand]
-  uint8_t *stages;  // [kStages][kTileBytes]
-  uint8_t *bop;     // picks, K-major 128-byte swizzle: [2][kCand rows][128 B]
-  uint8_t *cop;     // candidates, K-major 128-byte swizzle: [2][kCRows rows][128 B]
-  float *gram;      // [kCand][kCand]
-  uint32_t *whist;  // [kWarps][256] per-warp histograms of the selection
-  float *dist;      // [n]
-  float *inv;       // [n]
+  int *pick;        // [kCand] candidate slots picked this round, in order
+  float *pinv;      // [kPickRows] inverse norm of pick k (NaN past the last pick)
+  uint8_t *ring;    // [kStages][kTileBytes]
+  uint8_t *pop;     // picks, K-major 128-byte swizzle: [2][kPickRows][128 B]
+  float *gram;      // (ring) [kCand][kGramStride]
+  uint32_t *whist;  // (ring) [kWarps][256]
+  uint32_t *lkey;   // (ring) [kListMax]
+  int *lidx;        // (ring) [kListMax]
+  uint8_t *cop;     // (ring) candidates, K-major 128-byte swizzle: [2][kCand][128 B]
+  float *dist;      // [n] upper bound of the distance to the picked set; -1 = picked
+  float *inv;       // [n] inverse norms
+  uint8_t *stamp;   // [n] picks accounted for in dist
 };
 
+// Union point i of a query head: beacon i, or window row i - nb, which is row
+// (w_start + i - nb) mod w_cap of the head's window block -- a dense [W][d]
+// block, or the newest W rows of a decode-side query ring.
 struct Head {
   const __nv_bfloat16 *B, *Wp;
-  int nb, W;
+  int nb;
+  long long w_cap, w_start;
   __device__ const __nv_bfloat16 *point(int i) const {
-    return i < nb ? B + static_cast<size_t>(i) * kDim : Wp + static_cast<size_t>(i - nb) * kDim;
+    return i < nb ? B + static_cast<size_t>(i) * kDim
+                  : Wp + static_cast<size_t>((w_start + (i - nb)) % w_cap) * kDim;
+  }
+};
+
+// The window's tiles: the ring (or dense block) of a head is read in
+// row-aligned tiles of 128 slots; tile t of the pass's window part is ring
+// tile first + t.  A window that wraps around the end of the ring takes every
+// ring tile; otherwise the tiles from the one holding its first slot to the
+// one holding its last.  Each slot maps back to its window row.
+struct WindowTiles {
+  int first, count;
+  __device__ WindowTiles(const FpsGeom &g) {
+    if (g.W <= 0) {
+      first = count = 0;
+    } else if (g.w_start + g.W > g.w_cap) {
+      first = 0;
+      count = static_cast<int>((g.w_cap + kTileRows - 1) / kTileRows);
+    } else {
+      first = static_cast<int>(g.w_start / kTileRows);
+      count = static_cast<int>((g.w_start + g.W - 1) / kTileRows) - first + 1;
+    }
   }
 };
 
@@ -102,48 +171,65 @@ __device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-// Issue the TMA loads of tiles [j0, j1) of the pass that starts at `seq`
-// (producer thread only).  Returns false after a timeout.
+// Issue the TMA loads of tiles [0, n_tiles) of the pass that starts at
+// sequence number `seq` (producer thread only).  Returns false after a timeout.
 __device__ bool issue_tiles(const Layout &s, const CUtensorMap *bmap, const CUtensorMap *wmap,
-                            int qh, const FpsGeom &g, int n_btiles, uint32_t seq, int j0,
-                            int j1) {
+                            int qh, const FpsGeom &g, int n_btiles, int w_first, uint32_t seq,
+                            int n_tiles) {
   const uint32_t full0 = smem_u32(&s.bars[kBarFull]), empty0 = smem_u32(&s.bars[kBarEmpty]);
-  for (int j = j0; j < j1; ++j) {
+  for (int j = 0; j < n_tiles; ++j) {
     const uint32_t q = seq + j, st = q % kStages;
     if (!mbar_wait(empty0 + 8 * st, ((q / kStages) & 1) ^ 1, kWhereProd)) return false;
     mbar_arrive_expect_tx(full0 + 8 * st, kTileBytes);
-    const uint32_t dst = smem_u32(s.stages + st * kTileBytes);
+    const uint32_t dst = smem_u32(s.ring + st * kTileBytes);
     const CUtensorMap *map = j < n_btiles ? bmap : wmap;
-    const int y = j < n_btiles ? qh * g.M + j * kTileRows : qh * g.W + (j - n_btiles) * kTileRows;
+    const int y = j < n_btiles ? qh * g.M + j * kTileRows
+                               : static_cast<int>(qh * g.w_cap) + (w_first + j - n_btiles) * kTileRows;
     tma_load_2d(dst, map, full0 + 8 * st, 0, y);
     tma_load_2d(dst + kTileRows * 128, map, full0 + 8 * st, 64, y);
   }
   return true;
 }
 
-// One distance pass over every tile of the head: the producer (warp 0), the
-// two MMA threads (warps 1 and 2) and the epilogue warpgroups (warps 4..11)
-// run their own loops; `seq` is the number of tiles all passes so far have
-// moved through the ring, so every role derives the same stage, accumulator
-// and barrier phase for each tile.
+// Lower a point's distance by the picks s0 + j it has not seen: columns j of
+// one 32-column chunk of D = point . picks^T (j >= lo; pinv NaN past the last
+// pick, which fminf ignores).  x = 1 - dot * inv_i * inv_k, clamped later.
+template <int kCols>
+__device__ __forceinline__ float chunk_min(const float (&v)[32], const float *pinv, int c0,
+                                           int lo, float inv_i, float mn) {
+  const float2 ninv = make_float2(-inv_i, -inv_i);
+#pragma unroll
+  for (int k = 0; k < kCols; k += 2) {
+    const float2 x = __ffma2_rn(__fmul2_rn(make_float2(v[k], v[k + 1]), ninv),
+                                make_float2(pinv[c0 + k], pinv[c0 + k + 1]),
+                                make_float2(1.f, 1.f));
+    mn = fminf(mn, c0 + k >= lo ? x.x : INFINITY);
+    mn = fminf(mn, c0 + k + 1 >= lo ? x.y : INFINITY);
+  }
+  return mn;
+}
+
+// One distance pass over every tile of the head: each unselected point i
+// takes the picks [stamp_i, P) it has not seen (picks operand rows s0 .. P-1;
+// the seed pass: the seed, stamp 0) and its stamp becomes P.  The producer
+// (warp 0), the two MMA threads (warps 1 and 2) and the epilogue warpgroups
+// (warps 4..11) run their own loops; `seq` is the number of tiles all passes
+// so far have moved through the ring, so every role derives the same stage,
+// accumulator and barrier phase for each tile.
 __device__ void distance_pass(const Layout &s, const CUtensorMap *bmap, const CUtensorMap *wmap,
-                              uint32_t tmem, int qh, const FpsGeom &g, int n_btiles, int n_tiles,
-                              uint32_t seq, int np, bool first, int prefetched) {
+                              uint32_t tmem, int qh, const FpsGeom &g, int n_btiles, int w_first,
+                              int n_tiles, uint32_t seq, int s0, int P, bool first) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t full0 = smem_u32(&s.bars[kBarFull]), empty0 = smem_u32(&s.bars[kBarEmpty]);
   const uint32_t tfull0 = smem_u32(&s.bars[kBarTfull]), tempty0 = smem_u32(&s.bars[kBarTempty]);
+  const int N = (P - s0 + 15) & ~15;  // 16 .. 128
   if (warp == 0) {
-    if (lane == 0 &&
-        !issue_tiles(s, bmap, wmap, qh, g, n_btiles, seq, prefetched, n_tiles))
+    if (lane == 0 && !issue_tiles(s, bmap, wmap, qh, g, n_btiles, w_first, seq, n_tiles))
       s.scal[kAbort] = 1;
   } else if (warp == 1 || warp == 2) {
-    // two MMA threads, one per accumulator: warp 1 takes the even tiles of
-    // the sequence (stages 0, 2, accumulator 0), warp 2 the odd ones, so the
-    // issue latencies of their tcgen05 instructions and barrier waits overlap
     if (lane == 0) {
-      const int npad = (np + 15) & ~15;
-      const uint32_t idesc = idesc_bf16_f32(kTileRows, npad);
-      const uint32_t b_base = smem_u32(s.bop);
+      const uint32_t idesc = idesc_bf16_f32(kTileRows, N);
+      const uint32_t b_base = smem_u32(s.pop) + static_cast<uint32_t>(s0) * 128u;
       const uint32_t mine = static_cast<uint32_t>(warp - 1);
       for (int j = 0; j < n_tiles; ++j) {
         const uint32_t q = seq + j, st = q % kStages, a = q & 1;
@@ -154,14 +240,14 @@ __device__ void distance_pass(const Layout &s, const CUtensorMap *bmap, const CU
           break;
         }
         tc_fence_after();
-        const uint32_t a_base = smem_u32(s.stages + st * kTileBytes);
+        const uint32_t a_base = smem_u32(s.ring + st * kTileBytes);
 #pragma unroll
         for (int kb = 0; kb < 2; ++kb) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint64_t ad = smem_desc_k_sw128(a_base + kb * (kTileRows * 128) + kk * 32);
-            const uint64_t bd = smem_desc_k_sw128(b_base + kb * kBBlock + kk * 32);
-            umma_f16(tmem + a * 64, ad, bd, idesc, (kb | kk) != 0);
+            const uint64_t bd = smem_desc_k_sw128(b_base + kb * kPBlock + kk * 32);
+            umma_f16(tmem + a * 128, ad, bd, idesc, (kb | kk) != 0);
           }
         }
         // the stage is free once these MMAs complete (in the seed pass the
@@ -175,47 +261,36 @@ __device__ void distance_pass(const Layout &s, const CUtensorMap *bmap, const CU
     const int wg = (warp - 4) >> 2;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
-    const int npad = (np + 15) & ~15;
     bool ok = true;  // warp-uniform; after a timeout the warp keeps only the barriers
     for (int j = 0; j < n_tiles; ++j) {
       const uint32_t q = seq + j, a = q & 1;
       if (static_cast<int>(a) != wg) continue;
-      if (ok && !mbar_wait_warp(tfull0 + 8 * a, (q >> 1) & 1, kWhereEpi)) {
-        s.scal[kAbort] = 1;
-        ok = false;
-      }
-      float v0[32], v1[32];
-      if (ok) {
-        tc_fence_after();
-        const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + a * 64;
-        tmem_ld_32x32b_x32(taddr, v0);
-        if (npad > 32) tmem_ld_32x32b_x32(taddr + 32, v1);
-        tmem_ld_wait_regs(v0);
-        tmem_reg_fence(v1);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(tempty0 + 8 * a);
-      }
       int i;
       bool valid;
       if (j < n_btiles) {
         i = j * kTileRows + r;
         valid = i < g.nb_in;
       } else {
-        const int w = (j - n_btiles) * kTileRows + r;
-        i = g.nb_in + w;
-        valid = w < g.W;
+        // ring slot -> window row (slots past the ring's end, or outside the
+        // window, are not points of this head)
+        const long long slot = static_cast<long long>(w_first + j - n_btiles) * kTileRows + r;
+        long long w = slot - g.w_start;
+        if (w < 0) w += g.w_cap;
+        valid = slot < g.w_cap && w < g.W;
+        i = valid ? g.nb_in + static_cast<int>(w) : 0;
       }
       const uint32_t st = q % kStages;
+      if (ok && !mbar_wait_warp(tfull0 + 8 * a, (q >> 1) & 1, kWhereEpi)) {
+        s.scal[kAbort] = 1;
+        ok = false;
+      }
       if (first) {
         // the seed pass also takes every point's inverse norm from its row of
-        // the staged tile (0 for a zero vector, whose distance is then 1)
-        if (ok && !mbar_wait_warp(full0 + 8 * st, (q / kStages) & 1, kWhereEpi)) {
-          s.scal[kAbort] = 1;
-          ok = false;
-        }
+        // the staged tile (0 for a zero vector, whose distance is then 1).
+        // The tile's MMAs have completed (their commit was awaited above), so
+        // once the warpgroup has read its rows the stage can be released.
         if (ok) {
-          const uint8_t *row = s.stages + st * kTileBytes;
+          const uint8_t *row = s.ring + st * kTileBytes;
           float ss = 0.f;
 #pragma unroll
           for (int c16 = 0; c16 < 16; ++c16) {
@@ -229,80 +304,177 @@ __device__ void distance_pass(const Layout &s, const CUtensorMap *bmap, const CU
           if (valid) s.inv[i] = ss > 0.f ? 1.0f / sqrtf(ss) : 0.f;
         }
         named_barrier_sync(2 + wg, 128);
+        if (ok && warp == 4 + 4 * wg && lane == 0) mbar_arrive(empty0 + 8 * st);
       }
-      if (first && ok && warp == 4 + 4 * wg && lane == 0) mbar_arrive(empty0 + 8 * st);
       if (!ok) continue;
+      tc_fence_after();
       const float di = !valid ? -1.f : first ? 2.f : s.dist[i];
+      const int lo = (valid && !first) ? static_cast<int>(s.stamp[i]) - s0 : 0;
+      const float inv_i = valid ? s.inv[i] : 0.f;
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + a * 128;
+      // the TMEM loads are warp-wide: every lane takes part, the live ones use them
+      float mn = INFINITY;
+      for (int c0 = 0; c0 < N; c0 += 32) {
+        float v[32];
+        if (c0 + 32 <= N) {
+          tmem_ld_32x32b_x32(taddr + c0, v);
+          tmem_ld_wait_regs(v);
+          if (di >= 0.f) mn = chunk_min<32>(v, s.pinv + s0, c0, lo, inv_i, mn);
+        } else {
+          float h[16];
+          tmem_ld_32x32b_x16(taddr + c0, h);
+          tmem_ld_wait_regs(h);
+#pragma unroll
+          for (int k = 0; k < 16; ++k) v[k] = h[k];
+          if (di >= 0.f) mn = chunk_min<16>(v, s.pinv + s0, c0, lo, inv_i, mn);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty0 + 8 * a);
       // the range of the new keys, which the next selection starts from
       uint32_t kmn = 0xffffffffu, kmx = 0u;
       if (di >= 0.f) {  // a point not yet selected
-        // x_k = 1 - dot_k * inv_i * inv_k, as cos_dist computes it; padded
-        // picks carry a NaN inverse norm, which min ignores
-        const float inv_i = s.inv[i];
-        const float2 ninv = make_float2(-inv_i, -inv_i);
-        float mn = INFINITY;
-#pragma unroll
-        for (int k = 0; k < 32; k += 4) {
-          if (k < npad) {
-            const float4 pv = *reinterpret_cast<const float4 *>(s.pinv + k);
-            const float2 x0 = __ffma2_rn(__fmul2_rn(make_float2(v0[k], v0[k + 1]), ninv),
-                                         make_float2(pv.x, pv.y), make_float2(1.f, 1.f));
-            const float2 x1 = __ffma2_rn(__fmul2_rn(make_float2(v0[k + 2], v0[k + 3]), ninv),
-                                         make_float2(pv.z, pv.w), make_float2(1.f, 1.f));
-            mn = fminf(mn, fminf(fminf(x0.x, x0.y), fminf(x1.x, x1.y)));
-          }
-        }
-        if (npad > 32) {
-#pragma unroll
-          for (int k = 0; k < 32; k += 4) {
-            if (k + 32 < npad) {
-              const float4 pv = *reinterpret_cast<const float4 *>(s.pinv + 32 + k);
-              const float2 x0 = __ffma2_rn(__fmul2_rn(make_float2(v1[k], v1[k + 1]), ninv),
-                                           make_float2(pv.x, pv.y), make_float2(1.f, 1.f));
-              const float2 x1 = __ffma2_rn(__fmul2_rn(make_float2(v1[k + 2], v1[k + 3]), ninv),
-                                           make_float2(pv.z, pv.w), make_float2(1.f, 1.f));
-              mn = fminf(mn, fminf(fminf(x0.x, x0.y), fminf(x1.x, x1.y)));
-            }
-          }
-        }
         // min(di, clamp(x, 0, 2)) == max(min(di, x), 0) for di in [0, 2]
         const float nd = fmaxf(fminf(di, mn), 0.f);
         s.dist[i] = nd;
+        s.stamp[i] = static_cast<uint8_t>(P);
         kmn = kmx = dist_key(nd);
       }
       kmn = __reduce_min_sync(0xffffffffu, kmn);
       kmx = __reduce_max_sync(0xffffffffu, kmx);
       if (lane == 0) {
-        atomicMin(reinterpret_cast<unsigned int *>(&s.scal[6]), kmn);
-        atomicMax(reinterpret_cast<unsigned int *>(&s.scal[7]), kmx);
+        atomicMin(reinterpret_cast<unsigned int *>(&s.scal[kSKeyMin]), kmn);
+        atomicMax(reinterpret_cast<unsigned int *>(&s.scal[kSKeyMax]), kmx);
       }
     }
   }
 }
 
-// The picks of this round into the B operand (rows padded with zeros to a
-// multiple of 16) and the output beacons: the seed's row from global memory,
-// a round's picks from the staged candidate rows.
-__device__ void stage_picks(const Layout &s, const Head &h, __nv_bfloat16 *out, int picked,
-                            int np, bool seed) {
-  const int npad = (np + 15) & ~15;
-  for (int e = threadIdx.x; e < npad * 16; e += kThreads) {
-    const int k = e >> 4, c16 = e & 15, kb = c16 >> 3, c = c16 & 7;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (k < np) {
-      v = seed ? *reinterpret_cast<const uint4 *>(h.point(s.cidx[s.pick[k]]) + c16 * 8)
-               : *reinterpret_cast<const uint4 *>(s.cop + kb * kCBlock + sw128_offset(s.pick[k], c));
-      *reinterpret_cast<uint4 *>(out + static_cast<size_t>(picked + k) * kDim + c16 * 8) = v;
+// Append (i, d) to the candidate slots with one atomic per warp (lanes with
+// `take` set); slots past kCand are dropped.
+__device__ __forceinline__ void push_candidate(const Layout &s, bool take, int i, float d,
+                                               int base_slot) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t bal = __ballot_sync(0xffffffffu, take);
+  int wbase = 0;
+  if (lane == 0 && bal) wbase = atomicAdd(&s.scal[kSCand], __popc(bal));
+  wbase = __shfl_sync(0xffffffffu, wbase, 0);
+  if (take) {
+    const int slot = base_slot + wbase + __popc(bal & ((1u << lane) - 1u));
+    if (slot < kCand) {
+      s.cidx[slot] = i;
+      s.cdist[slot] = d;
     }
-    *reinterpret_cast<uint4 *>(s.bop + kb * kBBlock + sw128_offset(k, c)) = v;
   }
+}
+
+// Step 1 of a round: the `want` live points with the largest u in (u desc,
+// index asc) order: the first kCand in slots 0.. (any order), the (kCand+1)-th
+// -- the bound -- in slot kCand when `bounded`.  A 256-bin histogram of u
+// over [0, dmax] finds the bin holding the want-th key; keys above it are
+// taken, keys in it are ranked against each other.  Returns false (nothing
+// written) when that bin holds more than kListMax keys or the live keys are
+// fewer than counted (NaN distances): the caller then uses the radix select.
+__device__ bool select_hist(const Layout &s, int n, int want, bool bounded, float dmax) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const float scale = dmax > 0.f ? 256.f / dmax : 0.f;
+  for (int b = tid; b < 256; b += kThreads) s.hist[b] = 0u;
+  if (tid == 0) {
+    s.scal[kSCand] = 0;
+    s.scal[kSList] = 0;
+    s.scal[kSLive] = 0;
+  }
+  __syncthreads();
+  int live = 0;
+  for (int i = tid; i < n; i += kThreads) {
+    const float d = s.dist[i];
+    if (d >= 0.f) {
+      atomicAdd(&s.hist[min(255, static_cast<int>(d * scale))], 1u);
+      ++live;
+    }
+  }
+  live = __reduce_add_sync(0xffffffffu, live);
+  if (lane == 0) atomicAdd(&s.scal[kSLive], live);
+  __syncthreads();
+  if (warp == 0) {
+    // lane l holds bins 255-8l .. 248-8l (descending)
+    uint32_t cnt[8], local = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      cnt[j] = s.hist[255 - 8 * lane - j];
+      local += cnt[j];
+    }
+    uint32_t incl = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t o = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += o;
+    }
+    const uint32_t excl = incl - local;
+    if (static_cast<int>(excl) < want && want <= static_cast<int>(incl)) {
+      uint32_t acc = excl;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (static_cast<int>(acc + cnt[j]) >= want) {
+          s.scal[kSBin] = 255 - 8 * lane - j;
+          s.scal[kSAbove] = static_cast<int>(acc);
+          s.scal[kSNeed] = want - static_cast<int>(acc);
+          s.scal[kSFallback] = cnt[j] > static_cast<uint32_t>(kListMax) ? 1 : 0;
+          break;
+        }
+        acc += cnt[j];
+      }
+    }
+    if (lane == 31 && static_cast<int>(incl) < want) s.scal[kSFallback] = 1;
+  }
+  __syncthreads();
+  if (s.scal[kSFallback] || s.scal[kSLive] < want) return false;
+  const int bstar = s.scal[kSBin], above = s.scal[kSAbove], need = s.scal[kSNeed];
+  // keys above the threshold bin are candidates; the bin's keys are listed
+  for (int base = 0; base < n; base += kThreads) {
+    const int i = base + tid;
+    const float d = i < n ? s.dist[i] : -1.f;
+    const int b = d >= 0.f ? min(255, static_cast<int>(d * scale)) : -1;
+    push_candidate(s, b > bstar, i, d, 0);
+    const bool inbin = b == bstar;
+    const uint32_t bal = __ballot_sync(0xffffffffu, inbin);
+    int wbase = 0;
+    if (lane == 0 && bal) wbase = atomicAdd(&s.scal[kSList], __popc(bal));
+    wbase = __shfl_sync(0xffffffffu, wbase, 0);
+    if (inbin) {
+      const int pos = wbase + __popc(bal & ((1u << lane) - 1u));
+      s.lkey[pos] = dist_key(d);
+      s.lidx[pos] = i;
+    }
+  }
+  __syncthreads();
+  // rank the bin's keys (key desc, index asc): rank r < need is taken, the
+  // last taken one (rank need-1) is the bound when the selection is bounded
+  const int listed = s.scal[kSList];
+  for (int e = tid; e < listed; e += kThreads) {
+    const uint32_t ke = s.lkey[e];
+    const int ie = s.lidx[e];
+    int rank = 0;
+    for (int f = 0; f < listed; ++f) {
+      const uint32_t kf = s.lkey[f];
+      rank += (kf > ke || (kf == ke && s.lidx[f] < ie)) ? 1 : 0;
+    }
+    if (rank < need) {
+      const int slot = bounded && rank == need - 1 ? kCand : above + rank;
+      s.cidx[slot] = ie;
+      s.cdist[slot] = s.dist[ie];
+    }
+  }
+  __syncthreads();
+  return true;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
     fps_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__ CUtensorMap wmap,
                   const FpsGeom g, const __nv_bfloat16 *__restrict__ beacons_in,
                   const __nv_bfloat16 *__restrict__ window, __nv_bfloat16 *__restrict__ beacons_out,
-                  int n_qheads, float *__restrict__ gdist) {
+                  int n_qheads, uint8_t *__restrict__ garrays, size_t slice_bytes) {
   extern __shared__ uint8_t smem_raw[];
   const int n = g.nb_in + g.W;
   const int m = g.n_pick;
@@ -310,27 +482,32 @@ __global__ void __launch_bounds__(kThreads, 1)
   s.bars = reinterpret_cast<uint64_t *>(smem_raw);
   s.tmem_slot = reinterpret_cast<uint32_t *>(smem_raw + 128);
   s.scal = reinterpret_cast<int *>(smem_raw + 192);
-  s.hist = reinterpret_cast<uint32_t *>(smem_raw + 256);
-  s.cidx = reinterpret_cast<int *>(smem_raw + 1280);
-  s.cdist = reinterpret_cast<float *>(smem_raw + 1552);
-  s.pick = reinterpret_cast<int *>(smem_raw + 1824);
-  s.pinv = reinterpret_cast<float *>(smem_raw + 2096);
+  s.hist = reinterpret_cast<uint32_t *>(smem_raw + 320);
+  s.cidx = reinterpret_cast<int *>(smem_raw + 1344);
+  s.cdist = reinterpret_cast<float *>(smem_raw + 1872);
+  s.pick = reinterpret_cast<int *>(smem_raw + 2400);
+  s.pinv = reinterpret_cast<float *>(smem_raw + 2912);   // .. 3488
   const uint32_t raw_base = smem_u32(smem_raw);
   const uint32_t big = (raw_base + kSmallBytes + 1023u) & ~1023u;
-  s.stages = smem_raw + (big - raw_base);
-  s.bop = s.stages + kStages * kTileBytes;
-  s.cop = s.bop + kBBytes;
-  s.gram = reinterpret_cast<float *>(s.cop + kCBytes);
-  s.whist = reinterpret_cast<uint32_t *>(s.gram + kCand * kCand);
-  // the distance and inverse-norm arrays: in shared memory, or this CTA's
-  // slice of the workspace for a union too large for it
-  s.dist = gdist ? gdist + static_cast<size_t>(blockIdx.x) * 2 * n
-                 : reinterpret_cast<float *>(s.whist + kWarps * 256);
+  s.ring = smem_raw + (big - raw_base);
+  s.pop = s.ring + kStages * kTileBytes;
+  s.gram = reinterpret_cast<float *>(s.ring + kGramOff);
+  s.whist = reinterpret_cast<uint32_t *>(s.ring + kSelOff);
+  s.lkey = s.whist + kWarps * 256;
+  s.lidx = reinterpret_cast<int *>(s.lkey + kListMax);
+  s.cop = s.ring + kCopOff;
+  // the distance, inverse-norm and stamp arrays: in shared memory, or this
+  // CTA's slice of the workspace for a union too large for it
+  uint8_t *arrays = garrays ? garrays + static_cast<size_t>(blockIdx.x) * slice_bytes
+                            : s.pop + 2 * kPBlock;
+  s.dist = reinterpret_cast<float *>(arrays);
   s.inv = s.dist + n;
+  s.stamp = reinterpret_cast<uint8_t *>(s.inv + n);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n_btiles = (g.nb_in + kTileRows - 1) / kTileRows;
-  const int n_tiles = n_btiles + (g.W + kTileRows - 1) / kTileRows;
+  const WindowTiles wt(g);
+  const int n_tiles = n_btiles + wt.count;
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) {
       mbar_init(smem_u32(&s.bars[kBarFull + i]), 1);
@@ -341,7 +518,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&s.bars[kBarTempty + a]), 4);  // one arrive per warp of its warpgroup
       mbar_init(smem_u32(&s.bars[kBarDone + a]), 1);
     }
-    mbar_init(smem_u32(&s.bars[kBarGram]), 1);  // the Gram block's MMA
+    mbar_init(smem_u32(&s.bars[kBarGram]), 1);  // the round's Gram/refresh MMAs
     fence_barrier_init();
     prefetch_tensormap(&bmap);
     prefetch_tensormap(&wmap);
@@ -361,11 +538,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   for (int qh = blockIdx.x; qh < n_qheads; qh += gridDim.x) {
     Head h{beacons_in + static_cast<size_t>(qh) * g.M * kDim,
-           window + static_cast<size_t>(qh) * g.W * kDim, g.nb_in, g.W};
+           window + static_cast<size_t>(qh) * g.w_cap * kDim, g.nb_in,
+           g.w_cap > 0 ? g.w_cap : 1, g.w_start};
     __nv_bfloat16 *out = beacons_out + static_cast<size_t>(qh) * g.M * kDim;
+    // the seed U[0]: the first pick, row 0 of the picks operand and of the output
+    for (int c16 = tid; c16 < 16; c16 += kThreads) {
+      const uint4 v = *reinterpret_cast<const uint4 *>(h.point(0) + c16 * 8);
+      *reinterpret_cast<uint4 *>(s.pop + (c16 >> 3) * kPBlock + sw128_offset(0, c16 & 7)) = v;
+      *reinterpret_cast<uint4 *>(out + c16 * 8) = v;
+    }
     if (tid == 0) {
-      s.cidx[0] = 0;  // the seed U[0] is the first pick
-      s.pick[0] = 0;
       // its inverse norm, summed in the order the seed pass uses for every point
       float ss = 0.f;
       for (int t = 0; t < kDim; t += 8) {
@@ -374,88 +556,95 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = 0; e < 8; ++e) ss = fmaf(u[e], u[e], ss);
       }
       s.pinv[0] = ss > 0.f ? 1.0f / sqrtf(ss) : 0.f;
+      s.scal[kSKeyMin] = -1;
+      s.scal[kSKeyMax] = 0;
     }
-    if (tid > 0 && tid < 16) s.pinv[tid] = __int_as_float(0x7fc00000);
-    if (tid == 0) {  // the seed pass gathers the range of its keys (the seed's
-      s.scal[6] = -1;  // own 0 among them: a lower bound is all it needs)
-      s.scal[7] = 0;
-    }
-    __syncthreads();
-    stage_picks(s, h, out, 0, 1, true);
+    for (int k = 1 + tid; k < kPickRows; k += kThreads) s.pinv[k] = __int_as_float(0x7fc00000);
+    if (m <= 1) continue;  // nothing past the seed (every thread sees the same m)
     fence_proxy_async_smem();
     __syncthreads();
-    distance_pass(s, &bmap, &wmap, tmem, qh, g, n_btiles, n_tiles, seq, 1, true, 0);
+    distance_pass(s, &bmap, &wmap, tmem, qh, g, n_btiles, wt.first, n_tiles, seq, 0, 1, true);
     seq += n_tiles;
     __syncthreads();
     if (s.scal[kAbort]) break;
     if (tid == 0) s.dist[0] = -1.f;
     __syncthreads();
 
-    int picked = 1;
-    while (picked < m) {
-      const int unsel = n - picked;
+    int P = 1;          // picks so far
+    int E = 1;          // every unselected point's stamp is at least E
+    bool eager = true;  // the next round runs a distance pass
+    float dmax = __uint_as_float(static_cast<uint32_t>(s.scal[kSKeyMax]) & 0x7fffffffu);
+    while (P < m) {
+      const int unsel = n - P;
       const int nc = min(kCand, unsel);
       const bool bounded = unsel > kCand;
       const int want = bounded ? kCand + 1 : nc;
-      // the next distance pass streams the same tiles whatever this round
-      // picks: start its first loads now, behind the round's selection work
-      const int pre = min(kStages, n_tiles);
-      if (tid == 0 && !issue_tiles(s, &bmap, &wmap, qh, g, n_btiles, seq, 0, pre))
-        s.scal[kAbort] = 1;
-      select_best<kThreads>(s.dist, n, unsel, want, s.whist, s.hist, s.scal, s.cidx, s.cdist,
-                            true);  // the pass left the key range in scal[6..7]
-      __syncthreads();
-      // the candidates need no order; only the bound (the last of the kCand+1
-      // selected in (distance desc, index asc) order) moves to slot kCand
-      if (bounded && warp == 0) {
-        float wd = 3.f;
-        int wi = -1, ws = -1;
-        for (int j = lane; j < want; j += 32) {
-          const float dj = s.cdist[j];
-          const int ij = s.cidx[j];
-          if (ws < 0 || before(wd, wi, dj, ij)) {
-            wd = dj;
-            wi = ij;
-            ws = j;
+      // ---- 1. candidates
+      if (!select_hist(s, n, want, bounded, dmax)) {
+        // a threshold bin too crowded to rank (or distances that are not
+        // numbers): the radix select, then the bound moves to slot kCand
+        select_best<kThreads>(s.dist, n, unsel, want, s.whist, s.hist, s.scal, s.cidx, s.cdist,
+                              false);
+        __syncthreads();
+        if (bounded && warp == 0) {
+          float wd = 3.f;
+          int wi = -1, ws = -1;
+          for (int j = lane; j < want; j += 32) {
+            const float dj = s.cdist[j];
+            const int ij = s.cidx[j];
+            if (ws < 0 || before(wd, wi, dj, ij)) {
+              wd = dj;
+              wi = ij;
+              ws = j;
+            }
+          }
+          for (int off = 16; off > 0; off >>= 1) {
+            const float od = __shfl_xor_sync(0xffffffffu, wd, off);
+            const int oi = __shfl_xor_sync(0xffffffffu, wi, off);
+            const int os = __shfl_xor_sync(0xffffffffu, ws, off);
+            if (os >= 0 && (ws < 0 || before(wd, wi, od, oi))) {
+              wd = od;
+              wi = oi;
+              ws = os;
+            }
+          }
+          if (lane == 0 && ws != kCand) {
+            s.cidx[ws] = s.cidx[kCand];
+            s.cdist[ws] = s.cdist[kCand];
+            s.cidx[kCand] = wi;
+            s.cdist[kCand] = wd;
           }
         }
-        for (int off = 16; off > 0; off >>= 1) {
-          const float od = __shfl_xor_sync(0xffffffffu, wd, off);
-          const int oi = __shfl_xor_sync(0xffffffffu, wi, off);
-          const int os = __shfl_xor_sync(0xffffffffu, ws, off);
-          if (os >= 0 && (ws < 0 || before(wd, wi, od, oi))) {
-            wd = od;
-            wi = oi;
-            ws = os;
-          }
-        }
-        if (lane == 0 && ws != kCand) {
-          s.cidx[ws] = s.cidx[kCand];
-          s.cdist[ws] = s.cdist[kCand];
-          s.cidx[kCand] = wi;
-          s.cdist[kCand] = wd;
-        }
+        __syncthreads();
       }
+      // ---- 2. the candidates' rows into the swizzled operand, and the
+      // lowest stamp among them (candidates behind P are refreshed)
+      if (tid == 0) s.scal[kSRef] = P;
       __syncthreads();
-      // the candidates' rows into the swizzled operand (rows past nc keep
-      // whatever an earlier round left; their Gram entries are never read)
       for (int e = tid; e < nc * 16; e += kThreads) {
         const int a = e >> 4, c16 = e & 15, kb = c16 >> 3, c = c16 & 7;
+        const int i = s.cidx[a];
         *reinterpret_cast<uint4 *>(s.cop + kb * kCBlock + sw128_offset(a, c)) =
-            *reinterpret_cast<const uint4 *>(h.point(s.cidx[a]) + c16 * 8);
+            *reinterpret_cast<const uint4 *>(h.point(i) + c16 * 8);
+        if (c16 == 0) {
+          const int t = s.stamp[i];
+          if (t < P) atomicMin(&s.scal[kSRef], t);
+        }
       }
       fence_proxy_async_smem();
       tc_fence_before();
       __syncthreads();
-      // Gram block on the tensor cores: D[a][b] = cand_a . cand_b, N = kCand,
-      // K = 128, the same f32 accumulation of exact bf16 products as the
-      // distance pass.  M = 128: rows a >= kCand of A run on into the next
-      // 8 KB of shared memory (the other K block, then the Gram buffer), and
-      // those rows of D are never read.
+      const int t_lo = s.scal[kSRef];
+      const bool refresh = t_lo < P;
+      const int s_ref = t_lo & ~7;
+      const int n_ref = (P - s_ref + 15) & ~15;
+      // Gram block D[a][b] = cand_a . cand_b (M = N = 128), and the refresh
+      // block D[a][j] = cand_a . pick_(s_ref + j): the same f32 sums of exact
+      // bf16 products as the distance pass, with the candidate as operand A
       if (warp == 1 && lane == 0) {
         tc_fence_after();
-        const uint32_t idesc = idesc_bf16_f32(128, kCand);
         const uint32_t c_base = smem_u32(s.cop);
+        const uint32_t idesc = idesc_bf16_f32(128, kCand);
 #pragma unroll
         for (int kb = 0; kb < 2; ++kb) {
 #pragma unroll
@@ -464,23 +653,64 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma_f16(tmem + kGramCol, ad, ad, idesc, (kb | kk) != 0);
           }
         }
+        if (refresh) {
+          const uint32_t p_base = smem_u32(s.pop) + static_cast<uint32_t>(s_ref) * 128u;
+          const uint32_t ridesc = idesc_bf16_f32(128, n_ref);
+#pragma unroll
+          for (int kb = 0; kb < 2; ++kb) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t ad = smem_desc_k_sw128(c_base + kb * kCBlock + kk * 32);
+              const uint64_t bd = smem_desc_k_sw128(p_base + kb * kPBlock + kk * 32);
+              umma_f16(tmem + kRefCol, ad, bd, ridesc, (kb | kk) != 0);
+            }
+          }
+        }
         umma_commit(smem_u32(&s.bars[kBarGram]));
       }
-      if (warp == 4 || warp == 5) {
-        // TMEM lane = candidate a: warp 4 reads rows 0..31, warp 5 rows 32..63
+      if (warp >= 4 && (warp < 8 || refresh)) {
+        // TMEM lane = candidate a; warps 4-7 copy the Gram rows to shared
+        // memory, warps 8-11 refresh the candidates whose stamp is behind
+        const int quarter = warp & 3;
+        const int a = quarter * 32 + lane;
         if (mbar_wait_warp(smem_u32(&s.bars[kBarGram]), gram_phase & 1, kWhereEpi)) {
           tc_fence_after();
-          const uint32_t taddr = tmem + (static_cast<uint32_t>((warp - 4) * 32) << 16) + kGramCol;
-          float *row = s.gram + ((warp - 4) * 32 + lane) * kCand;
+          const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+          if (warp < 8) {
+            float *row = s.gram + a * kGramStride;
 #pragma unroll 1
-          for (int half = 0; half < 2; ++half) {
-            float x[32];
-            tmem_ld_32x32b_x32(taddr + half * 32, x);
-            tmem_ld_wait_regs(x);
+            for (int c0 = 0; c0 < kCand; c0 += 32) {
+              float x[32];
+              tmem_ld_32x32b_x32(lane_base + kGramCol + c0, x);
+              tmem_ld_wait_regs(x);
+              if (a < nc) {
 #pragma unroll
-            for (int b = 0; b < 32; b += 4)
-              *reinterpret_cast<float4 *>(row + half * 32 + b) =
-                  make_float4(x[b], x[b + 1], x[b + 2], x[b + 3]);
+                for (int b = 0; b < 32; b += 4)
+                  *reinterpret_cast<float4 *>(row + c0 + b) =
+                      make_float4(x[b], x[b + 1], x[b + 2], x[b + 3]);
+              }
+            }
+          } else {
+            const int i = a < nc ? s.cidx[a] : 0;
+            const int t = a < nc ? static_cast<int>(s.stamp[i]) : P;
+            const float inv_a = a < nc ? s.inv[i] : 0.f;
+            float mn = INFINITY;
+            for (int c0 = 0; c0 < n_ref; c0 += 32) {
+              float v[32];
+              if (c0 + 32 <= n_ref) {
+                tmem_ld_32x32b_x32(lane_base + kRefCol + c0, v);
+                tmem_ld_wait_regs(v);
+                if (t < P) mn = chunk_min<32>(v, s.pinv + s_ref, c0, t - s_ref, inv_a, mn);
+              } else {
+                float hv[16];
+                tmem_ld_32x32b_x16(lane_base + kRefCol + c0, hv);
+                tmem_ld_wait_regs(hv);
+#pragma unroll
+                for (int k = 0; k < 16; ++k) v[k] = hv[k];
+                if (t < P) mn = chunk_min<16>(v, s.pinv + s_ref, c0, t - s_ref, inv_a, mn);
+              }
+            }
+            if (t < P) s.cdist[a] = fmaxf(fminf(s.cdist[a], mn), 0.f);
           }
         } else {
           s.scal[kAbort] = 1;
@@ -489,76 +719,135 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       ++gram_phase;
       __syncthreads();
-      // replay the greedy choice among the candidates (warp 0, two per lane).
-      // The argmax in (distance desc, index asc) order takes two warp
-      // reductions: the largest distance key, then the lowest index holding it.
+      if (s.scal[kAbort]) break;
+      // ---- 3. replay the greedy choice among the candidates (warp 0, four
+      // per lane: slots lane, lane+32, lane+64, lane+96).  The argmax in
+      // (distance desc, index asc) order takes two warp reductions: the
+      // largest distance key, then the lowest index holding it.
       if (warp == 0) {
-        const int a0 = lane, a1 = lane + 32;
-        bool t0 = a0 >= nc, t1 = a1 >= nc;  // taken or absent
-        float c0 = t0 ? 0.f : s.cdist[a0], c1 = t1 ? 0.f : s.cdist[a1];
-        const int i0 = t0 ? 0x7fffffff : s.cidx[a0], i1 = t1 ? 0x7fffffff : s.cidx[a1];
-        const float inv0 = t0 ? 0.f : s.inv[i0], inv1 = t1 ? 0.f : s.inv[i1];
+        float c[4], iv[4];
+        int ix[4];
+        bool taken[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int a = lane + 32 * q;
+          taken[q] = a >= nc;
+          c[q] = taken[q] ? 0.f : s.cdist[a];
+          ix[q] = taken[q] ? 0x7fffffff : s.cidx[a];
+          iv[q] = taken[q] ? 0.f : s.inv[ix[q]];
+        }
         const float bd = bounded ? s.cdist[kCand] : -3.f;
         const int bi = bounded ? s.cidx[kCand] : 0x7fffffff;
         int np = 0;
-        while (picked + np < m) {
+        while (P + np < m) {
           // distances are >= 0, so their bits order like the values; +1 keeps
           // 0 free for "taken"
-          const uint32_t k0 = t0 ? 0u : __float_as_uint(c0) + 1u;
-          const uint32_t k1 = t1 ? 0u : __float_as_uint(c1) + 1u;
-          const uint32_t kbest = __reduce_max_sync(0xffffffffu, max(k0, k1));
+          uint32_t kq[4], kmax = 0u;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            kq[q] = taken[q] ? 0u : __float_as_uint(c[q]) + 1u;
+            kmax = max(kmax, kq[q]);
+          }
+          const uint32_t kbest = __reduce_max_sync(0xffffffffu, kmax);
           if (kbest == 0u) break;  // no candidate left
-          const uint32_t mine = min(k0 == kbest ? static_cast<uint32_t>(i0) : 0xffffffffu,
-                                    k1 == kbest ? static_cast<uint32_t>(i1) : 0xffffffffu);
+          uint32_t mine = 0xffffffffu;
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            if (kq[q] == kbest) mine = min(mine, static_cast<uint32_t>(ix[q]));
           const int best_i = static_cast<int>(__reduce_min_sync(0xffffffffu, mine));
           const float best_d = __uint_as_float(kbest - 1u);
           if (bounded && !before(best_d, best_i, bd, bi)) break;
-          const bool own0 = k0 == kbest && i0 == best_i, own1 = k1 == kbest && i1 == best_i;
-          const uint32_t owners = __ballot_sync(0xffffffffu, own0 || own1);
+          int own = -1;
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            if (kq[q] == kbest && ix[q] == best_i) own = q;
+          const uint32_t owners = __ballot_sync(0xffffffffu, own >= 0);
           const int src = __ffs(owners) - 1;
-          const int best_a = __shfl_sync(0xffffffffu, own0 ? a0 : a1, src);
+          const int best_a = __shfl_sync(0xffffffffu, lane + 32 * max(own, 0), src);
+          const float inv_b = __shfl_sync(0xffffffffu, own >= 0 ? iv[own] : 0.f, src);
           if (lane == 0) s.pick[np] = best_a;
           ++np;
-          if (own0) t0 = true;
-          if (own1) t1 = true;
-          const float inv_b = s.inv[best_i];
-          if (!t0) c0 = fminf(c0, cos_dist(make_float2(s.gram[best_a * kCand + a0], 0.f), inv0, inv_b));
-          if (!t1) c1 = fminf(c1, cos_dist(make_float2(s.gram[best_a * kCand + a1], 0.f), inv1, inv_b));
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            if (q == own) taken[q] = true;
+            if (!taken[q]) {
+              // D[a][best] has the candidate as operand A, like the pass
+              const float dot = s.gram[(lane + 32 * q) * kGramStride + best_a];
+              c[q] = fminf(c[q], cos_dist(make_float2(dot, 0.f), iv[q], inv_b));
+            }
+          }
         }
-        if (lane == 0) s.scal[4] = np;
+        // the candidates not picked keep exact distances to all P + np picks;
+        // every other point's u is at most the bound
+        float dm = bounded ? bd : 0.f;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          if (!taken[q]) {
+            s.dist[ix[q]] = c[q];
+            s.stamp[ix[q]] = static_cast<uint8_t>(P + np);
+            dm = fmaxf(dm, c[q]);
+          }
+        }
+        dm = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(dm)));
+        if (lane == 0) {
+          s.scal[kSNp] = np;
+          s.scal[kSDmax] = __float_as_int(dm);
+        }
       }
       __syncthreads();
-      const int np = s.scal[4];
-      if (np == 0) {
-        // only distances that are not numbers (NaN input rows) can stop the
-        // replay before its first pick; report and stop instead of looping
+      const int np = s.scal[kSNp];
+      if (np == 0 && eager) {
+        // an eager round's best candidate is the true argmax, so only
+        // distances that are not numbers (NaN input rows) can stop it: report
+        // and stop instead of looping
         if (tid == 0) record_device_status(BKV_DEV_ASSERT, 405);
         stuck = true;
-        seq += pre;  // the coming pass's first tiles are in flight: drain them
         break;
       }
-      if (tid < ((np + 15) & ~15))
-        s.pinv[tid] = tid < np ? s.inv[s.cidx[s.pick[tid]]] : __int_as_float(0x7fc00000);
-      stage_picks(s, h, out, picked, np, false);
-      __syncthreads();
-      if (tid < np) s.dist[s.cidx[s.pick[tid]]] = -1.f;
-      if (tid == 0) {  // the coming pass gathers the range of its new keys
-        s.scal[6] = -1;
-        s.scal[7] = 0;
+      // ---- 4. the picks: rows P .. P+np-1 of the picks operand and of the
+      // output (from the staged candidate rows), their inverse norms, and
+      // their distances set to -1
+      for (int e = tid; e < np * 16; e += kThreads) {
+        const int k = e >> 4, c16 = e & 15, kb = c16 >> 3, c = c16 & 7;
+        const int a = s.pick[k];
+        const uint4 v = *reinterpret_cast<const uint4 *>(s.cop + kb * kCBlock + sw128_offset(a, c));
+        *reinterpret_cast<uint4 *>(s.pop + kb * kPBlock + sw128_offset(P + k, c)) = v;
+        *reinterpret_cast<uint4 *>(out + static_cast<size_t>(P + k) * kDim + c16 * 8) = v;
+        if (c16 == 0) {
+          const int i = s.cidx[a];
+          s.pinv[P + k] = s.inv[i];
+          s.dist[i] = -1.f;
+        }
+      }
+      P += np;
+      dmax = __int_as_float(s.scal[kSDmax]);
+      if (P >= m) {
+        __syncthreads();
+        break;
+      }
+      if (eager && np >= kSwitch) eager = false;
+      else if (!eager && np == 0) eager = true;
+      if (tid == 0) {  // the pass gathers the range of its new keys
+        s.scal[kSKeyMin] = -1;
+        s.scal[kSKeyMax] = 0;
       }
       fence_proxy_async_smem();
       __syncthreads();
-      distance_pass(s, &bmap, &wmap, tmem, qh, g, n_btiles, n_tiles, seq, np, false, pre);
-      seq += n_tiles;
-      __syncthreads();
-      if (s.scal[kAbort]) break;
-      picked += np;
+      if (eager) {
+        distance_pass(s, &bmap, &wmap, tmem, qh, g, n_btiles, wt.first, n_tiles, seq, E & ~7, P,
+                      false);
+        seq += n_tiles;
+        __syncthreads();
+        if (s.scal[kAbort]) break;
+        E = P;
+        dmax = __uint_as_float(static_cast<uint32_t>(s.scal[kSKeyMax]) & 0x7fffffffu);
+      }
     }
     if (s.scal[kAbort] || stuck) break;
   }
 
   // drain: every TMA load and MMA issued by this CTA has completed before the
-  // CTA exits and frees its TMEM
+  // CTA exits and frees its TMEM (after a timeout, loads may be in flight)
   if (warp == 0 && lane == 0 && seq > 0) {
     const uint32_t first = seq > kStages ? seq - kStages : 0;
     for (uint32_t q = first; q < seq; ++q)
@@ -582,10 +871,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 namespace {
 
 // The persistent grid never exceeds this many CTAs (the workspace holds one
-// distance slice per CTA when the arrays live there).
+// slice of the per-point arrays per CTA when they live there).
 constexpr int kMaxCtas = 148;
 
-size_t union_array_bytes(const FpsGeom &g) { return 8 * (static_cast<size_t>(g.nb_in) + g.W); }
+// dist (f32), inv (f32) and stamp (u8) of one union, rounded to 16 bytes
+size_t union_array_bytes(const FpsGeom &g) {
+  const size_t n = static_cast<size_t>(g.nb_in) + g.W;
+  return (9 * n + 15) / 16 * 16;
+}
 
 bool arrays_in_smem(const FpsGeom &g) {
   return static_cast<size_t>(kFixedBytes) + union_array_bytes(g) <= static_cast<size_t>(kSmemLimit);
@@ -604,12 +897,15 @@ size_t fps_tc_workspace_bytes(const FpsGeom &g) {
 }
 
 bool fps_tc_supported(const FpsGeom &g) {
-  return g.dtype == BKV_BF16 && g.head_dim == kDim &&
-         static_cast<long long>(g.n_layers) * g.n_q_heads * std::max(g.M, g.W) < (1LL << 31) - 256;
+  return g.dtype == BKV_BF16 && g.head_dim == kDim && g.M <= kMaxPick &&
+         static_cast<long long>(g.n_layers) * g.n_q_heads *
+                 std::max<long long>(g.M, std::max<long long>(g.W, g.w_cap)) <
+             (1LL << 31) - 256;
 }
 
 bkv_status launch_fps_tc(const FpsGeom &g, const void *beacons_in, const void *window,
                          void *beacons_out, void *ws, size_t ws_bytes, cudaStream_t stream) {
+  if (injected_launch_failure()) return BKV_ERR_CUDA;
   const size_t ws_need = fps_tc_workspace_bytes(g);
   if (ws_need > 0 && (ws == nullptr || ws_bytes < ws_need ||
                       (reinterpret_cast<uintptr_t>(ws) & 15u) != 0))
@@ -623,7 +919,7 @@ bkv_status launch_fps_tc(const FpsGeom &g, const void *beacons_in, const void *w
   const unsigned long long brows =
       static_cast<unsigned long long>(n_qheads) * static_cast<unsigned long long>(g.nb_in > 0 ? g.M : g.W);
   const unsigned long long wrows =
-      static_cast<unsigned long long>(n_qheads) * static_cast<unsigned long long>(g.W > 0 ? g.W : g.M);
+      static_cast<unsigned long long>(n_qheads) * static_cast<unsigned long long>(g.W > 0 ? g.w_cap : g.M);
   CUtensorMap bmap, wmap;
   if (!make_bf16_rows_map(&bmap, bsrc, brows, kTileRows) ||
       !make_bf16_rows_map(&wmap, wsrc, wrows, kTileRows))
@@ -638,7 +934,7 @@ bkv_status launch_fps_tc(const FpsGeom &g, const void *beacons_in, const void *w
   fps_tc_kernel<<<grid, kThreads, smem, stream>>>(
       bmap, wmap, g, static_cast<const __nv_bfloat16 *>(beacons_in),
       static_cast<const __nv_bfloat16 *>(window), static_cast<__nv_bfloat16 *>(beacons_out),
-      n_qheads, ws_need > 0 ? static_cast<float *>(ws) : nullptr);
+      n_qheads, ws_need > 0 ? static_cast<uint8_t *>(ws) : nullptr, union_array_bytes(g));
   return cudaGetLastError() == cudaSuccess ? BKV_OK : BKV_ERR_CUDA;
 }
 

@@ -22,7 +22,8 @@ __device__ __forceinline__ const float *obs_row_f32(const ScoreGeom &g, const fl
   const int i = o - gq * per;
   const long long qh = static_cast<long long>(layer) * g.n_q_heads +
                        static_cast<long long>(kvh) * g.group + gq;
-  if (i < g.R) return recent + (qh * g.R + i) * g.head_dim;
+  if (i < g.R)  // row (recent_start + i) mod recent_cap of the head's block (a ring or dense)
+    return recent + (qh * g.recent_cap + (g.recent_start + i) % g.recent_cap) * g.head_dim;
   return beacons + (qh * g.M + (i - g.R)) * g.head_dim;
 }
 
@@ -119,6 +120,7 @@ __global__ void __launch_bounds__(kKeysPerBlock) colmax_simt_kernel(
 
 bkv_status launch_score_rowstats_simt(const ScoreGeom &g, const float *k, const float *recent,
                                       const float *beacons, float *c, cudaStream_t stream) {
+  if (injected_launch_failure()) return BKV_ERR_CUDA;
   dim3 grid((g.n_obs + kRowsPerBlock - 1) / kRowsPerBlock, g.n_heads());
   rowstats_simt_kernel<<<grid, 256, 0, stream>>>(g, k, recent, beacons, c);
   return cudaGetLastError() == cudaSuccess ? BKV_OK : BKV_ERR_CUDA;
@@ -127,6 +129,7 @@ bkv_status launch_score_rowstats_simt(const ScoreGeom &g, const float *k, const 
 bkv_status launch_score_colmax_simt(const ScoreGeom &g, const float *k, const float *recent,
                                     const float *beacons, const float *c, float *ypart,
                                     bool mean, cudaStream_t stream) {
+  if (injected_launch_failure()) return BKV_ERR_CUDA;
   dim3 grid(static_cast<unsigned>((g.L + kKeysPerBlock - 1) / kKeysPerBlock), g.n_heads());
   if (mean)
     colmax_simt_kernel<true><<<grid, kKeysPerBlock, 0, stream>>>(g, k, recent, beacons, c, ypart);

@@ -153,7 +153,9 @@ __device__ __forceinline__ uint4 ldg_nc_v4(const void *p) {
 }
 
 // Pointer to observation row o of KV head (layer, kvh): query head g of the
-// group, row i of [recent (R rows); beacons (nb rows)].
+// group, row i of [recent (R rows); beacons (nb rows)].  The recent rows are
+// read where they are: a dense [R][d] block per query head, or the newest R
+// rows of a decode-side query ring (ScoreGeom::recent_cap / recent_start).
 __device__ __forceinline__ const uint16_t *obs_row(const ScoreGeom &g, const uint16_t *recent,
                                                    const uint16_t *beacons, int layer, int kvh,
                                                    int o) {
@@ -162,7 +164,8 @@ __device__ __forceinline__ const uint16_t *obs_row(const ScoreGeom &g, const uin
   const int i = o - gq * per;
   const long long qh = static_cast<long long>(layer) * g.n_q_heads +
                        static_cast<long long>(kvh) * g.group + gq;
-  if (i < g.R) return recent + (qh * g.R + i) * kDim;
+  if (i < g.R)  // row (recent_start + i) mod recent_cap of the head's block (a ring or dense)
+    return recent + (qh * g.recent_cap + (g.recent_start + i) % g.recent_cap) * kDim;
   return beacons + (qh * g.M + (i - g.R)) * kDim;
 }
 
@@ -753,6 +756,7 @@ bool make_key_map(CUtensorMap *map, const void *k, const ScoreGeom &g, int box_r
 
 bkv_status launch_score_rowstats_tc(const ScoreGeom &g, const void *k, const void *recent,
                                     const void *beacons, float *c, cudaStream_t stream) {
+  if (injected_launch_failure()) return BKV_ERR_CUDA;
   CUtensorMap map;
   if (!make_key_map(&map, k, g, kP1Keys)) return BKV_ERR_CUDA;
   static int attr_done[64];
@@ -766,6 +770,7 @@ bkv_status launch_score_rowstats_tc(const ScoreGeom &g, const void *k, const voi
 bkv_status launch_score_colmax_tc(const ScoreGeom &g, const void *k, const void *recent,
                                   const void *beacons, const float *c, float *ypart, bool mean,
                                   cudaStream_t stream) {
+  if (injected_launch_failure()) return BKV_ERR_CUDA;
   CUtensorMap map;
   if (!make_key_map(&map, k, g, kP2Keys)) return BKV_ERR_CUDA;
   int max_rows_pad = 0;

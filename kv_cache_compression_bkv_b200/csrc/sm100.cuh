@@ -58,17 +58,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Wait until the phase with the given parity has completed.  Returns false
-// (and records a timeout) if that does not happen within kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int where) {
+// (and records a timeout at `where`) if that does not happen within
+// `limit_ns` of wall-clock time.
+__device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, int where,
+                                              unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
+    if ((it & 63u) == 0 && globaltimer_ns() - t0 > limit_ns) {
       record_device_status(BKV_DEV_TIMEOUT, where);
       return false;
     }
   }
+}
+
+// The kernels' wait: mbar_wait_for with the library's limit, kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int where) {
+  return mbar_wait_for(bar, parity, where, kWaitLimitNs);
 }
 
 // mbar_wait by every lane of a warp, with one outcome for the whole warp (so
@@ -76,6 +83,10 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int whe
 // lanes or by none).
 __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, int where) {
   return __all_sync(0xffffffffu, mbar_wait(bar, parity, where));
+}
+__device__ __forceinline__ bool mbar_wait_warp_for(uint32_t bar, uint32_t parity, int where,
+                                                   unsigned long long limit_ns) {
+  return __all_sync(0xffffffffu, mbar_wait_for(bar, parity, where, limit_ns));
 }
 
 // ---------------------------------------------------------------- fences

@@ -98,8 +98,9 @@ def test_select_rejects():
     assert f(A, 4, 100, 0, A, None, 0, S) == INVALID
     assert f(A, 4, 100, 10, None, None, 0, S) == INVALID
     assert f(A + 4, 4, 100, 10, A, None, 0, S) == INVALID
-    # a row too long for shared memory needs workspace
-    assert f(A, 4, 1 << 20, 10, A, None, 0, S) == WORKSPACE
+    # rows of any length need no workspace (the select streams them)
+    d = desc()
+    assert LIB.bkv_workspace_size(ctypes.byref(d), 1 << 20, 8, 16, 0, 10) > 0
 
 
 def test_compact_rejects():
@@ -237,3 +238,89 @@ def test_step_args_layout_matches_the_header(tmp_path):
                                           check=True).stdout.split()]
     assert got[0] == ctypes.sizeof(bkv.StepArgs)
     assert got[1:] == [getattr(bkv.StepArgs, f).offset for f in fields]
+
+
+INJECT_SCRIPT = r"""
+import ctypes, sys
+import numpy as np
+sys.path.insert(0, {root!r})
+from kv_cache_compression_bkv_b200 import bkv
+LIB = bkv.LIB
+CUDA = 4
+# host buffers stand in for device ones: with the injected failure no launch
+# (and no access) happens, on a machine with or without a GPU
+cap, keep, d = 64, 16, 128
+src = np.arange(2 * 2 * cap * d, dtype=np.uint16).reshape(2, 2, cap, d)
+dst = np.full((2, 2, keep, d), 7, dtype=np.uint16)
+idx = np.tile(np.arange(keep, dtype=np.int32) * 2, (4, 1))
+g = bkv.CacheDesc(2, 4, 2, d, cap, bkv.BKV_BF16)
+gd = bkv.CacheDesc(2, 4, 2, d, keep, bkv.BKV_BF16)
+p = lambda a: ctypes.c_void_p(a.ctypes.data)
+before = dst.copy()
+st = LIB.bkv_compact(ctypes.byref(g), p(src), None, p(idx), keep, ctypes.byref(gd), p(dst), None, None)
+assert st == CUDA, st
+assert np.array_equal(dst, before)
+scores = np.full((4, cap), 3.0, dtype=np.float32)
+out_idx = np.full((4, keep), -5, dtype=np.int32)
+st = LIB.bkv_select_topk(p(scores), 4, cap, keep, p(out_idx), None, 0, None)
+assert st == CUDA, st
+assert (out_idx == -5).all()
+outcome = np.full(1, 9, dtype=np.int32)
+assert LIB.bkv_selftest_wait_timeout(1000000, p(outcome), None) == CUDA
+assert outcome[0] == 9
+print("injected launch failures reported")
+"""
+
+
+def test_injected_launch_failure_is_reported_and_outputs_untouched(tmp_path):
+    """BKV_INJECT_LAUNCH_FAILURE makes every kernel launch fail before it is
+    enqueued: the entry points return BKV_ERR_CUDA and leave their outputs as
+    they were (run in a fresh process, since the flag is read once)."""
+    import subprocess
+    import sys
+    script = tmp_path / "inject.py"
+    script.write_text(INJECT_SCRIPT.format(root=ROOT))
+    env = dict(os.environ, BKV_INJECT_LAUNCH_FAILURE="1")
+    r = subprocess.run([sys.executable, str(script)], env=env, capture_output=True, text=True,
+                       timeout=300)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "injected launch failures reported" in r.stdout
+
+
+def test_selftest_rejects_bad_arguments():
+    assert LIB.bkv_selftest_wait_timeout(10, A, S) == INVALID          # limit too short
+    assert LIB.bkv_selftest_wait_timeout(10**9, A, S) == INVALID       # limit too long
+    assert LIB.bkv_selftest_wait_timeout(10**6, 0, S) == INVALID       # no outcome
+    assert LIB.bkv_selftest_wait_timeout(10**6, A + 2, S) == INVALID   # misaligned
+
+
+def test_compress_step_rejects_bad_rings():
+    """A decode-side query ring replaces recent_q and window; its sizes are
+    checked before anything is launched."""
+    def args(**kw):
+        a = bkv.StepArgs()
+        a.cache = desc()
+        a.k = a.v = A
+        a.L, a.K = 1000, 100
+        a.R, a.M, a.W = 8, 16, 64
+        a.beacons_in, a.n_beacons_in = A + 0x100000, 16
+        a.beacons_out = A + 0x200000
+        a.dst_cache = desc(cap=100)
+        a.k_dst, a.v_dst = A + 0x400000, A + 0x800000
+        a.workspace, a.workspace_bytes = A + 0x1000000, 1 << 40
+        a.query_ring, a.ring_cap, a.ring_pos = A + 0x2000000, 128, 500
+        for k, v in kw.items():
+            setattr(a, k, v)
+        return a
+
+    def call(a):
+        return LIB.bkv_compress_step(ctypes.byref(a), None, None)
+
+    assert call(args(recent_q=A)) == INVALID            # the ring replaces recent_q
+    assert call(args(window=A)) == INVALID              # ... and the window
+    assert call(args(ring_cap=0)) == INVALID
+    assert call(args(ring_cap=32)) == INVALID           # W > ring_cap
+    assert call(args(ring_pos=40)) == INVALID           # fewer queries written than W
+    assert call(args(query_ring=A + 0x2000008)) == INVALID  # misaligned
+    # the updated beacons must not overlap the ring
+    assert call(args(beacons_out=A + 0x2000000 + 256)) == INVALID

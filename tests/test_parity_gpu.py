@@ -464,3 +464,94 @@ def test_compress_step_in_place(case, dev):
     assert torch.equal(idx, out["idx"])
     assert np.array_equal(raw(t["k"])[:, :, :keep], raw(out["kd"]))
     assert np.array_equal(raw(t["v"])[:, :, :keep], raw(out["vd"]))
+
+
+RING_CASES = {
+    # ring of 300 slots, 700 queries written: the 200-row window starts at
+    # slot 200 and wraps to slot 99; the 8 recent rows are slots 92..99
+    "wraps_mid_window": dict(cap=300, pos=700, W=200, R=8),
+    # the window ends exactly at the ring's end (no wrap), recent rows too
+    "ends_at_ring_end": dict(cap=256, pos=512, W=128, R=16),
+    # the whole ring is the window, starting mid-ring; recent rows wrap
+    "full_ring": dict(cap=260, pos=1000 + 3, W=260, R=5),
+}
+
+
+@pytest.mark.parametrize("case", sorted(RING_CASES))
+def test_compress_step_query_ring(case, dev):
+    """The step reading its recent queries and window in place from a
+    decode-side query ring (slot of query t = t mod cap) equals the step on
+    the same queries unrolled into dense blocks, bit for bit, and matches the
+    oracle on the ring's newest rows (oracle.ring_rows)."""
+    bkv, synth = _lib(), _synth()
+    rc = RING_CASES[case]
+    cap, pos, W, R = rc["cap"], rc["pos"], rc["W"], rc["R"]
+    wl = small(n_layers=2, W=W, R=R, M=24, n_beacons_in=10, L=900, K=250, capacity=1000)
+    inp = synth.make_step_inputs(wl, seed=9)
+    gen = torch.Generator().manual_seed(cap + pos)
+    # the decode history: pos queries per query head, written into the ring in order
+    hist = (8.0 * torch.randn(wl.n_layers, wl.n_q_heads, 1, 128, generator=gen)
+            + 0.5 * torch.randn(wl.n_layers, wl.n_q_heads, pos, 128, generator=gen)
+            ).to(torch.bfloat16)
+    ring = torch.zeros(wl.n_layers, wl.n_q_heads, cap, 128, dtype=torch.bfloat16)
+    for t in range(pos):
+        ring[:, :, t % cap] = hist[:, :, t]
+    window = hist[:, :, pos - W:].contiguous()
+    recent = hist[:, :, pos - R:].contiguous()
+    np.testing.assert_array_equal(raw(window), oracle.ring_rows(raw(ring), pos % cap, W))
+    np.testing.assert_array_equal(raw(recent), oracle.ring_rows(raw(ring), pos % cap, R))
+    g = bkv.geometry_of(inp.k, wl.n_q_heads)
+    keep = min(wl.K, wl.L)
+    dst = bkv.Geometry(g.n_layers, g.n_q_heads, g.n_kv_heads, g.head_dim, keep, g.dtype)
+    k, v, bq = inp.k.to(dev), inp.v.to(dev), inp.beacons.to(dev)
+    ws = torch.empty(bkv.bkv_workspace_size(g, wl.L, R, wl.M, cap, wl.K), dtype=torch.uint8,
+                     device=dev)
+    outs = []
+    for use_ring in (False, True):
+        o = dict(bout=torch.zeros_like(bq),
+                 kd=torch.empty(wl.n_layers, wl.n_kv_heads, keep, 128, dtype=torch.bfloat16,
+                                device=dev),
+                 scores=torch.empty(wl.n_layers, wl.n_kv_heads, wl.L, device=dev),
+                 idx=torch.empty(wl.n_layers, wl.n_kv_heads, keep, dtype=torch.int32,
+                                 device=dev))
+        o["vd"] = torch.empty_like(o["kd"])
+        if use_ring:
+            nb, nl = bkv.bkv_compress_step(
+                g, k, v, wl.L, wl.K, None, R, bq, wl.beacons_in, wl.M, None, W, o["bout"], 0.0,
+                dst, o["kd"], o["vd"], o["scores"], o["idx"], ws, query_ring=ring.to(dev),
+                ring_pos=pos)
+        else:
+            nb, nl = bkv.bkv_compress_step(
+                g, k, v, wl.L, wl.K, recent.to(dev), R, bq, wl.beacons_in, wl.M,
+                window.to(dev), W, o["bout"], 0.0, dst, o["kd"], o["vd"], o["scores"], o["idx"],
+                ws)
+        torch.cuda.synchronize()
+        assert bkv.bkv_read_device_status()[0] == 0
+        assert (nb, nl) == (min(wl.M, wl.beacons_in + W), keep)
+        outs.append(o)
+    for name in ("bout", "kd", "vd", "scores", "idx"):
+        assert torch.equal(outs[0][name], outs[1][name]), name
+    # the oracle on the ring's newest rows
+    G = wl.group
+    out_b = raw(outs[1]["bout"])
+    s_all = outs[1]["scores"].double().cpu().numpy()
+    idx_all = outs[1]["idx"].cpu().numpy()
+    for l in range(wl.n_layers):
+        for h in range(wl.n_kv_heads):
+            kk, vv, _, bb, _ = synth.head_slice(inp, l, h)
+            rg = raw(ring[l, h * G:(h + 1) * G])
+            win_raw = oracle.ring_rows(rg, pos % cap, W)
+            win64 = oracle.ring_rows(f64(ring[l, h * G:(h + 1) * G]), pos % cap, W)
+            rec64 = oracle.newest_rows(win64, R) if R <= W else None
+            exact = True
+            for gq in range(G):
+                U_raw = np.concatenate([raw(bb[gq, :wl.beacons_in]), win_raw[gq]])
+                U64 = np.concatenate([f64(bb[gq, :wl.beacons_in]), win64[gq]])
+                picks = picks_from_rows(U_raw, out_b[l, h * G + gq, :nb])
+                exact &= check_fps(U64, picks, wl.M, f"ring {case} FPS l{l} q{h * G + gq}")
+            rec64 = oracle.ring_rows(f64(ring[l, h * G:(h + 1) * G]), pos % cap, R)
+            s_ref, _ = oracle.score_head(f64(kk), rec64,
+                                         outs[1]["bout"][l, h * G:(h + 1) * G].double().cpu().numpy(),
+                                         nb)
+            check_scores(s_all[l, h], s_ref, f"ring {case} scores l{l} h{h}")
+            check_topk(idx_all[l, h], s_ref, wl.K, f"ring {case} top-K l{l} h{h}")
