@@ -219,6 +219,15 @@ typedef struct {
   const void *query_ring;
   int64_t ring_cap;            /* slots per query head */
   int64_t ring_pos;            /* queries written so far (the next slot is ring_pos mod ring_cap) */
+  /* Optional second stream (cudaStream_t as void*, NULL: none).  With it, the
+   * aggregation runs in head batches on `stream` and each batch's top-K and
+   * compaction run on aux_stream while the next batch is aggregated; the step
+   * still starts after the work already on `stream` and everything it does is
+   * finished before anything enqueued on `stream` after it.  aux_stream must
+   * not be `stream`.  Applies to bf16 steps that evict rows; with it, phase
+   * event [3] marks the end of the last batch's aggregation and [4] and [5]
+   * the end of the selections and compactions still running after it. */
+  void *aux_stream;
 } bkv_step_args;
 
 #define BKV_STEP_EVENTS 6

@@ -56,7 +56,7 @@ class StepArgs(ctypes.Structure):
                 ("phase_events", ctypes.POINTER(ctypes.c_void_p)),
                 ("aggregate", ctypes.c_int32),
                 ("query_ring", ctypes.c_void_p), ("ring_cap", ctypes.c_int64),
-                ("ring_pos", ctypes.c_int64)]
+                ("ring_pos", ctypes.c_int64), ("aux_stream", ctypes.c_void_p)]
 
 STEP_EVENTS = 6
 
@@ -216,7 +216,8 @@ def bkv_compress_step(geom: Geometry, k, v, L: int, K: int, recent_q, R: int, be
                       n_beacons_in: int, M: int, window, W: int, beacons_out, scale: float,
                       dst: Geometry, k_dst, v_dst, scores_out=None, idx_out=None,
                       workspace=None, stream=None, phase_events=None,
-                      aggregate: str = "max", query_ring=None, ring_pos: int = 0) -> tuple[int, int]:
+                      aggregate: str = "max", query_ring=None, ring_pos: int = 0,
+                      aux_stream=None) -> tuple[int, int]:
     """One whole compression step; returns (beacons valid after, new cache length).
 
     phase_events: optional list of STEP_EVENTS torch.cuda.Event (timing enabled)
@@ -224,6 +225,8 @@ def bkv_compress_step(geom: Geometry, k, v, L: int, K: int, recent_q, R: int, be
     query_ring: optional decode-side ring [layers, q_heads, cap, d] holding query
     t in slot t % cap, with ring_pos queries written; recent_q and window must
     then be None (the recent rows and the window are the ring's newest R and W).
+    aux_stream: optional second torch.cuda.Stream on which each head batch's
+    top-K and compaction overlap the next batch's aggregation.
     """
     a = StepArgs()
     a.cache = geom.desc()
@@ -241,6 +244,8 @@ def bkv_compress_step(geom: Geometry, k, v, L: int, K: int, recent_q, R: int, be
     a.workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     a.stream = _stream(stream)
     a.aggregate = AGGREGATE[aggregate]
+    if aux_stream is not None:
+        a.aux_stream = _stream(aux_stream)
     if query_ring is not None:
         a.query_ring = _ptr(query_ring)
         a.ring_cap = query_ring.shape[2]

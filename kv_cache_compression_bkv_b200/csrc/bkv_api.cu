@@ -194,6 +194,70 @@ bkv_status score_entry(const bkv_cache_desc *desc, const void *k, int64_t L,
                                 scores, s);
 }
 
+// The aggregation, top-K and compaction of a step in head batches: batch b's
+// aggregation on `s`, its top-K and compaction on `aux` after an event, so
+// that they overlap the aggregation of batch b + 1 (the compaction, bound by
+// HBM, shares the SMs with the tensor-bound aggregation).  `s` finally waits
+// for `aux`.  Events [3] (after the last aggregation), [4] and [5] (after the
+// join) are recorded through `mark`.
+template <typename Mark>
+bkv_status run_batched_tail(const ScoreGeom &g, bool mean, const void *k, const void *recent,
+                            const void *bq, const ScoreWorkspace &w, const SelectInput &in,
+                            const CompactArgs &c, int32_t *idx, float *scores_out,
+                            long long keep, bool in_place, cudaStream_t s, cudaStream_t aux,
+                            Mark &&mark) {
+  constexpr int kBatches = 4;
+  const int H = g.n_heads();
+  const int nbat = std::min(kBatches, H);
+  cudaEvent_t ev[kBatches + 1] = {};
+  bkv_status st = BKV_OK;
+  for (int b = 0; b <= nbat && st == BKV_OK; ++b)
+    if (cudaEventCreateWithFlags(&ev[b], cudaEventDisableTiming) != cudaSuccess) st = BKV_ERR_CUDA;
+  const ScoreGeom gg = mean ? mean_grouping(g) : g;
+  const size_t row_bytes = static_cast<size_t>(c.row_bytes);
+  for (int b = 0; b < nbat && st == BKV_OK; ++b) {
+    const int h0 = static_cast<int>(static_cast<long long>(H) * b / nbat);
+    const int h1 = static_cast<int>(static_cast<long long>(H) * (b + 1) / nbat);
+    {
+      PhaseRange r("bkv aggregation (head batch)");
+      st = launch_score_colmax_tc(gg, k, recent, bq, w.c, w.ypart, mean, s, h0, h1 - h0);
+    }
+    if (st != BKV_OK) break;
+    if (cudaEventRecord(ev[b], s) != cudaSuccess || cudaStreamWaitEvent(aux, ev[b], 0) != cudaSuccess) {
+      st = BKV_ERR_CUDA;
+      break;
+    }
+    PhaseRange r("bkv top-K + compaction (head batch)");
+    SelectInput ib = in;
+    ib.src = in.src + static_cast<size_t>(h0) * static_cast<size_t>(g.L);
+    st = launch_select_topk(ib, h1 - h0, g.L, keep, idx + static_cast<size_t>(h0) * keep,
+                            scores_out ? scores_out + static_cast<size_t>(h0) * g.L : nullptr,
+                            nullptr, 0, aux);
+    if (st != BKV_OK) break;
+    CompactArgs cb = c;
+    const size_t src_off = static_cast<size_t>(h0) * static_cast<size_t>(c.src_cap) * row_bytes;
+    const size_t dst_off = static_cast<size_t>(h0) * static_cast<size_t>(c.dst_cap) * row_bytes;
+    cb.k_src = c.k_src ? c.k_src + src_off : nullptr;
+    cb.v_src = c.v_src ? c.v_src + src_off : nullptr;
+    cb.k_dst = c.k_dst ? c.k_dst + dst_off : nullptr;
+    cb.v_dst = c.v_dst ? c.v_dst + dst_off : nullptr;
+    cb.idx = c.idx + static_cast<size_t>(h0) * static_cast<size_t>(keep);
+    cb.n_heads = h1 - h0;
+    st = in_place ? launch_compact_inplace(cb, aux) : launch_compact(cb, aux);
+  }
+  if (st == BKV_OK && !mark(3)) st = BKV_ERR_CUDA;
+  // join (also after an error, so that `s` never runs ahead of work on `aux`)
+  if (ev[nbat] != nullptr) {
+    if (cudaEventRecord(ev[nbat], aux) != cudaSuccess ||
+        cudaStreamWaitEvent(s, ev[nbat], 0) != cudaSuccess)
+      st = BKV_ERR_CUDA;
+  }
+  for (int b = 0; b <= nbat; ++b)
+    if (ev[b] != nullptr) cudaEventDestroy(ev[b]);
+  if (st == BKV_OK && (!mark(4) || !mark(5))) st = BKV_ERR_CUDA;
+  return st;
+}
+
 }  // namespace
 }  // namespace bkv
 
@@ -399,6 +463,9 @@ bkv_status bkv_compress_step(const bkv_step_args *a, int32_t *n_beacons_out, int
                   overlaps(a->k_dst, db, a->v_dst, db)))
     return BKV_ERR_INVALID_ARG;
 
+  if (a->aux_stream != nullptr && a->aux_stream == a->stream) return BKV_ERR_INVALID_ARG;
+  const bool overlap = a->aux_stream != nullptr && d->dtype == BKV_BF16 && keep < a->L &&
+                       d->n_layers * d->n_kv_heads >= 2;
   FpsGeom f{d->n_layers, d->n_q_heads, d->head_dim, d->dtype, a->n_beacons_in, a->M, a->W,
             nb_used, w_cap, w_start};
   if (update && !fps_supported(f)) return BKV_ERR_UNSUPPORTED;
@@ -441,8 +508,6 @@ bkv_status bkv_compress_step(const bkv_step_args *a, int32_t *n_beacons_out, int
       st = launch_score_rowstats_tc(g, a->k, recent_src, bq, w.c, s);
       if (st != BKV_OK) return st;
       if (!mark(2)) return BKV_ERR_CUDA;
-      st = launch_score_colmax_tc(mean ? mean_grouping(g) : g, a->k, recent_src, bq, w.c, w.ypart,
-                                  mean, s);
     } else {
       st = launch_score_rowstats_simt(g, static_cast<const float *>(a->k),
                                       static_cast<const float *>(recent_src),
@@ -457,9 +522,39 @@ bkv_status bkv_compress_step(const bkv_step_args *a, int32_t *n_beacons_out, int
   } else if (!mark(2)) {
     return BKV_ERR_CUDA;
   }
-  if (!mark(3)) return BKV_ERR_CUDA;
   const SelectInput in = score_select_input(g, d->dtype, w, mean);
   const bool copy_all = keep >= a->L;
+  CompactArgs c;
+  c.k_src = static_cast<const uint8_t *>(a->k);
+  c.v_src = static_cast<const uint8_t *>(a->v);
+  c.k_dst = static_cast<uint8_t *>(a->k_dst);
+  c.v_dst = static_cast<uint8_t *>(a->v_dst);
+  c.idx = copy_all ? nullptr : idx;
+  c.n_heads = g.n_heads();
+  c.n_keep = keep;
+  c.src_cap = d->capacity;
+  c.dst_cap = dd->capacity;
+  c.row_bytes = static_cast<int>(d->head_dim * elem_size(d->dtype));
+  if (overlap) {
+    // Head batches: the aggregation of batch b on `s`; then, on the aux
+    // stream, batch b's top-K and compaction, which touch only batch b's
+    // heads, while `s` aggregates batch b + 1.  The compaction reads the
+    // cache only after the aggregation of its own heads (the event), and
+    // the row statistics of every head finished before the first batch.
+    st = run_batched_tail(g, mean, a->k, recent_src, bq, w, in, c, idx, a->scores_out, keep,
+                          in_place, s, static_cast<cudaStream_t>(a->aux_stream), mark);
+    if (st != BKV_OK) return st;
+    if (n_beacons_out) *n_beacons_out = nb_used;
+    if (new_len) *new_len = keep;
+    return BKV_OK;
+  }
+  if (need_scores && d->dtype == BKV_BF16) {
+    PhaseRange r("bkv aggregation");
+    st = launch_score_colmax_tc(mean ? mean_grouping(g) : g, a->k, recent_src, bq, w.c, w.ypart,
+                                mean, s);
+    if (st != BKV_OK) return st;
+  }
+  if (!mark(3)) return BKV_ERR_CUDA;
   {
     PhaseRange r("bkv top-K");
     if (!copy_all) {
@@ -478,17 +573,6 @@ bkv_status bkv_compress_step(const bkv_step_args *a, int32_t *n_beacons_out, int
   }
   if (!mark(4)) return BKV_ERR_CUDA;
   PhaseRange compact_range("bkv compaction");
-  CompactArgs c;
-  c.k_src = static_cast<const uint8_t *>(a->k);
-  c.v_src = static_cast<const uint8_t *>(a->v);
-  c.k_dst = static_cast<uint8_t *>(a->k_dst);
-  c.v_dst = static_cast<uint8_t *>(a->v_dst);
-  c.idx = copy_all ? nullptr : idx;
-  c.n_heads = g.n_heads();
-  c.n_keep = keep;
-  c.src_cap = d->capacity;
-  c.dst_cap = dd->capacity;
-  c.row_bytes = static_cast<int>(d->head_dim * elem_size(d->dtype));
   if (in_place) {
     // nothing to move when every row is kept
     st = copy_all ? BKV_OK : launch_compact_inplace(c, s);

@@ -61,9 +61,10 @@ ScoreWorkspace carve_score_workspace(const ScoreGeom &g, void *ws);
 // ---- score_tc.cu: bf16, head_dim 128, tcgen05 tensor cores
 bkv_status launch_score_rowstats_tc(const ScoreGeom &g, const void *k, const void *recent,
                                     const void *beacons, float *c, cudaStream_t stream);
+// heads [head0, head0 + head_count) only (head_count < 0: through the last head)
 bkv_status launch_score_colmax_tc(const ScoreGeom &g, const void *k, const void *recent,
                                   const void *beacons, const float *c, float *ypart, bool mean,
-                                  cudaStream_t stream);
+                                  cudaStream_t stream, int head0 = 0, int head_count = -1);
 
 // ---- score_simt.cu: f32, head_dim <= 128 (multiple of 4), CUDA cores
 bkv_status launch_score_rowstats_simt(const ScoreGeom &g, const float *k, const float *recent,

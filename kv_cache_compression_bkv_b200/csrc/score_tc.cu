@@ -414,7 +414,7 @@ __global__ void __launch_bounds__(p2_threads(kMean), 1)
     score_colmax_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreGeom g,
                         const uint16_t *__restrict__ recent, const uint16_t *__restrict__ beacons,
                         const float *__restrict__ c_in, float *__restrict__ ypart, int n_chunks,
-                        int chunk_tiles, int n_stages) {
+                        int chunk_tiles, int n_stages, int head0) {
   constexpr int kEpiWG = p2_epi_warpgroups(kMean);
   constexpr int kSplit = kEpiWG / 2;  // warpgroups per column sub-chunk
   extern __shared__ uint8_t smem_raw[];
@@ -429,7 +429,7 @@ __global__ void __launch_bounds__(p2_threads(kMean), 1)
   const int gi = bid % g.n_groups;
   bid /= g.n_groups;
   const int ci = bid % n_chunks;
-  const int head = bid / n_chunks;
+  const int head = head0 + bid / n_chunks;
   const int layer = head / g.n_kv_heads, kvh = head - layer * g.n_kv_heads;
   const long long L = g.L;
   const int n_tiles_all = static_cast<int>((L + kP2Keys - 1) / kP2Keys);
@@ -769,7 +769,7 @@ bkv_status launch_score_rowstats_tc(const ScoreGeom &g, const void *k, const voi
 
 bkv_status launch_score_colmax_tc(const ScoreGeom &g, const void *k, const void *recent,
                                   const void *beacons, const float *c, float *ypart, bool mean,
-                                  cudaStream_t stream) {
+                                  cudaStream_t stream, int head0, int head_count) {
   if (injected_launch_failure()) return BKV_ERR_CUDA;
   CUtensorMap map;
   if (!make_key_map(&map, k, g, kP2Keys)) return BKV_ERR_CUDA;
@@ -798,7 +798,9 @@ bkv_status launch_score_colmax_tc(const ScoreGeom &g, const void *k, const void 
     if (cudaGetDevice(&dev) == cudaSuccess)
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   }
-  const long long units = static_cast<long long>(g.n_heads()) * g.n_groups;
+  if (head_count < 0) head_count = g.n_heads() - head0;
+  if (head0 < 0 || head_count <= 0 || head0 + head_count > g.n_heads()) return BKV_OK;
+  const long long units = static_cast<long long>(head_count) * g.n_groups;
   int n_chunks = 1, chunk_tiles = n_tiles;
   double best_fill = 0.0;
   for (int nc = 1; nc <= std::max(1, n_tiles / 8) && nc <= 32; ++nc) {
@@ -819,10 +821,10 @@ bkv_status launch_score_colmax_tc(const ScoreGeom &g, const void *k, const void 
   const auto *bq = static_cast<const uint16_t *>(beacons);
   if (mean)
     score_colmax_kernel<true><<<static_cast<unsigned>(grid), p2_threads(true), smem, stream>>>(
-        map, g, rq, bq, c, ypart, n_chunks, chunk_tiles, stages);
+        map, g, rq, bq, c, ypart, n_chunks, chunk_tiles, stages, head0);
   else
     score_colmax_kernel<false><<<static_cast<unsigned>(grid), p2_threads(false), smem, stream>>>(
-        map, g, rq, bq, c, ypart, n_chunks, chunk_tiles, stages);
+        map, g, rq, bq, c, ypart, n_chunks, chunk_tiles, stages, head0);
   return cudaGetLastError() == cudaSuccess ? BKV_OK : BKV_ERR_CUDA;
 }
 

@@ -8,6 +8,13 @@ budget K and compacts into the other of two cache buffers.  The decode step
 itself is not simulated: the keys, values and queries of each interval come
 from the seeded trace generator (synth.trace_*) and are appended in one copy.
 With in_place the step compacts into the cache it scored (one cache buffer).
+
+With ring_cap set, the decode loop keeps the queries the way a serving loop
+would: every decode step appends its query of every (layer, query head) to a
+device ring of ring_cap slots (query t in slot t % ring_cap), and the step
+reads the recent queries and the window in place from that ring (the window
+wraps around the ring's end whenever ring_cap is not a multiple of the
+interval); no window or recent-query buffer is assembled.
 """
 from __future__ import annotations
 
@@ -36,6 +43,7 @@ class TraceRun:
     device: torch.device
     layers: int | None = None      # use only the first `layers` layers
     in_place: bool = False         # compact into the cache itself (one cache buffer)
+    ring_cap: int | None = None    # keep the queries in a decode-side ring of this many slots
     events: list[TraceEvent] = field(default_factory=list)
 
     def __post_init__(self):
@@ -60,8 +68,15 @@ class TraceRun:
         if self.in_place:  # source and destination are the same buffers
             self.cache.append(self.cache[0])
         self.beacons = [torch.zeros(Ly, Hq, tr.M, d, dtype=dt, device=dev) for _ in range(2)]
-        self.window = torch.empty(Ly, Hq, tr.interval, d, dtype=dt, device=dev)
-        self.recent = torch.empty(Ly, Hq, tr.R, d, dtype=dt, device=dev)
+        if self.ring_cap is not None:
+            if self.ring_cap < tr.interval:
+                raise ValueError("the ring must hold a whole interval of queries")
+            self.ring = torch.zeros(Ly, Hq, self.ring_cap, d, dtype=dt, device=dev)
+            self.window = self.recent = None
+        else:
+            self.ring = None
+            self.window = torch.empty(Ly, Hq, tr.interval, d, dtype=dt, device=dev)
+            self.recent = torch.empty(Ly, Hq, tr.R, d, dtype=dt, device=dev)
         self.idx_flat = torch.empty(Ly * Hkv * tr.K, dtype=torch.int32, device=dev)
         self.last_idx = None    # kept positions of the last event, [Ly][Hkv][kept]
         self.geom = bkv.Geometry(Ly, Hq, Hkv, d, self.cap, dt)
@@ -82,8 +97,14 @@ class TraceRun:
             kc, vc = self.cache[self.cur]
             kc[:, :, self.L:self.L + tr.interval].copy_(self.keys[:, :, t0:t1])
             vc[:, :, self.L:self.L + tr.interval].copy_(self.values[:, :, t0:t1])
-            self.window.copy_(self.queries[:, :, t0:t1])
-            self.recent.copy_(self.queries[:, :, t1 - tr.R:t1])
+            if self.ring is not None:
+                # each decode step appends its query to the ring
+                q = self.queries[:, :, t0:t1].to(self.device)
+                for t in range(t0, t1):
+                    self.ring[:, :, t % self.ring_cap].copy_(q[:, :, t - t0])
+            else:
+                self.window.copy_(self.queries[:, :, t0:t1])
+                self.recent.copy_(self.queries[:, :, t1 - tr.R:t1])
             L = self.L + tr.interval
             kd, vd = self.cache[1 - self.cur]
             bin_, bout = self.beacons[self.cur], self.beacons[1 - self.cur]
@@ -95,7 +116,8 @@ class TraceRun:
             nb, nl = bkv.bkv_compress_step(
                 self.geom, kc, vc, L, tr.K, self.recent, tr.R,
                 bin_ if self.n_beacons else None, self.n_beacons, tr.M, self.window,
-                tr.interval, bout, 0.0, self.geom, kd, vd, None, idx, self.ws, stream)
+                tr.interval, bout, 0.0, self.geom, kd, vd, None, idx, self.ws, stream,
+                query_ring=self.ring, ring_pos=t1)
             ev1.record(stream)
             torch.cuda.synchronize(self.device)
             event = TraceEvent(e, t1, L, nl, self.n_beacons, nb, ev0.elapsed_time(ev1))

@@ -201,7 +201,7 @@ def test_update_beacons(case, dev):
             check_fps(f64(U), picks, wl.M, f"{case} l{l} q{qh}")
 
 
-def _run_step(wl, inp, dev, scores=True, aggregate="max"):
+def _run_step(wl, inp, dev, scores=True, aggregate="max", aux=False):
     bkv = _lib()
     g = bkv.geometry_of(inp.k, wl.n_q_heads)
     keep = min(wl.K, wl.L)
@@ -221,7 +221,8 @@ def _run_step(wl, inp, dev, scores=True, aggregate="max"):
         g, t["k"], t["v"], wl.L, wl.K, t["recent"] if wl.R else None, wl.R,
         t["beacons"] if wl.beacons_in else None, wl.beacons_in, wl.M,
         t["window"] if wl.W else None, wl.W, out["bout"], 0.0, dst, out["kd"], out["vd"],
-        out["scores"], out["idx"], ws, aggregate=aggregate)
+        out["scores"], out["idx"], ws, aggregate=aggregate,
+        aux_stream=torch.cuda.Stream(device=dev, priority=-1) if aux else None)
     torch.cuda.synchronize()
     assert bkv.bkv_read_device_status()[0] == 0
     assert nl == keep
@@ -319,7 +320,7 @@ def test_full_size_sampled(name, dev):
     synth = _synth()
     wl = synth.WORKLOADS[name]
     inp = synth.make_step_inputs(wl, seed=0)
-    out, nb = _run_step(wl, inp, dev)
+    out, nb = _run_step(wl, inp, dev, aux=True)
     rng = np.random.default_rng(123)
     heads = sorted({(int(rng.integers(wl.n_layers)), int(rng.integers(wl.n_kv_heads)))
                     for _ in range(7)} | {(0, 0), (wl.n_layers - 1, wl.n_kv_heads - 1)})
@@ -341,7 +342,7 @@ def test_full_size_sampled_mean(dev):
     synth = _synth()
     wl = synth.WORKLOADS["qwen3_14b"]
     inp = synth.make_step_inputs(wl, seed=5)
-    out, nb = _run_step(wl, inp, dev, aggregate="mean")
+    out, nb = _run_step(wl, inp, dev, aggregate="mean", aux=True)
     rng = np.random.default_rng(321)
     heads = sorted({(int(rng.integers(wl.n_layers)), int(rng.integers(wl.n_kv_heads)))
                     for _ in range(2)} | {(0, 0)})
@@ -555,3 +556,37 @@ def test_compress_step_query_ring(case, dev):
                                          nb)
             check_scores(s_all[l, h], s_ref, f"ring {case} scores l{l} h{h}")
             check_topk(idx_all[l, h], s_ref, wl.K, f"ring {case} top-K l{l} h{h}")
+
+
+@pytest.mark.parametrize("case,aggregate", [("bf16_fps", "max"), ("bf16_fps", "mean"),
+                                            ("no_window", "max")])
+def test_compress_step_aux_stream(case, aggregate, dev):
+    """With a second stream, each head batch's top-K and compaction overlap the
+    next batch's aggregation; the results are those of the one-stream step,
+    bit for bit (out of place, then in place)."""
+    wl = STEP_CASES[case]().replace(n_layers=3, n_kv_heads=2, n_q_heads=8)
+    inp = _synth().make_step_inputs(wl, seed=13)
+    one, nb1 = _run_step(wl, inp, dev, aggregate=aggregate)
+    two, nb2 = _run_step(wl, inp, dev, aggregate=aggregate, aux=True)
+    assert nb1 == nb2
+    for name in ("bout", "kd", "vd", "scores", "idx"):
+        assert torch.equal(one[name], two[name]), name
+    # in place with the aux stream: the cache itself becomes the compacted one
+    bkv = _lib()
+    g = bkv.geometry_of(inp.k, wl.n_q_heads)
+    t = {n: getattr(inp, n).to(dev) for n in ("k", "v", "recent", "beacons", "window")}
+    keep = min(wl.K, wl.L)
+    idx = torch.empty(wl.n_layers, wl.n_kv_heads, keep, dtype=torch.int32, device=dev)
+    ws = torch.empty(bkv.bkv_workspace_size(g, wl.L, wl.R, wl.M, wl.W, wl.K), dtype=torch.uint8,
+                     device=dev)
+    bkv.bkv_compress_step(
+        g, t["k"], t["v"], wl.L, wl.K, t["recent"] if wl.R else None, wl.R,
+        t["beacons"] if wl.beacons_in else None, wl.beacons_in, wl.M,
+        t["window"] if wl.W else None, wl.W, torch.zeros_like(t["beacons"]), 0.0, g, t["k"],
+        t["v"], None, idx, ws, aggregate=aggregate,
+        aux_stream=torch.cuda.Stream(device=dev, priority=-1))
+    torch.cuda.synchronize()
+    assert bkv.bkv_read_device_status()[0] == 0
+    assert torch.equal(idx, one["idx"])
+    assert np.array_equal(raw(t["k"])[:, :, :keep], raw(one["kd"]))
+    assert np.array_equal(raw(t["v"])[:, :, :keep], raw(one["vd"]))

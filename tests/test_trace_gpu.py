@@ -23,15 +23,19 @@ from parity_helpers import check_fps, check_topk, f64, picks_from_rows, raw
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
 
-@pytest.mark.parametrize("in_place", [False, True])
-def test_qwen3_4b_trace_follows_the_oracle_trace(in_place):
+@pytest.mark.parametrize("in_place,ring_cap", [(False, None), (True, None), (False, 5000)])
+def test_qwen3_4b_trace_follows_the_oracle_trace(in_place, ring_cap):
+    """ring_cap: the decode loop appends every query to a 5000-slot ring and
+    the step reads the window and recent queries from it in place (the
+    4096-query window wraps around the ring's end at most events)."""
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA device")
     from kv_cache_compression_bkv_b200 import synth
     from kv_cache_compression_bkv_b200.trace import TraceRun
 
     tr = synth.TRACES["qwen3_4b_trace"]
-    run = TraceRun(tr, seed=0, device=torch.device("cuda:0"), layers=1, in_place=in_place)
+    run = TraceRun(tr, seed=0, device=torch.device("cuda:0"), layers=1, in_place=in_place,
+                   ring_cap=ring_cap)
     G, Hkv, I, K, M, R = tr.group, tr.n_kv_heads, tr.interval, tr.K, tr.M, tr.R
     keys_raw = raw(run.keys[0])          # [Hkv, steps, d]
     vals_raw = raw(run.values[0])
@@ -86,4 +90,5 @@ def test_qwen3_4b_trace_follows_the_oracle_trace(in_place):
     assert events[0].L == I and events[0].new_len == min(K, I) and events[0].n_beacons_out == M
     assert all(e.L == K + I and e.new_len == K for e in events[1:])
     assert sum(counts.values()) == Hkv * len(events), counts
-    print(f"trace ({'in place' if in_place else 'out of place'}): {counts}")
+    print(f"trace ({'in place' if in_place else 'out of place'}"
+          f"{', query ring' if ring_cap else ''}): {counts}")
