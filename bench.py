@@ -467,9 +467,10 @@ def main():
                     help="use only this many layers (small cases for profiler captures)")
     ap.add_argument("--aggregate", default="max", choices=["max", "mean"],
                     help="aggregation over the observation rows (mean: Table 2's ablation)")
-    ap.add_argument("--no-overlap", action="store_true",
-                    help="run the step on one stream (no overlap of the top-K and compaction "
-                         "of one head batch with the aggregation of the next)")
+    ap.add_argument("--overlap", action="store_true",
+                    help="give the step a second stream: each head batch's top-K and compaction "
+                         "overlap the next batch's aggregation (measured slower on B200 than one "
+                         "stream, so off by default)")
     ap.add_argument("--in-place", action="store_true",
                     help="compact into the scored cache itself (bkv_compress_step with "
                          "k_dst == k)")
@@ -542,7 +543,7 @@ def main():
     stream = torch.cuda.current_stream()
     # the second stream on which each head batch's top-K and compaction overlap
     # the next batch's aggregation (high priority: its CTAs go first)
-    aux = None if args.no_overlap else torch.cuda.Stream(device=dev, priority=-1)
+    aux = torch.cuda.Stream(device=dev, priority=-1) if args.overlap else None
 
     def step(events=None, t=devt, o=None, st=None, overlap=True):
         o = o or {"kd": kd, "vd": vd, "bout": bout, "idx": idx}

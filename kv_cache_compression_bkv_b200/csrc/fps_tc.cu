@@ -351,107 +351,151 @@ __device__ void distance_pass(const Layout &s, const CUtensorMap *bmap, const CU
   }
 }
 
-// Append (i, d) to the candidate slots with one atomic per warp (lanes with
-// `take` set); slots past kCand are dropped.
-__device__ __forceinline__ void push_candidate(const Layout &s, bool take, int i, float d,
-                                               int base_slot) {
+// Exclusive prefix sum over the block of one value per thread (`scratch`:
+// kWarps words); every thread gets its own prefix.
+__device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t *scratch) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) scratch[warp] = incl;
+  __syncthreads();
+  uint32_t before = 0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w)
+    if (w < warp) before += scratch[w];
+  return before + incl - v;
+}
+
+// Points of a union that the selection keeps in registers (n <= kPerThread *
+// kThreads); larger unions take the radix select.
+constexpr int kPerThread = 16;
+
+// Warp 0: the bin of `hist` (256 bins, highest first) that holds the
+// want-th key: its index, the keys in the bins above it, and the keys still
+// wanted from it, in scal[kSBin], [kSAbove], [kSNeed]; scal[kSFallback] is set
+// when that bin holds more than `list_max` keys or fewer than `want` keys
+// are counted at all.
+__device__ __forceinline__ void find_threshold_bin(const Layout &s, int want, int list_max) {
   const int lane = threadIdx.x & 31;
-  const uint32_t bal = __ballot_sync(0xffffffffu, take);
-  int wbase = 0;
-  if (lane == 0 && bal) wbase = atomicAdd(&s.scal[kSCand], __popc(bal));
-  wbase = __shfl_sync(0xffffffffu, wbase, 0);
-  if (take) {
-    const int slot = base_slot + wbase + __popc(bal & ((1u << lane) - 1u));
-    if (slot < kCand) {
-      s.cidx[slot] = i;
-      s.cdist[slot] = d;
+  // lane l holds bins 255-8l .. 248-8l: two 16-byte loads of its 8
+  // consecutive words (no bank conflicts), highest bin first
+  const uint4 lo4 = *reinterpret_cast<const uint4 *>(s.hist + 248 - 8 * lane);
+  const uint4 hi4 = *reinterpret_cast<const uint4 *>(s.hist + 252 - 8 * lane);
+  const uint32_t cnt[8] = {hi4.w, hi4.z, hi4.y, hi4.x, lo4.w, lo4.z, lo4.y, lo4.x};
+  uint32_t local = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) local += cnt[j];
+  uint32_t incl = local;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t o = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += o;
+  }
+  const uint32_t excl = incl - local;
+  if (static_cast<int>(excl) < want && want <= static_cast<int>(incl)) {
+    uint32_t acc = excl;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (static_cast<int>(acc + cnt[j]) >= want) {
+        s.scal[kSBin] = 255 - 8 * lane - j;
+        s.scal[kSAbove] = static_cast<int>(acc);
+        s.scal[kSNeed] = want - static_cast<int>(acc);
+        s.scal[kSFallback] = cnt[j] > static_cast<uint32_t>(list_max) ? 1 : 0;
+        break;
+      }
+      acc += cnt[j];
     }
   }
+  if (lane == 31 && static_cast<int>(incl) < want) s.scal[kSFallback] = 1;
 }
 
 // Step 1 of a round: the `want` live points with the largest u in (u desc,
-// index asc) order: the first kCand in slots 0.. (any order), the (kCand+1)-th
-// -- the bound -- in slot kCand when `bounded`.  A 256-bin histogram of u
-// over [0, dmax] finds the bin holding the want-th key; keys above it are
-// taken, keys in it are ranked against each other.  Returns false (nothing
-// written) when that bin holds more than kListMax keys or the live keys are
-// fewer than counted (NaN distances): the caller then uses the radix select.
+// index asc) order: the first kCand in slots 0.. , the (kCand+1)-th -- the
+// bound -- in slot kCand when `bounded`.  Two histogram levels: 256 bins of u
+// over [0, dmax] find the bin holding the want-th key, then 256 sub-bins of
+// that bin's range find the sub-bin holding it; keys above are taken and the
+// keys of that sub-bin are ranked against each other.  Both bin maps are
+// monotonic in u, so the order is exact.  Each thread keeps its points' u
+// and bins in registers, and the points are placed by a block-wide prefix sum
+// of per-thread counts (no atomic counters).  Returns false (nothing written)
+// when the union is too large for that, the final sub-bin holds more than
+// kListMax keys, or the live keys are fewer than counted (NaN distances): the
+// caller then uses the radix select.
 __device__ bool select_hist(const Layout &s, int n, int want, bool bounded, float dmax) {
+  if (n > kPerThread * kThreads) return false;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const float scale = dmax > 0.f ? 256.f / dmax : 0.f;
   for (int b = tid; b < 256; b += kThreads) s.hist[b] = 0u;
-  if (tid == 0) {
-    s.scal[kSCand] = 0;
-    s.scal[kSList] = 0;
-    s.scal[kSLive] = 0;
-  }
+  if (tid == 0) s.scal[kSLive] = 0;
   __syncthreads();
+  float du[kPerThread];
+  int bins[kPerThread];
   int live = 0;
-  for (int i = tid; i < n; i += kThreads) {
-    const float d = s.dist[i];
-    if (d >= 0.f) {
-      atomicAdd(&s.hist[min(255, static_cast<int>(d * scale))], 1u);
+#pragma unroll
+  for (int k = 0; k < kPerThread; ++k) {
+    const int i = tid + k * kThreads;
+    du[k] = i < n ? s.dist[i] : -1.f;
+    bins[k] = du[k] >= 0.f ? min(255, static_cast<int>(du[k] * scale)) : -1;
+    if (bins[k] >= 0) {
+      atomicAdd(&s.hist[bins[k]], 1u);
       ++live;
     }
   }
   live = __reduce_add_sync(0xffffffffu, live);
   if (lane == 0) atomicAdd(&s.scal[kSLive], live);
   __syncthreads();
-  if (warp == 0) {
-    // lane l holds bins 255-8l .. 248-8l (descending)
-    uint32_t cnt[8], local = 0;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      cnt[j] = s.hist[255 - 8 * lane - j];
-      local += cnt[j];
-    }
-    uint32_t incl = local;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const uint32_t o = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += o;
-    }
-    const uint32_t excl = incl - local;
-    if (static_cast<int>(excl) < want && want <= static_cast<int>(incl)) {
-      uint32_t acc = excl;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (static_cast<int>(acc + cnt[j]) >= want) {
-          s.scal[kSBin] = 255 - 8 * lane - j;
-          s.scal[kSAbove] = static_cast<int>(acc);
-          s.scal[kSNeed] = want - static_cast<int>(acc);
-          s.scal[kSFallback] = cnt[j] > static_cast<uint32_t>(kListMax) ? 1 : 0;
-          break;
-        }
-        acc += cnt[j];
-      }
-    }
-    if (lane == 31 && static_cast<int>(incl) < want) s.scal[kSFallback] = 1;
-  }
+  if (warp == 0) find_threshold_bin(s, want, n);
   __syncthreads();
   if (s.scal[kSFallback] || s.scal[kSLive] < want) return false;
-  const int bstar = s.scal[kSBin], above = s.scal[kSAbove], need = s.scal[kSNeed];
-  // keys above the threshold bin are candidates; the bin's keys are listed
-  for (int base = 0; base < n; base += kThreads) {
-    const int i = base + tid;
-    const float d = i < n ? s.dist[i] : -1.f;
-    const int b = d >= 0.f ? min(255, static_cast<int>(d * scale)) : -1;
-    push_candidate(s, b > bstar, i, d, 0);
-    const bool inbin = b == bstar;
-    const uint32_t bal = __ballot_sync(0xffffffffu, inbin);
-    int wbase = 0;
-    if (lane == 0 && bal) wbase = atomicAdd(&s.scal[kSList], __popc(bal));
-    wbase = __shfl_sync(0xffffffffu, wbase, 0);
-    if (inbin) {
-      const int pos = wbase + __popc(bal & ((1u << lane) - 1u));
-      s.lkey[pos] = dist_key(d);
-      s.lidx[pos] = i;
-    }
+  const int bstar = s.scal[kSBin], above1 = s.scal[kSAbove], need1 = s.scal[kSNeed];
+  __syncthreads();  // the scalars are read; hist and scal are reused below
+  // level 2: the threshold bin's range in 256 sub-bins
+  for (int b = tid; b < 256; b += kThreads) s.hist[b] = 0u;
+  __syncthreads();
+  const float fb = static_cast<float>(bstar);
+  int sub[kPerThread];
+#pragma unroll
+  for (int k = 0; k < kPerThread; ++k) {
+    sub[k] = bins[k] == bstar ? min(255, max(0, static_cast<int>((du[k] * scale - fb) * 256.f)))
+                              : -1;
+    if (sub[k] >= 0) atomicAdd(&s.hist[sub[k]], 1u);
   }
   __syncthreads();
-  // rank the bin's keys (key desc, index asc): rank r < need is taken, the
-  // last taken one (rank need-1) is the bound when the selection is bounded
-  const int listed = s.scal[kSList];
+  if (warp == 0) find_threshold_bin(s, need1, kListMax);
+  __syncthreads();
+  if (s.scal[kSFallback]) return false;
+  const int sstar = s.scal[kSBin], above = above1 + s.scal[kSAbove], need = s.scal[kSNeed];
+  // keys above the threshold (slots 0 .. above-1) and the keys of the final
+  // sub-bin (listed), placed by a prefix sum of (above count << 16 | listed)
+  uint32_t na = 0, nl = 0;
+#pragma unroll
+  for (int k = 0; k < kPerThread; ++k) {
+    na += (bins[k] > bstar || (bins[k] == bstar && sub[k] > sstar)) ? 1u : 0u;
+    nl += (bins[k] == bstar && sub[k] == sstar) ? 1u : 0u;
+  }
+  const uint32_t pre = block_exclusive_scan((na << 16) | nl, s.whist);
+  int pa = static_cast<int>(pre >> 16), pb = static_cast<int>(pre & 0xffffu);
+#pragma unroll
+  for (int k = 0; k < kPerThread; ++k) {
+    const int i = tid + k * kThreads;
+    if (bins[k] > bstar || (bins[k] == bstar && sub[k] > sstar)) {
+      s.cidx[pa] = i;
+      s.cdist[pa] = du[k];
+      ++pa;
+    } else if (bins[k] == bstar && sub[k] == sstar) {
+      s.lkey[pb] = dist_key(du[k]);
+      s.lidx[pb] = i;
+      ++pb;
+    }
+  }
+  const int listed = static_cast<int>(s.hist[sstar]);
+  __syncthreads();
+  // rank the sub-bin's keys (key desc, index asc): rank r < need is taken,
+  // the last taken one (rank need-1) is the bound when the selection is bounded
   for (int e = tid; e < listed; e += kThreads) {
     const uint32_t ke = s.lkey[e];
     const int ie = s.lidx[e];
@@ -463,7 +507,7 @@ __device__ bool select_hist(const Layout &s, int n, int want, bool bounded, floa
     if (rank < need) {
       const int slot = bounded && rank == need - 1 ? kCand : above + rank;
       s.cidx[slot] = ie;
-      s.cdist[slot] = s.dist[ie];
+      s.cdist[slot] = __uint_as_float(ke & 0x7fffffffu);
     }
   }
   __syncthreads();
@@ -621,13 +665,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       // lowest stamp among them (candidates behind P are refreshed)
       if (tid == 0) s.scal[kSRef] = P;
       __syncthreads();
-      for (int e = tid; e < nc * 16; e += kThreads) {
-        const int a = e >> 4, c16 = e & 15, kb = c16 >> 3, c = c16 & 7;
-        const int i = s.cidx[a];
-        *reinterpret_cast<uint4 *>(s.cop + kb * kCBlock + sw128_offset(a, c)) =
-            *reinterpret_cast<const uint4 *>(h.point(i) + c16 * 8);
-        if (c16 == 0) {
-          const int t = s.stamp[i];
+      {
+        // every load of this thread's pieces is issued before the first store
+        constexpr int kIters = (kCand * 16 + kThreads - 1) / kThreads;
+        uint4 v[kIters];
+#pragma unroll
+        for (int u = 0; u < kIters; ++u) {
+          const int e = tid + u * kThreads;
+          if (e < nc * 16)
+            v[u] = __ldg(reinterpret_cast<const uint4 *>(h.point(s.cidx[e >> 4]) + (e & 15) * 8));
+        }
+#pragma unroll
+        for (int u = 0; u < kIters; ++u) {
+          const int e = tid + u * kThreads;
+          if (e < nc * 16) {
+            const int a = e >> 4, c16 = e & 15;
+            *reinterpret_cast<uint4 *>(s.cop + (c16 >> 3) * kCBlock + sw128_offset(a, c16 & 7)) =
+                v[u];
+          }
+        }
+        if (tid < nc) {
+          const int t = s.stamp[s.cidx[tid]];
           if (t < P) atomicMin(&s.scal[kSRef], t);
         }
       }

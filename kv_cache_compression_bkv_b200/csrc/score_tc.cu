@@ -171,15 +171,16 @@ __device__ __forceinline__ const uint16_t *obs_row(const ScoreGeom &g, const uin
 
 // Gather observation rows [row0, row0 + nrows) into shared memory as a
 // K-major operand: two K blocks of nrows x 128 B, 128-byte swizzle.  Rows at
-// or past n_obs are zero.
+// or past n_obs are zero.  With `dup_half`, rows nrows/2.. repeat rows 0..
+// (row r holds observation row row0 + r mod nrows/2).
 __device__ __forceinline__ void load_obs_rows_sw128(uint8_t *dst, int nrows, int row0,
                                                     const ScoreGeom &g, const uint16_t *recent,
-                                                    const uint16_t *beacons, int layer,
-                                                    int kvh) {
+                                                    const uint16_t *beacons, int layer, int kvh,
+                                                    bool dup_half = false) {
   const int kb_stride = nrows * kKbBytes;
   for (int id = threadIdx.x; id < nrows * 16; id += blockDim.x) {
     const int r = id >> 4, c16 = id & 15, kb = c16 >> 3, c = c16 & 7;
-    const int o = row0 + r;
+    const int o = row0 + (dup_half ? r % (nrows / 2) : r);
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
     if (o < g.n_obs) v = ldg_nc_v4(obs_row(g, recent, beacons, layer, kvh, o) + c16 * 8);
     *reinterpret_cast<uint4 *>(dst + kb * kb_stride + sw128_offset(r, c)) = v;
@@ -239,7 +240,11 @@ __global__ void __launch_bounds__(kP1Threads, 1)
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
-  load_obs_rows_sw128(sA, kP1Rows, rb * kP1Rows, g, recent, beacons, layer, kvh);
+  // A block with at most 64 valid rows (the ragged last block) holds them
+  // twice, in TMEM lanes 0-63 and 64-127; each copy then takes half of every
+  // tile's columns, so the block's exps are not spent on padding rows.
+  const bool half = g.n_obs - rb * kP1Rows <= kP1Rows / 2;
+  load_obs_rows_sw128(sA, kP1Rows, rb * kP1Rows, g, recent, beacons, layer, kvh, half);
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -303,6 +308,10 @@ __global__ void __launch_bounds__(kP1Threads, 1)
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const float kz = g.scale * kLog2e;
+    // in a half block, lanes 0-63 take the first 64-column block of this
+    // warpgroup's 128 columns and lanes 64-127 (the same rows) the second
+    const int b_first = half ? (quarter >> 1) : 0;
+    const int b_last = half ? (quarter >> 1) : 1;
     float m = -INFINITY, ssum = 0.f;
     bool ok = true;
     for (int t = wg >> 1; t < n_tiles && ok; t += 2) {
@@ -310,7 +319,7 @@ __global__ void __launch_bounds__(kP1Threads, 1)
       if (!mbar_wait_warp(tfull0 + 8 * acc, (t >> 1) & 1, kWhereP1Epi)) { ok = false; break; }
       tc_fence_after();
 #pragma unroll 1
-      for (int b = 0; b < 2; ++b) {
+      for (int b = b_first; b <= b_last; ++b) {
         const int col = (wg & 1) * 128 + b * 64;
         const uint32_t taddr =
             tmem + (static_cast<uint32_t>(quarter * 32) << 16) + acc * kP1Keys + col;
@@ -320,7 +329,7 @@ __global__ void __launch_bounds__(kP1Threads, 1)
         tmem_ld_32x32b_x32(taddr + 32, vb);
         tmem_ld_wait_regs(va);
         tmem_reg_fence(vb);
-        if (b == 1) {
+        if (b == b_last) {
           // the accumulator is free once this warp's last loads have landed
           tc_fence_before();
           __syncwarp();
@@ -348,29 +357,32 @@ __global__ void __launch_bounds__(kP1Threads, 1)
         ssum += bs;
       }
     }
-    // combine the four warpgroups' partial sums of each row; the exchange
-    // reuses the key stages, free once every tile's MMAs have completed --
-    // which the warpgroup of the last tile has seen, so all wait for it
+    // combine the partial sums of each row: the four warpgroups' (and, in a
+    // half block, the two lanes that hold the same row); the exchange reuses
+    // the key stages, free once every tile's MMAs have completed -- which the
+    // warpgroup of the last tile has seen, so all wait for it
     named_barrier_sync(1, 32 * kP1EpiWarps);
-    float *xchg = reinterpret_cast<float *>(sB);  // [3][128][2]
-    if (wg > 0) {
-      xchg[((wg - 1) * kP1Rows + row) * 2] = m;
-      xchg[((wg - 1) * kP1Rows + row) * 2 + 1] = ok ? ssum : -1.f;
-    }
+    float *xchg = reinterpret_cast<float *>(sB);  // [4][128][2]
+    xchg[(wg * kP1Rows + row) * 2] = m;
+    xchg[(wg * kP1Rows + row) * 2 + 1] = ok ? ssum : -1.f;
     named_barrier_sync(1, 32 * kP1EpiWarps);
-    if (wg == 0) {
+    const int n_lanes = half ? kP1Rows / 2 : kP1Rows;  // lanes holding distinct rows
+    if (wg == 0 && row < n_lanes) {
       const int o = rb * kP1Rows + row;
-      float M = m;
-      bool all_ok = ok;
-      for (int w = 0; w < 3; ++w) {
-        M = fmaxf(M, xchg[(w * kP1Rows + row) * 2]);
-        all_ok &= xchg[(w * kP1Rows + row) * 2 + 1] >= 0.f;
+      const int n_parts = half ? 8 : 4;
+      float M = -INFINITY;
+      bool all_ok = true;
+      for (int p = 0; p < n_parts; ++p) {
+        const int w = p & 3, r = row + (p >> 2) * (kP1Rows / 2);
+        M = fmaxf(M, xchg[(w * kP1Rows + r) * 2]);
+        all_ok &= xchg[(w * kP1Rows + r) * 2 + 1] >= 0.f;
       }
       if (all_ok && o < g.n_obs) {
-        float S = m == -INFINITY ? 0.f : ssum * ex2_approx(m - M);
-        for (int w = 0; w < 3; ++w) {
-          const float mw = xchg[(w * kP1Rows + row) * 2];
-          const float sw = xchg[(w * kP1Rows + row) * 2 + 1];
+        float S = 0.f;
+        for (int p = 0; p < n_parts; ++p) {
+          const int w = p & 3, r = row + (p >> 2) * (kP1Rows / 2);
+          const float mw = xchg[(w * kP1Rows + r) * 2];
+          const float sw = xchg[(w * kP1Rows + r) * 2 + 1];
           if (mw != -INFINITY) S += sw * ex2_approx(mw - M);
         }
         c_out[static_cast<size_t>(head) * g.n_obs_pad + o] = (M + log2f(S)) * kLn2;

@@ -77,6 +77,37 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t *w
   return wpre + incl - v;
 }
 
+// Four consecutive values of a row (off a multiple of 4, the row 16-byte
+// aligned), merged over the parts like load_key_value.
+__device__ __forceinline__ float4 load_key_value4(const SelectInput &in, size_t off) {
+  float4 v = *reinterpret_cast<const float4 *>(in.src + off);
+  for (int p = 1; p < in.n_parts; ++p) {
+    const float4 w = *reinterpret_cast<const float4 *>(in.src + p * in.part_stride + off);
+    if (in.mean) {
+      v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
+    } else {
+      v.x = fmaxf(v.x, w.x); v.y = fmaxf(v.y, w.y); v.z = fmaxf(v.z, w.z); v.w = fmaxf(v.w, w.w);
+    }
+  }
+  if (in.mean) {
+    v.x *= in.inv_count; v.y *= in.inv_count; v.z *= in.inv_count; v.w *= in.inv_count;
+  }
+  return v;
+}
+
+// Inclusive prefix sum across the warp.
+__device__ __forceinline__ uint32_t warp_inclusive_scan(uint32_t v, int lane) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += t;
+  }
+  return v;
+}
+
+// kVec: the row length is a multiple of 4 and rows are 16-byte aligned, so
+// every pass reads float4s (four keys per thread and load).
+template <bool kVec>
 __global__ void __launch_bounds__(kThreads)
     select_topk_kernel(const SelectInput in, long long L, long long K, int32_t *__restrict__ idx,
                        float *__restrict__ s_out) {
@@ -98,11 +129,37 @@ __global__ void __launch_bounds__(kThreads)
     const int nb = 1 << nbits;
     for (int b = tid; b < nb; b += kThreads) hist[b] = 0u;
     __syncthreads();
-    for (long long j = tid; j < L; j += kThreads) {
-      const float v = load_key_value(in, rbase + j);
-      if (hi == 32 && s_out) s_out[rbase + j] = score_of_key(in, v);
-      const uint32_t key = order_key(v);
+    auto count = [&](uint32_t key) {
       if ((key & mask) == prefix) atomicAdd(&hist[(key >> lo) & dmask], 1u);
+    };
+    if (kVec) {
+      // two float4 loads in flight per thread before their keys are counted
+      const long long L4 = L >> 2;
+      for (long long q = tid; q < L4; q += 2 * kThreads) {
+        const long long q2 = q + kThreads;
+        const float4 a = load_key_value4(in, rbase + 4 * q);
+        float4 b = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (q2 < L4) b = load_key_value4(in, rbase + 4 * q2);
+        if (hi == 32 && s_out) {
+          *reinterpret_cast<float4 *>(s_out + rbase + 4 * q) =
+              make_float4(score_of_key(in, a.x), score_of_key(in, a.y), score_of_key(in, a.z),
+                          score_of_key(in, a.w));
+          if (q2 < L4)
+            *reinterpret_cast<float4 *>(s_out + rbase + 4 * q2) =
+                make_float4(score_of_key(in, b.x), score_of_key(in, b.y), score_of_key(in, b.z),
+                            score_of_key(in, b.w));
+        }
+        count(order_key(a.x)); count(order_key(a.y)); count(order_key(a.z)); count(order_key(a.w));
+        if (q2 < L4) {
+          count(order_key(b.x)); count(order_key(b.y)); count(order_key(b.z)); count(order_key(b.w));
+        }
+      }
+    } else {
+      for (long long j = tid; j < L; j += kThreads) {
+        const float v = load_key_value(in, rbase + j);
+        if (hi == 32 && s_out) s_out[rbase + j] = score_of_key(in, v);
+        count(order_key(v));
+      }
     }
     __syncthreads();
     // bins in descending digit order, 4 per thread: thread t holds digits
@@ -138,17 +195,44 @@ __global__ void __launch_bounds__(kThreads)
   const uint32_t T = prefix;
   const long long need_eq = krem;  // keys equal to T that are kept
 
-  // ---- ordered emission: warp w owns positions [w * chunk, (w + 1) * chunk)
-  const long long chunk = (L + 32 * kWarps - 1) / (32 * kWarps) * 32;
+  // ---- ordered emission: warp w owns positions [w * chunk, (w + 1) * chunk);
+  // a warp step covers 32 * V consecutive positions, lane l the V positions
+  // from V * l (so lane order is position order)
+  constexpr int V = kVec ? 4 : 1;
+  const long long chunk = (L + 32 * V * kWarps - 1) / (32 * V * kWarps) * (32 * V);
   const long long j0 = warp * chunk, j1 = min(L, j0 + chunk);
+  auto keys_at = [&](long long base, uint32_t (&k)[V]) {
+    const long long j = base + V * lane;
+    if (kVec) {
+      if (j < j1) {
+        const float4 v = load_key_value4(in, rbase + j);
+        k[0] = order_key(v.x);
+        k[V > 1 ? 1 : 0] = order_key(v.y);
+        k[V > 2 ? 2 : 0] = order_key(v.z);
+        k[V > 3 ? 3 : 0] = order_key(v.w);
+      } else {
+#pragma unroll
+        for (int u = 0; u < V; ++u) k[u] = 0u;
+      }
+    } else {
+      k[0] = j < j1 ? order_key(load_key_value(in, rbase + j)) : 0u;
+    }
+  };
   const uint32_t lt = (1u << lane) - 1u;
   uint32_t n_gt = 0, n_eq = 0;
-  for (long long base = j0; base < j1; base += 32) {
-    const long long j = base + lane;
-    const uint32_t key = j < j1 ? order_key(load_key_value(in, rbase + j)) : 0u;
-    n_gt += __popc(__ballot_sync(0xffffffffu, j < j1 && key > T));
-    n_eq += __popc(__ballot_sync(0xffffffffu, j < j1 && key == T));
+  for (long long base = j0; base < j1; base += 32 * V) {
+    uint32_t k[V];
+    keys_at(base, k);
+    const long long j = base + V * lane;
+#pragma unroll
+    for (int u = 0; u < V; ++u) {
+      const bool in_range = j + u < j1;
+      n_gt += (in_range && k[u] > T) ? 1u : 0u;
+      n_eq += (in_range && k[u] == T) ? 1u : 0u;
+    }
   }
+  n_gt = __reduce_add_sync(0xffffffffu, n_gt);
+  n_eq = __reduce_add_sync(0xffffffffu, n_eq);
   if (lane == 0) {
     wcnt[0][warp] = n_gt;
     wcnt[1][warp] = n_eq;
@@ -169,21 +253,41 @@ __global__ void __launch_bounds__(kThreads)
   }
   int32_t *out = idx + static_cast<size_t>(row) * static_cast<size_t>(K);
   long long run_eq = eq_off, run_out = out_off;
-  for (long long base = j0; base < j1; base += 32) {
-    const long long j = base + lane;
-    const uint32_t key = j < j1 ? order_key(load_key_value(in, rbase + j)) : 0u;
-    const bool gt = j < j1 && key > T;
-    const bool eq = j < j1 && key == T;
-    const uint32_t eb = __ballot_sync(0xffffffffu, eq);
-    const bool kept = gt || (eq && run_eq + __popc(eb & lt) < need_eq);
-    const uint32_t kb = __ballot_sync(0xffffffffu, kept);
-    if (kept) {
-      const long long pos = run_out + __popc(kb & lt);
-      if (pos < K) out[pos] = static_cast<int32_t>(j);
-      else record_device_status(BKV_DEV_ASSERT, 301);
+  for (long long base = j0; base < j1; base += 32 * V) {
+    uint32_t k[V];
+    keys_at(base, k);
+    const long long j = base + V * lane;
+    bool gt[V], eq[V];
+    uint32_t my_eq = 0;
+#pragma unroll
+    for (int u = 0; u < V; ++u) {
+      const bool in_range = j + u < j1;
+      gt[u] = in_range && k[u] > T;
+      eq[u] = in_range && k[u] == T;
+      my_eq += eq[u] ? 1u : 0u;
     }
-    run_eq += __popc(eb);
-    run_out += __popc(kb);
+    const uint32_t eq_incl = warp_inclusive_scan(my_eq, lane);
+    long long eq_rank = run_eq + eq_incl - my_eq;  // rank of this lane's first equal key
+    bool kept[V];
+    uint32_t my_kept = 0;
+#pragma unroll
+    for (int u = 0; u < V; ++u) {
+      kept[u] = gt[u] || (eq[u] && eq_rank < need_eq);
+      if (eq[u]) ++eq_rank;
+      my_kept += kept[u] ? 1u : 0u;
+    }
+    const uint32_t kept_incl = warp_inclusive_scan(my_kept, lane);
+    long long pos = run_out + kept_incl - my_kept;
+#pragma unroll
+    for (int u = 0; u < V; ++u) {
+      if (kept[u]) {
+        if (pos < K) out[pos] = static_cast<int32_t>(j + u);
+        else record_device_status(BKV_DEV_ASSERT, 301);
+        ++pos;
+      }
+    }
+    run_eq += __shfl_sync(0xffffffffu, eq_incl, 31);
+    run_out += __shfl_sync(0xffffffffu, kept_incl, 31);
   }
   if (tid == 0 && total_kept != K) record_device_status(BKV_DEV_ASSERT, 302);
 }
@@ -213,7 +317,14 @@ bkv_status launch_select_topk(const SelectInput &in, int n_rows, long long L, lo
                               int32_t *idx, float *s_out, void *, size_t, cudaStream_t stream) {
   if (injected_launch_failure()) return BKV_ERR_CUDA;
   if (n_rows <= 0) return BKV_OK;
-  select_topk_kernel<<<n_rows, kThreads, 0, stream>>>(in, L, K, idx, s_out);
+  // float4 passes when every row (and every part) starts on a 16-byte boundary
+  const bool vec = (L & 3) == 0 && (in.part_stride & 3) == 0 &&
+                   (reinterpret_cast<uintptr_t>(in.src) & 15u) == 0 &&
+                   (reinterpret_cast<uintptr_t>(s_out) & 15u) == 0;
+  if (vec)
+    select_topk_kernel<true><<<n_rows, kThreads, 0, stream>>>(in, L, K, idx, s_out);
+  else
+    select_topk_kernel<false><<<n_rows, kThreads, 0, stream>>>(in, L, K, idx, s_out);
   return cudaGetLastError() == cudaSuccess ? BKV_OK : BKV_ERR_CUDA;
 }
 

@@ -320,7 +320,7 @@ def test_full_size_sampled(name, dev):
     synth = _synth()
     wl = synth.WORKLOADS[name]
     inp = synth.make_step_inputs(wl, seed=0)
-    out, nb = _run_step(wl, inp, dev, aux=True)
+    out, nb = _run_step(wl, inp, dev)
     rng = np.random.default_rng(123)
     heads = sorted({(int(rng.integers(wl.n_layers)), int(rng.integers(wl.n_kv_heads)))
                     for _ in range(7)} | {(0, 0), (wl.n_layers - 1, wl.n_kv_heads - 1)})
@@ -342,7 +342,7 @@ def test_full_size_sampled_mean(dev):
     synth = _synth()
     wl = synth.WORKLOADS["qwen3_14b"]
     inp = synth.make_step_inputs(wl, seed=5)
-    out, nb = _run_step(wl, inp, dev, aggregate="mean", aux=True)
+    out, nb = _run_step(wl, inp, dev, aggregate="mean")
     rng = np.random.default_rng(321)
     heads = sorted({(int(rng.integers(wl.n_layers)), int(rng.integers(wl.n_kv_heads)))
                     for _ in range(2)} | {(0, 0)})
