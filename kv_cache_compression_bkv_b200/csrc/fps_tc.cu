@@ -73,11 +73,15 @@ constexpr int kCBlock = kCand * 128;              // one 64-element K block of t
 constexpr int kGramStride = kCand + 4;            // floats per Gram row (bank spread)
 constexpr int kListMax = 512;                     // threshold-bin keys ranked directly
 constexpr int kSwitch = 8;                        // picks that end the eager rounds
+constexpr int kAhead = 4;                         // tiles prefetched into L2 beyond the ring
 constexpr int kSmallBytes = 4096;
 constexpr int kFixedBytes = kSmallBytes + 1024 + kStages * kTileBytes + 2 * kPBlock;
 constexpr int kSmemLimit = 232448;
 // TMEM: two pass accumulators of up to 128 columns, the Gram and refresh blocks
 constexpr uint32_t kTmemCols = 512;
+// Pass accumulators (128 columns each): all of TMEM, since the Gram and
+// refresh blocks (columns 256 ..) are idle while a pass runs.
+constexpr int kAcc = 4;
 constexpr uint32_t kGramCol = 256, kRefCol = 384;
 // the serial phase's buffers inside the ring (idle between passes)
 constexpr int kGramOff = 0;                        // [kCand][kGramStride] f32
@@ -108,10 +112,10 @@ enum {
 
 enum { kWhereProd = 401, kWhereMma = 402, kWhereEpi = 403, kWhereDrain = 404 };
 
-// Barriers: full[4] empty[4] tfull[2] tempty[2], the two MMA threads' drain
+// Barriers: full[4] empty[4] tfull[4] tempty[4], the two MMA threads' drain
 // barriers, the round's Gram/refresh commit.
-constexpr int kBarFull = 0, kBarEmpty = 4, kBarTfull = 8, kBarTempty = 10, kBarDone = 12,
-              kBarGram = 14;
+constexpr int kBarFull = 0, kBarEmpty = 4, kBarTfull = 8, kBarTempty = 12, kBarDone = 16,
+              kBarGram = 18;
 
 struct Layout {
   uint64_t *bars;
@@ -177,16 +181,30 @@ __device__ bool issue_tiles(const Layout &s, const CUtensorMap *bmap, const CUte
                             int qh, const FpsGeom &g, int n_btiles, int w_first, uint32_t seq,
                             int n_tiles) {
   const uint32_t full0 = smem_u32(&s.bars[kBarFull]), empty0 = smem_u32(&s.bars[kBarEmpty]);
+  auto map_of = [&](int j) { return j < n_btiles ? bmap : wmap; };
+  auto row_of = [&](int j) {
+    return j < n_btiles ? qh * g.M + j * kTileRows
+                        : static_cast<int>(qh * g.w_cap) + (w_first + j - n_btiles) * kTileRows;
+  };
+  // Tiles past the ring's depth are prefetched into L2 kAhead tiles before
+  // their stage frees, so that their loads are L2 hits: the ring holds
+  // kStages tiles, and a load from HBM takes about as long as kStages tiles'
+  // MMAs and epilogues.
+  auto prefetch = [&](int j) {
+    tma_prefetch_2d(map_of(j), 0, row_of(j));
+    tma_prefetch_2d(map_of(j), 64, row_of(j));
+  };
+  for (int j = kStages; j < min(n_tiles, kStages + kAhead); ++j) prefetch(j);
   for (int j = 0; j < n_tiles; ++j) {
     const uint32_t q = seq + j, st = q % kStages;
     if (!mbar_wait(empty0 + 8 * st, ((q / kStages) & 1) ^ 1, kWhereProd)) return false;
     mbar_arrive_expect_tx(full0 + 8 * st, kTileBytes);
     const uint32_t dst = smem_u32(s.ring + st * kTileBytes);
-    const CUtensorMap *map = j < n_btiles ? bmap : wmap;
-    const int y = j < n_btiles ? qh * g.M + j * kTileRows
-                               : static_cast<int>(qh * g.w_cap) + (w_first + j - n_btiles) * kTileRows;
+    const CUtensorMap *map = map_of(j);
+    const int y = row_of(j);
     tma_load_2d(dst, map, full0 + 8 * st, 0, y);
     tma_load_2d(dst + kTileRows * 128, map, full0 + 8 * st, 64, y);
+    if (j + kStages + kAhead < n_tiles) prefetch(j + kStages + kAhead);
   }
   return true;
 }
@@ -229,24 +247,29 @@ __device__ void distance_pass(const Layout &s, const CUtensorMap *bmap, const CU
   } else if (warp == 1 || warp == 2) {
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(kTileRows, N);
-      const uint32_t b_base = smem_u32(s.pop) + static_cast<uint32_t>(s0) * 128u;
-      const uint32_t mine = static_cast<uint32_t>(warp - 1);
+      // descriptors of the K steps: the start-address field (address / 16,
+      // 14 bits) is the only part that moves, and shared addresses stay
+      // below 256 KB, so an offset is added to it directly
+      const uint64_t b_desc =
+          smem_desc_k_sw128(smem_u32(s.pop) + static_cast<uint32_t>(s0) * 128u);
+      const uint64_t a_desc0 = smem_desc_k_sw128(smem_u32(s.ring));
+      const uint32_t mine = static_cast<uint32_t>(warp - 1);  // accumulators mine, mine + 2
       for (int j = 0; j < n_tiles; ++j) {
-        const uint32_t q = seq + j, st = q % kStages, a = q & 1;
-        if (a != mine) continue;
+        const uint32_t q = seq + j, st = q % kStages, a = q % kAcc;
+        if ((a & 1u) != mine) continue;
         if (!mbar_wait(full0 + 8 * st, (q / kStages) & 1, kWhereMma) ||
-            !mbar_wait(tempty0 + 8 * a, ((q >> 1) & 1) ^ 1, kWhereMma)) {
+            !mbar_wait(tempty0 + 8 * a, ((q / kAcc) & 1) ^ 1, kWhereMma)) {
           s.scal[kAbort] = 1;
           break;
         }
         tc_fence_after();
-        const uint32_t a_base = smem_u32(s.ring + st * kTileBytes);
+        const uint64_t a_desc = a_desc0 + ((st * kTileBytes) >> 4);
 #pragma unroll
         for (int kb = 0; kb < 2; ++kb) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = smem_desc_k_sw128(a_base + kb * (kTileRows * 128) + kk * 32);
-            const uint64_t bd = smem_desc_k_sw128(b_base + kb * kPBlock + kk * 32);
+            const uint64_t ad = a_desc + ((kb * (kTileRows * 128) + kk * 32) >> 4);
+            const uint64_t bd = b_desc + ((kb * kPBlock + kk * 32) >> 4);
             umma_f16(tmem + a * 128, ad, bd, idesc, (kb | kk) != 0);
           }
         }
@@ -257,14 +280,15 @@ __device__ void distance_pass(const Layout &s, const CUtensorMap *bmap, const CU
       }
     }
   } else if (warp >= 4) {
-    // epilogue warpgroup w consumes accumulator w, i.e. every other tile
+    // epilogue warpgroup w consumes accumulators w and w + 2, i.e. every
+    // other tile
     const int wg = (warp - 4) >> 2;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     bool ok = true;  // warp-uniform; after a timeout the warp keeps only the barriers
     for (int j = 0; j < n_tiles; ++j) {
-      const uint32_t q = seq + j, a = q & 1;
-      if (static_cast<int>(a) != wg) continue;
+      const uint32_t q = seq + j, a = q % kAcc;
+      if (static_cast<int>(a & 1u) != wg) continue;
       int i;
       bool valid;
       if (j < n_btiles) {
@@ -280,7 +304,7 @@ __device__ void distance_pass(const Layout &s, const CUtensorMap *bmap, const CU
         i = valid ? g.nb_in + static_cast<int>(w) : 0;
       }
       const uint32_t st = q % kStages;
-      if (ok && !mbar_wait_warp(tfull0 + 8 * a, (q >> 1) & 1, kWhereEpi)) {
+      if (ok && !mbar_wait_warp(tfull0 + 8 * a, (q / kAcc) & 1, kWhereEpi)) {
         s.scal[kAbort] = 1;
         ok = false;
       }
@@ -524,13 +548,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int m = g.n_pick;
   Layout s;
   s.bars = reinterpret_cast<uint64_t *>(smem_raw);
-  s.tmem_slot = reinterpret_cast<uint32_t *>(smem_raw + 128);
-  s.scal = reinterpret_cast<int *>(smem_raw + 192);
-  s.hist = reinterpret_cast<uint32_t *>(smem_raw + 320);
-  s.cidx = reinterpret_cast<int *>(smem_raw + 1344);
-  s.cdist = reinterpret_cast<float *>(smem_raw + 1872);
-  s.pick = reinterpret_cast<int *>(smem_raw + 2400);
-  s.pinv = reinterpret_cast<float *>(smem_raw + 2912);   // .. 3488
+  s.tmem_slot = reinterpret_cast<uint32_t *>(smem_raw + 192);  // bars: 24 slots
+  s.scal = reinterpret_cast<int *>(smem_raw + 256);
+  s.hist = reinterpret_cast<uint32_t *>(smem_raw + 384);
+  s.cidx = reinterpret_cast<int *>(smem_raw + 1408);
+  s.cdist = reinterpret_cast<float *>(smem_raw + 1936);
+  s.pick = reinterpret_cast<int *>(smem_raw + 2464);
+  s.pinv = reinterpret_cast<float *>(smem_raw + 2976);   // .. 3552
   const uint32_t raw_base = smem_u32(smem_raw);
   const uint32_t big = (raw_base + kSmallBytes + 1023u) & ~1023u;
   s.ring = smem_raw + (big - raw_base);
@@ -557,11 +581,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&s.bars[kBarFull + i]), 1);
       mbar_init(smem_u32(&s.bars[kBarEmpty + i]), 1);  // the MMA's commit (seed pass: the epilogue)
     }
-    for (int a = 0; a < 2; ++a) {
+    for (int a = 0; a < kAcc; ++a) {
       mbar_init(smem_u32(&s.bars[kBarTfull + a]), 1);
       mbar_init(smem_u32(&s.bars[kBarTempty + a]), 4);  // one arrive per warp of its warpgroup
-      mbar_init(smem_u32(&s.bars[kBarDone + a]), 1);
     }
+    for (int a = 0; a < 2; ++a) mbar_init(smem_u32(&s.bars[kBarDone + a]), 1);
     mbar_init(smem_u32(&s.bars[kBarGram]), 1);  // the round's Gram/refresh MMAs
     fence_barrier_init();
     prefetch_tensormap(&bmap);

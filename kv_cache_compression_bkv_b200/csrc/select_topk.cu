@@ -1,23 +1,34 @@
 // select_topk.cu -- top-K budget selection (BeaconKV Fig. 5(c); Table 1's
 // "maximum KV cache budget").
 //
-// One CTA of 512 threads per row, all rows resident at once (a few CTAs per
-// SM, ~8 KB of shared memory each).  Scores become order-preserving unsigned
-// keys (larger score -> larger key; -0 and +0 map to one key).  The row is
-// never staged: every pass re-reads it (from L2 after the first) and rebuilds
-// the keys, which for the step's max form also merges the observation
-// groups' partial maxima.  Three MSB-first radix passes with 11-, 11- and
-// 10-bit digits (one shared histogram, block-wide scan of its bins) find the
-// K-th largest key T and how many keys equal to T are kept; two more passes
-// write the kept positions in ascending order: each warp owns a contiguous
-// slice of the row, counts its keys above T and equal to T, the warps' slices
-// are placed by a prefix sum, and each warp then emits its kept positions in
-// order with ballots -- every key > T, plus the first `need_eq` keys equal to
-// T (ties go to the lower position).
+// One CTA per row (a (layer, KV head)); scores become order-preserving
+// unsigned keys (larger score -> larger key; -0 and +0 map to one key).  The
+// row is never staged whole: each pass re-reads it (from HBM the first time,
+// L2 after) and rebuilds the keys -- for the step's max form that also
+// merges the observation groups' partial maxima.
+//
+// The common path (rows of a multiple of 4 keys, 16-byte aligned, at most
+// 65536 of them) reads the row twice and does the rest in shared memory:
+//   1. (HBM) a histogram of the keys' top 12 bits finds the bin holding the
+//      K-th largest key (and the step's scores are written);
+//   2. (L2) every key above that bin is certainly kept: it is marked in a
+//      bitmask of the row's positions (each 8 lanes of a warp assemble one
+//      32-position word with three shuffles); the keys of the bin itself are
+//      collected, with their positions, in a list;
+//   3. a radix select over the listed keys' low 20 bits finds the K-th largest
+//      key T and how many keys equal to T are kept; listed keys above T are
+//      marked, and the first `need_eq` keys equal to T (ties to the lower
+//      position: a prefix count over a second bitmask) too;
+//   4. the marked positions are written in ascending order, each thread
+//      taking a run of mask words at its prefix-sum offset.
+// A row whose threshold bin holds more keys than the list can take (scores
+// piled into a narrow range), longer rows, and rows not laid out for 16-byte
+// loads take the general path: MSB-first radix passes over the streamed row
+// for the remaining bits, then a counting pass and a writing pass in which
+// each warp emits the kept positions of its slice of the row.
 #include <cuda_runtime.h>
 
 #include <algorithm>
-#include <mutex>
 
 #include "bkv_device_status.cuh"
 #include "bkv_internal.h"
@@ -27,14 +38,23 @@ BKV_DEFINE_STATUS_ACCESSOR(take_status_select)
 namespace bkv {
 namespace {
 
-constexpr int kThreads = 512;
+constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kMaxBins = 2048;  // 11-bit digits
+constexpr int kTopBits = 12;                 // the first pass's digit
+constexpr int kTopBins = 1 << kTopBits;      // 4096
+constexpr int kListCap = 6144;               // threshold-bin keys held in shared memory
+constexpr int kMaskMaxL = 65536;             // longest row whose bitmasks are held
+// histogram (4096 words) + list keys and positions + two bitmasks of L bits
+constexpr int mask_smem_bytes(long long L) {
+  return static_cast<int>((kTopBins + 2 * kListCap + 2 * ((L + 127) / 128 * 4)) * 4);
+}
 
 __device__ __forceinline__ uint32_t order_key(float f) {
-  if (f == 0.f) f = 0.f;  // -0 -> +0
-  const uint32_t u = __float_as_uint(f);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  // f + 0 is +0 for f = -0 (round to nearest) and f otherwise; then the
+  // sign's arithmetic shift flips all bits of a negative and only the sign
+  // bit of a positive
+  const uint32_t u = __float_as_uint(f + 0.f);
+  return u ^ (static_cast<uint32_t>(static_cast<int32_t>(u) >> 31) | 0x80000000u);
 }
 
 __device__ __forceinline__ float load_key_value(const SelectInput &in, size_t off) {
@@ -49,7 +69,29 @@ __device__ __forceinline__ float load_key_value(const SelectInput &in, size_t of
 
 // The score a key stands for: the max form keeps log-domain maxima.
 __device__ __forceinline__ float score_of_key(const SelectInput &in, float v) {
-  return in.mean ? v : expf(v);
+  return in.mean ? v : __expf(v);
+}
+
+// Four consecutive values of a row (off a multiple of 4, the row 16-byte
+// aligned), merged over the parts like load_key_value.
+__device__ __forceinline__ float4 load_key_value4(const SelectInput &in, size_t off) {
+  float4 v = *reinterpret_cast<const float4 *>(in.src + off);
+  for (int p = 1; p < in.n_parts; ++p) {
+    const float4 w = *reinterpret_cast<const float4 *>(in.src + p * in.part_stride + off);
+    if (in.mean) {
+      v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
+    } else {
+      v.x = fmaxf(v.x, w.x); v.y = fmaxf(v.y, w.y); v.z = fmaxf(v.z, w.z); v.w = fmaxf(v.w, w.w);
+    }
+  }
+  if (in.mean) {
+    v.x *= in.inv_count; v.y *= in.inv_count; v.z *= in.inv_count; v.w *= in.inv_count;
+  }
+  return v;
+}
+
+__device__ __forceinline__ uint4 keys_of(float4 v) {
+  return make_uint4(order_key(v.x), order_key(v.y), order_key(v.z), order_key(v.w));
 }
 
 // Exclusive prefix sum over the block of one value per thread; returns the
@@ -77,24 +119,6 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t *w
   return wpre + incl - v;
 }
 
-// Four consecutive values of a row (off a multiple of 4, the row 16-byte
-// aligned), merged over the parts like load_key_value.
-__device__ __forceinline__ float4 load_key_value4(const SelectInput &in, size_t off) {
-  float4 v = *reinterpret_cast<const float4 *>(in.src + off);
-  for (int p = 1; p < in.n_parts; ++p) {
-    const float4 w = *reinterpret_cast<const float4 *>(in.src + p * in.part_stride + off);
-    if (in.mean) {
-      v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
-    } else {
-      v.x = fmaxf(v.x, w.x); v.y = fmaxf(v.y, w.y); v.z = fmaxf(v.z, w.z); v.w = fmaxf(v.w, w.w);
-    }
-  }
-  if (in.mean) {
-    v.x *= in.inv_count; v.y *= in.inv_count; v.z *= in.inv_count; v.w *= in.inv_count;
-  }
-  return v;
-}
-
 // Inclusive prefix sum across the warp.
 __device__ __forceinline__ uint32_t warp_inclusive_scan(uint32_t v, int lane) {
 #pragma unroll
@@ -105,145 +129,53 @@ __device__ __forceinline__ uint32_t warp_inclusive_scan(uint32_t v, int lane) {
   return v;
 }
 
-// kVec: the row length is a multiple of 4 and rows are 16-byte aligned, so
-// every pass reads float4s (four keys per thread and load).
-template <bool kVec>
-__global__ void __launch_bounds__(kThreads)
-    select_topk_kernel(const SelectInput in, long long L, long long K, int32_t *__restrict__ idx,
-                       float *__restrict__ s_out) {
-  __shared__ uint32_t hist[kMaxBins];
-  __shared__ uint32_t wsum[kWarps];
-  __shared__ uint32_t wcnt[2][kWarps];
-  __shared__ long long sel[2];
-  const int row = blockIdx.x;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const size_t rbase = static_cast<size_t>(row) * static_cast<size_t>(L);
-
-  // ---- radix select of the K-th largest key: bits [lo, hi) per pass
-  uint32_t prefix = 0, mask = 0;
-  long long krem = K;  // rank of the wanted key among those matching the prefix
-  for (int hi = 32; hi > 0;) {
-    const int lo = hi > 11 ? hi - 11 : 0;
-    const int nbits = hi - lo;
-    const uint32_t dmask = (1u << nbits) - 1u;
-    const int nb = 1 << nbits;
-    for (int b = tid; b < nb; b += kThreads) hist[b] = 0u;
-    __syncthreads();
-    auto count = [&](uint32_t key) {
-      if ((key & mask) == prefix) atomicAdd(&hist[(key >> lo) & dmask], 1u);
-    };
-    if (kVec) {
-      // two float4 loads in flight per thread before their keys are counted
-      const long long L4 = L >> 2;
-      for (long long q = tid; q < L4; q += 2 * kThreads) {
-        const long long q2 = q + kThreads;
-        const float4 a = load_key_value4(in, rbase + 4 * q);
-        float4 b = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (q2 < L4) b = load_key_value4(in, rbase + 4 * q2);
-        if (hi == 32 && s_out) {
-          *reinterpret_cast<float4 *>(s_out + rbase + 4 * q) =
-              make_float4(score_of_key(in, a.x), score_of_key(in, a.y), score_of_key(in, a.z),
-                          score_of_key(in, a.w));
-          if (q2 < L4)
-            *reinterpret_cast<float4 *>(s_out + rbase + 4 * q2) =
-                make_float4(score_of_key(in, b.x), score_of_key(in, b.y), score_of_key(in, b.z),
-                            score_of_key(in, b.w));
-        }
-        count(order_key(a.x)); count(order_key(a.y)); count(order_key(a.z)); count(order_key(a.w));
-        if (q2 < L4) {
-          count(order_key(b.x)); count(order_key(b.y)); count(order_key(b.z)); count(order_key(b.w));
-        }
-      }
-    } else {
-      for (long long j = tid; j < L; j += kThreads) {
-        const float v = load_key_value(in, rbase + j);
-        if (hi == 32 && s_out) s_out[rbase + j] = score_of_key(in, v);
-        count(order_key(v));
-      }
-    }
-    __syncthreads();
-    // bins in descending digit order, 4 per thread: thread t holds digits
-    // nb-1-4t .. nb-4-4t
-    uint32_t c4[4], local = 0;
+// The digit of `hist` (nb bins, highest digit first, nb / kThreads per
+// thread) holding the krem-th key: sel[0] = the digit, sel[1] = the keys in
+// higher digits.  Every thread calls it; it synchronises.
+template <int kPer>
+__device__ __forceinline__ void find_digit(const uint32_t *hist, int nb, long long krem,
+                                           uint32_t *wsum, long long *sel) {
+  const int tid = threadIdx.x;
+  uint32_t c[kPer], local = 0;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int d = nb - 1 - 4 * tid - q;
-      c4[q] = d >= 0 ? hist[d] : 0u;
-      local += c4[q];
-    }
-    uint32_t total;
-    const uint32_t excl = block_exclusive_scan(local, wsum, &total);
-    if (static_cast<long long>(excl) < krem && krem <= static_cast<long long>(excl + local)) {
-      uint32_t acc = excl;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        if (static_cast<long long>(acc + c4[q]) >= krem) {
-          sel[0] = nb - 1 - 4 * tid - q;
-          sel[1] = acc;
-          break;
-        }
-        acc += c4[q];
-      }
-    }
-    __syncthreads();
-    prefix |= static_cast<uint32_t>(sel[0]) << lo;
-    mask |= dmask << lo;
-    krem -= sel[1];
-    hi = lo;
-    __syncthreads();  // sel and hist are rewritten by the next pass
+  for (int q = 0; q < kPer; ++q) {
+    const int d = nb - 1 - kPer * tid - q;
+    c[q] = d >= 0 ? hist[d] : 0u;
+    local += c[q];
   }
-  const uint32_t T = prefix;
-  const long long need_eq = krem;  // keys equal to T that are kept
-
-  // ---- ordered emission: warp w owns positions [w * chunk, (w + 1) * chunk);
-  // a warp step covers 32 * V consecutive positions, lane l the V positions
-  // from V * l (so lane order is position order)
-  constexpr int V = kVec ? 4 : 1;
-  const long long chunk = (L + 32 * V * kWarps - 1) / (32 * V * kWarps) * (32 * V);
-  const long long j0 = warp * chunk, j1 = min(L, j0 + chunk);
-  auto keys_at = [&](long long base, uint32_t (&k)[V]) {
-    const long long j = base + V * lane;
-    if (kVec) {
-      if (j < j1) {
-        const float4 v = load_key_value4(in, rbase + j);
-        k[0] = order_key(v.x);
-        k[V > 1 ? 1 : 0] = order_key(v.y);
-        k[V > 2 ? 2 : 0] = order_key(v.z);
-        k[V > 3 ? 3 : 0] = order_key(v.w);
-      } else {
+  uint32_t total;
+  const uint32_t excl = block_exclusive_scan(local, wsum, &total);
+  if (static_cast<long long>(excl) < krem && krem <= static_cast<long long>(excl + local)) {
+    uint32_t acc = excl;
 #pragma unroll
-        for (int u = 0; u < V; ++u) k[u] = 0u;
+    for (int q = 0; q < kPer; ++q) {
+      if (static_cast<long long>(acc + c[q]) >= krem) {
+        sel[0] = nb - 1 - kPer * tid - q;
+        sel[1] = acc;
+        break;
       }
-    } else {
-      k[0] = j < j1 ? order_key(load_key_value(in, rbase + j)) : 0u;
+      acc += c[q];
     }
-  };
-  const uint32_t lt = (1u << lane) - 1u;
-  uint32_t n_gt = 0, n_eq = 0;
-  for (long long base = j0; base < j1; base += 32 * V) {
-    uint32_t k[V];
-    keys_at(base, k);
-    const long long j = base + V * lane;
-#pragma unroll
-    for (int u = 0; u < V; ++u) {
-      const bool in_range = j + u < j1;
-      n_gt += (in_range && k[u] > T) ? 1u : 0u;
-      n_eq += (in_range && k[u] == T) ? 1u : 0u;
-    }
-  }
-  n_gt = __reduce_add_sync(0xffffffffu, n_gt);
-  n_eq = __reduce_add_sync(0xffffffffu, n_eq);
-  if (lane == 0) {
-    wcnt[0][warp] = n_gt;
-    wcnt[1][warp] = n_eq;
   }
   __syncthreads();
-  // eq_off: equal keys in the warps before this one (the rank of this warp's
-  // first equal key); out_off: keys those warps keep (this warp's first slot)
+}
+
+// Ordered emission of row `row`'s kept positions given the threshold key T:
+// warp w owns positions [w * chunk, (w + 1) * chunk); cnt_gt[w] / cnt_eq[w]
+// (shared) hold the keys > T and == T of each slice.  Writes idx[row][..].
+template <bool kVec>
+__device__ void emit_kept(const SelectInput &in, long long L, long long K, int32_t *idx,
+                          size_t rbase, int row, uint32_t T, long long need_eq, long long chunk,
+                          const uint32_t *cnt_gt, const uint32_t *cnt_eq) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  constexpr int V = kVec ? 4 : 1;
+  const long long j0 = warp * chunk, j1 = min(L, j0 + chunk);
+  // eq_off: equal keys in the slices before this one (the rank of this
+  // slice's first equal key); out_off: keys those slices keep
   long long eq_off = 0, out_off = 0, total_kept = 0, eo = 0;
   for (int w = 0; w < kWarps; ++w) {
-    const long long e = wcnt[1][w];
-    const long long k = wcnt[0][w] + max(0LL, min(e, need_eq - eo));
+    const long long e = cnt_eq[w];
+    const long long k = cnt_gt[w] + max(0LL, min(e, need_eq - eo));
     if (w < warp) {
       eq_off += e;
       out_off += k;
@@ -255,8 +187,16 @@ __global__ void __launch_bounds__(kThreads)
   long long run_eq = eq_off, run_out = out_off;
   for (long long base = j0; base < j1; base += 32 * V) {
     uint32_t k[V];
-    keys_at(base, k);
     const long long j = base + V * lane;
+    if constexpr (kVec) {
+      const uint4 kk = j < j1 ? keys_of(load_key_value4(in, rbase + j)) : make_uint4(0u, 0u, 0u, 0u);
+      k[0] = kk.x;
+      k[1] = kk.y;
+      k[2] = kk.z;
+      k[3] = kk.w;
+    } else {
+      k[0] = j < j1 ? order_key(load_key_value(in, rbase + j)) : 0u;
+    }
     bool gt[V], eq[V];
     uint32_t my_eq = 0;
 #pragma unroll
@@ -292,6 +232,312 @@ __global__ void __launch_bounds__(kThreads)
   if (tid == 0 && total_kept != K) record_device_status(BKV_DEV_ASSERT, 302);
 }
 
+// The general path from a known prefix: MSB-first radix passes over the
+// streamed row for bits [0, hi) (11 bits at a time) with the keys matching
+// `prefix` under `mask`, then a counting pass and the ordered emission.
+// s_out is written by the first pass when hi == 32.
+template <bool kVec>
+__device__ void stream_select(const SelectInput &in, long long L, long long K, int32_t *idx,
+                              float *s_out, int row, uint32_t prefix, uint32_t mask,
+                              long long krem, int hi, uint32_t *hist, uint32_t *wsum,
+                              long long *sel, uint32_t *cnt_gt, uint32_t *cnt_eq) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const size_t rbase = static_cast<size_t>(row) * static_cast<size_t>(L);
+  while (hi > 0) {
+    const int lo = hi > 11 ? hi - 11 : 0;
+    const int nbits = hi - lo;
+    const uint32_t dmask = (1u << nbits) - 1u;
+    const int nb = 1 << nbits;
+    for (int b = tid; b < nb; b += kThreads) hist[b] = 0u;
+    __syncthreads();
+    auto count = [&](uint32_t key) {
+      if ((key & mask) == prefix) atomicAdd(&hist[(key >> lo) & dmask], 1u);
+    };
+    if constexpr (kVec) {
+      const long long L4 = L >> 2;
+      for (long long q = tid; q < L4; q += kThreads) {
+        const float4 a = load_key_value4(in, rbase + 4 * q);
+        if (hi == 32 && s_out)
+          *reinterpret_cast<float4 *>(s_out + rbase + 4 * q) =
+              make_float4(score_of_key(in, a.x), score_of_key(in, a.y), score_of_key(in, a.z),
+                          score_of_key(in, a.w));
+        const uint4 k = keys_of(a);
+        count(k.x); count(k.y); count(k.z); count(k.w);
+      }
+    } else {
+      for (long long j = tid; j < L; j += kThreads) {
+        const float v = load_key_value(in, rbase + j);
+        if (hi == 32 && s_out) s_out[rbase + j] = score_of_key(in, v);
+        count(order_key(v));
+      }
+    }
+    __syncthreads();
+    find_digit<(1 << 11) / kThreads>(hist, nb, krem, wsum, sel);
+    prefix |= static_cast<uint32_t>(sel[0]) << lo;
+    mask |= dmask << lo;
+    krem -= sel[1];
+    hi = lo;
+    __syncthreads();  // sel and hist are rewritten by the next pass
+  }
+  const uint32_t T = prefix;
+  const long long need_eq = krem;  // keys equal to T that are kept
+  constexpr int V = kVec ? 4 : 1;
+  const long long chunk = (L + 32 * V * kWarps - 1) / (32 * V * kWarps) * (32 * V);
+  const long long j0 = warp * chunk, j1 = min(L, j0 + chunk);
+  uint32_t n_gt = 0, n_eq = 0;
+  for (long long base = j0; base < j1; base += 32 * V) {
+    const long long j = base + V * lane;
+    if constexpr (kVec) {
+      if (j < j1) {
+        const uint4 k = keys_of(load_key_value4(in, rbase + j));
+        n_gt += (k.x > T) + (k.y > T) + (k.z > T) + (k.w > T);
+        n_eq += (k.x == T) + (k.y == T) + (k.z == T) + (k.w == T);
+      }
+    } else if (j < j1) {
+      const uint32_t k = order_key(load_key_value(in, rbase + j));
+      n_gt += k > T;
+      n_eq += k == T;
+    }
+  }
+  n_gt = __reduce_add_sync(0xffffffffu, n_gt);
+  n_eq = __reduce_add_sync(0xffffffffu, n_eq);
+  if (lane == 0) {
+    cnt_gt[warp] = n_gt;
+    cnt_eq[warp] = n_eq;
+  }
+  __syncthreads();
+  emit_kept<kVec>(in, L, K, idx, rbase, row, T, need_eq, chunk, cnt_gt, cnt_eq);
+}
+
+// The general path for a whole row.
+template <bool kVec>
+__global__ void __launch_bounds__(kThreads)
+    select_topk_kernel(const SelectInput in, long long L, long long K, int32_t *__restrict__ idx,
+                       float *__restrict__ s_out) {
+  __shared__ uint32_t hist[1 << 11];
+  __shared__ uint32_t wsum[kWarps];
+  __shared__ uint32_t cnt[2][kWarps];
+  __shared__ long long sel[2];
+  stream_select<kVec>(in, L, K, idx, s_out, blockIdx.x, 0u, 0u, K, 32, hist, wsum, sel, cnt[0],
+                      cnt[1]);
+}
+
+// Four consecutive merged values at p (16-byte aligned), with the part count
+// fixed at compile time (kP > 0) or read from the input (kP == 0).
+template <int kP, bool kMean>
+__device__ __forceinline__ float4 merged4(const SelectInput &in, const float *p) {
+  float4 v = *reinterpret_cast<const float4 *>(p);
+  const int np = kP > 0 ? kP : in.n_parts;
+#pragma unroll
+  for (int q = 1; q < (kP > 0 ? kP : 64); ++q) {
+    if (kP == 0 && q >= np) break;
+    const float4 w = *reinterpret_cast<const float4 *>(p + q * in.part_stride);
+    if constexpr (kMean) {
+      v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
+    } else {
+      v.x = fmaxf(v.x, w.x); v.y = fmaxf(v.y, w.y); v.z = fmaxf(v.z, w.z); v.w = fmaxf(v.w, w.w);
+    }
+  }
+  if constexpr (kMean) {
+    v.x *= in.inv_count; v.y *= in.inv_count; v.z *= in.inv_count; v.w *= in.inv_count;
+  }
+  return v;
+}
+
+// The common path: two streaming passes, then shared memory only (see the
+// file comment).  Shared memory: the histogram, the threshold bin's list, and
+// two bitmasks of the row's positions (kept; equal to T).
+template <int kP, bool kMean>
+__global__ void __launch_bounds__(kThreads, 3)
+    select_topk_mask_kernel(const SelectInput in, int L, int K, int32_t *__restrict__ idx,
+                            float *__restrict__ s_out) {
+  extern __shared__ uint32_t sm[];
+  const int n_words = (L + 127) / 128 * 4;  // mask words, whole 128-position groups
+  uint32_t *hist = sm;                      // [kTopBins]
+  uint32_t *lkey = hist + kTopBins;         // [kListCap]
+  uint32_t *lpos = lkey + kListCap;         // [kListCap]
+  uint32_t *mask = lpos + kListCap;         // [n_words] kept positions
+  uint32_t *eqm = mask + n_words;           // [n_words] positions of keys equal to T
+  __shared__ uint32_t wsum[kWarps];
+  __shared__ long long sel[2];
+  __shared__ int n_list;
+  const int row = blockIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const float *src = in.src + static_cast<size_t>(row) * static_cast<size_t>(L);
+  float *so = s_out ? s_out + static_cast<size_t>(row) * static_cast<size_t>(L) : nullptr;
+  const int L4 = L >> 2;
+  constexpr int U = 4;  // float4 loads in flight per thread
+
+  for (int b = tid; b < kTopBins; b += kThreads) hist[b] = 0u;
+  for (int w = tid; w < 2 * n_words; w += kThreads) mask[w] = 0u;  // mask and eqm
+  if (tid == 0) n_list = 0;
+  __syncthreads();
+
+  // ---- pass 1 (HBM): histogram of the top 12 bits, and the scores
+  for (int q0 = tid; q0 < L4; q0 += U * kThreads) {
+    float4 a[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      if (q0 + u * kThreads < L4) a[u] = merged4<kP, kMean>(in, src + 4 * (q0 + u * kThreads));
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int q = q0 + u * kThreads;
+      if (q < L4) {
+        if (so) {
+          const float4 v = a[u];
+          *reinterpret_cast<float4 *>(so + 4 * q) =
+              kMean ? v : make_float4(__expf(v.x), __expf(v.y), __expf(v.z), __expf(v.w));
+        }
+        const uint4 k = keys_of(a[u]);
+        atomicAdd(&hist[k.x >> (32 - kTopBits)], 1u);
+        atomicAdd(&hist[k.y >> (32 - kTopBits)], 1u);
+        atomicAdd(&hist[k.z >> (32 - kTopBits)], 1u);
+        atomicAdd(&hist[k.w >> (32 - kTopBits)], 1u);
+      }
+    }
+  }
+  __syncthreads();
+  find_digit<kTopBins / kThreads>(hist, kTopBins, K, wsum, sel);
+  const uint32_t b1 = static_cast<uint32_t>(sel[0]);
+  const long long need1 = K - sel[1];
+  const uint32_t in_bin = hist[b1];
+  __syncthreads();
+  if (in_bin > static_cast<uint32_t>(kListCap)) {
+    // scores piled into one bin: the general path for the remaining bits
+    stream_select<true>(in, L, K, idx, nullptr, row, b1 << (32 - kTopBits),
+                        0xffffffffu << (32 - kTopBits), need1, 32 - kTopBits, hist, wsum, sel,
+                        lkey, lkey + kWarps);
+    return;
+  }
+
+  const uint32_t key_lo = b1 << (32 - kTopBits);
+  const uint32_t key_top = key_lo | ((1u << (32 - kTopBits)) - 1u);  // the bin's largest key
+  // ---- pass 2 (L2): keys above the bin -> mask bits; the bin's keys -> list.
+  // Lane l of a warp holds positions 4q .. 4q+3 with q = base + l, so lanes
+  // 8m .. 8m+7 cover one 32-position mask word; base is warp-uniform.
+  for (int base = warp * 32; base < L4; base += U * kThreads) {
+    float4 a[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int q = base + u * kThreads + lane;
+      if (q < L4) a[u] = merged4<kP, kMean>(in, src + 4 * q);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int q = base + u * kThreads + lane;
+      uint32_t nib = 0u;
+      uint32_t k[4] = {0u, 0u, 0u, 0u};
+      bool in_bin_any = false;
+      if (q < L4) {
+        const uint4 k4 = keys_of(a[u]);
+        k[0] = k4.x; k[1] = k4.y; k[2] = k4.z; k[3] = k4.w;
+        // above the bin: key > key_top; in it: key - key_lo < bin width
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          nib |= (k[e] > key_top ? 1u : 0u) << e;
+          in_bin_any |= k[e] - key_lo < (1u << (32 - kTopBits));
+        }
+      }
+      if (__any_sync(0xffffffffu, in_bin_any)) {  // about 2% of keys: rare per warp step
+        if (in_bin_any) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            if (k[e] - key_lo < (1u << (32 - kTopBits))) {
+              const int p = atomicAdd(&n_list, 1);
+              if (p < kListCap) {
+                lkey[p] = k[e];
+                lpos[p] = static_cast<uint32_t>(4 * q + e);
+              }
+            }
+          }
+        }
+      }
+      uint32_t word = nib << (4 * (lane & 7));
+      word |= __shfl_xor_sync(0xffffffffu, word, 1);
+      word |= __shfl_xor_sync(0xffffffffu, word, 2);
+      word |= __shfl_xor_sync(0xffffffffu, word, 4);
+      const int wi = (base + u * kThreads + lane) >> 3;
+      if ((lane & 7) == 0 && wi < n_words) mask[wi] = word;
+    }
+  }
+  __syncthreads();
+  const int listed = min(n_list, kListCap);
+
+  // ---- the K-th key within the collected bin: bits 19..0 in two 10-bit
+  // digits over the list
+  uint32_t prefix = b1 << (32 - kTopBits), pmask = 0xffffffffu << (32 - kTopBits);
+  long long krem = need1;
+  for (int hi = 32 - kTopBits; hi > 0;) {
+    const int lo = hi > 10 ? hi - 10 : 0;
+    const uint32_t dmask = (1u << (hi - lo)) - 1u;
+    const int nb = 1 << (hi - lo);
+    for (int b = tid; b < nb; b += kThreads) hist[b] = 0u;
+    __syncthreads();
+    for (int e = tid; e < listed; e += kThreads) {
+      const uint32_t key = lkey[e];
+      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> lo) & dmask], 1u);
+    }
+    __syncthreads();
+    find_digit<(1 << 10) / kThreads>(hist, nb, krem, wsum, sel);
+    prefix |= static_cast<uint32_t>(sel[0]) << lo;
+    pmask |= dmask << lo;
+    krem -= sel[1];
+    hi = lo;
+    __syncthreads();
+  }
+  const uint32_t T = prefix;
+  const int need_eq = static_cast<int>(krem);  // keys equal to T that are kept
+
+  // ---- listed keys above T are kept; those equal to T are marked
+  for (int e = tid; e < listed; e += kThreads) {
+    const uint32_t key = lkey[e], pos = lpos[e];
+    if (key > T) atomicOr(&mask[pos >> 5], 1u << (pos & 31));
+    else if (key == T) atomicOr(&eqm[pos >> 5], 1u << (pos & 31));
+  }
+  __syncthreads();
+
+  // ---- the first need_eq keys equal to T (lowest positions), then the
+  // kept positions in ascending order; thread t owns a run of words
+  const int wpt = (n_words + kThreads - 1) / kThreads;
+  const int w0 = min(n_words, tid * wpt), w1 = min(n_words, w0 + wpt);
+  uint32_t n_eq = 0;
+  for (int w = w0; w < w1; ++w) n_eq += __popc(eqm[w]);
+  uint32_t total;
+  uint32_t rank = block_exclusive_scan(n_eq, wsum, &total);
+  uint32_t n_kept = 0;
+  for (int w = w0; w < w1; ++w) {
+    uint32_t e = eqm[w];
+    const uint32_t c = __popc(e);
+    if (rank >= static_cast<uint32_t>(need_eq)) {
+      e = 0u;
+    } else if (rank + c > static_cast<uint32_t>(need_eq)) {
+      uint32_t keep = 0u;  // the lowest need_eq - rank set bits
+      for (uint32_t r = rank; r < static_cast<uint32_t>(need_eq); ++r) {
+        const uint32_t low = e & (0u - e);
+        keep |= low;
+        e ^= low;
+      }
+      e = keep;
+    }
+    rank += c;
+    const uint32_t m = mask[w] | e;
+    mask[w] = m;
+    n_kept += __popc(m);
+  }
+  uint32_t out = block_exclusive_scan(n_kept, wsum, &total);
+  int32_t *dst = idx + static_cast<size_t>(row) * static_cast<size_t>(K);
+  for (int w = w0; w < w1; ++w) {
+    uint32_t m = mask[w];
+    while (m) {
+      const int b = __ffs(m) - 1;
+      m &= m - 1u;
+      if (out < static_cast<uint32_t>(K)) dst[out] = 32 * w + b;
+      ++out;
+    }
+  }
+  if (tid == 0 && total != static_cast<uint32_t>(K)) record_device_status(BKV_DEV_ASSERT, 303);
+}
+
 __global__ void finalize_scores_kernel(const SelectInput in, size_t total, float *__restrict__ s) {
   for (size_t e = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; e < total;
        e += static_cast<size_t>(gridDim.x) * blockDim.x)
@@ -321,10 +567,42 @@ bkv_status launch_select_topk(const SelectInput &in, int n_rows, long long L, lo
   const bool vec = (L & 3) == 0 && (in.part_stride & 3) == 0 &&
                    (reinterpret_cast<uintptr_t>(in.src) & 15u) == 0 &&
                    (reinterpret_cast<uintptr_t>(s_out) & 15u) == 0;
-  if (vec)
+  if (vec && L <= kMaskMaxL) {
+    const int smem = mask_smem_bytes(L);
+    const int parts = in.n_parts >= 1 && in.n_parts <= 4 ? in.n_parts : 0;
+    bkv_status st = BKV_OK;
+    auto run = [&](auto kernel, int *attr_done) {
+      if (!ensure_smem_limit(kernel, mask_smem_bytes(kMaskMaxL), attr_done)) {
+        st = BKV_ERR_CUDA;
+        return;
+      }
+      kernel<<<n_rows, kThreads, smem, stream>>>(in, static_cast<int>(L), static_cast<int>(K),
+                                                 idx, s_out);
+    };
+    static int done[10][64];
+    if (in.mean) {
+      switch (parts) {
+        case 1: run(select_topk_mask_kernel<1, true>, done[0]); break;
+        case 2: run(select_topk_mask_kernel<2, true>, done[1]); break;
+        case 3: run(select_topk_mask_kernel<3, true>, done[2]); break;
+        case 4: run(select_topk_mask_kernel<4, true>, done[3]); break;
+        default: run(select_topk_mask_kernel<0, true>, done[4]); break;
+      }
+    } else {
+      switch (parts) {
+        case 1: run(select_topk_mask_kernel<1, false>, done[5]); break;
+        case 2: run(select_topk_mask_kernel<2, false>, done[6]); break;
+        case 3: run(select_topk_mask_kernel<3, false>, done[7]); break;
+        case 4: run(select_topk_mask_kernel<4, false>, done[8]); break;
+        default: run(select_topk_mask_kernel<0, false>, done[9]); break;
+      }
+    }
+    if (st != BKV_OK) return st;
+  } else if (vec) {
     select_topk_kernel<true><<<n_rows, kThreads, 0, stream>>>(in, L, K, idx, s_out);
-  else
+  } else {
     select_topk_kernel<false><<<n_rows, kThreads, 0, stream>>>(in, L, K, idx, s_out);
+  }
   return cudaGetLastError() == cudaSuccess ? BKV_OK : BKV_ERR_CUDA;
 }
 

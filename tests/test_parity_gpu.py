@@ -163,6 +163,63 @@ def test_score_mean(case, dev):
             check_topk(idx_all[l * wl.n_kv_heads + h], s_ref, wl.K, f"{case} mean top-K l{l} h{h}")
 
 
+def _threshold_bin_rows(rng, n_bin):
+    """Rows whose K-th largest score falls in [1, 1.125) -- one bin of the
+    select's first 12-bit digit (sign, exponent, 3 mantissa bits) -- holding
+    exactly n_bin keys: 100 keys above it, the rest below."""
+    L = 32768
+    rows = []
+    for _ in range(2):
+        x = rng.uniform(0.0, 0.5, L)
+        pos = rng.permutation(L)
+        x[pos[:100]] = rng.uniform(2.0, 4.0, 100)
+        x[pos[100:100 + n_bin]] = rng.uniform(1.0, 1.125, n_bin)
+        rows.append(x)
+    return np.stack(rows), 3100
+
+
+SELECT_CASES = {
+    "normal": lambda rng: (rng.standard_normal((6, 32768)), 6144),
+    "scores_like": lambda rng: (np.exp(rng.standard_normal((8, 32768)) * 2.0 - 12.0), 6144),
+    "rows_unaligned": lambda rng: (rng.standard_normal((5, 1001)), 300),
+    "ragged_slices": lambda rng: (rng.standard_normal((3, 1004)), 17),
+    "all_equal": lambda rng: (np.full((3, 20000), 0.25), 777),
+    "one_top_bin": lambda rng: (1.0 + rng.integers(0, 4096, (4, 32768)) * 2.0 ** -20, 5000),
+    "few_levels": lambda rng: (rng.integers(0, 7, (4, 32768)).astype(np.float64), 10000),
+    "signed_zeros": lambda rng: (rng.choice([-0.0, 0.0, -1.0, 1.0, 0.5], size=(4, 4096)), 1500),
+    "infinities": lambda rng: (np.where(rng.random((3, 8192)) < 0.01,
+                                        rng.choice([np.inf, -np.inf], size=(3, 8192)),
+                                        rng.standard_normal((3, 8192)) * 1e30), 700),
+    "bin_at_list_capacity": lambda rng: _threshold_bin_rows(rng, 6144),
+    "bin_past_list_capacity": lambda rng: _threshold_bin_rows(rng, 6145),
+    "k_one": lambda rng: (rng.standard_normal((2, 5000)), 1),
+    "k_all_but_one": lambda rng: (rng.standard_normal((2, 4096)), 4095),
+    "long_rows": lambda rng: (np.exp(rng.uniform(-60.0, 0.0, (2, 1 << 20))), 1 << 17),
+}
+
+
+@pytest.mark.parametrize("case", sorted(SELECT_CASES))
+def test_select_topk_exact(case, dev):
+    """The select on float32 scores is exact: the same positions, in the same
+    order, as the oracle's selection on those scores (ties to the lower
+    position, -0 equal to +0), over both of the kernel's routes -- a threshold
+    bin collected in shared memory, and the streaming radix for rows whose
+    threshold bin is too full or whose rows are not 16-byte aligned."""
+    bkv = _lib()
+    x, K = SELECT_CASES[case](np.random.default_rng(31))
+    x32 = np.ascontiguousarray(x, dtype=np.float32)
+    n_rows, L = x32.shape
+    scores = torch.from_numpy(x32).to(dev)
+    idx = torch.full((n_rows, min(K, L)), -1, dtype=torch.int32, device=dev)
+    bkv.bkv_select_topk(scores, n_rows, L, K, idx, None)
+    torch.cuda.synchronize()
+    assert bkv.bkv_read_device_status()[0] == 0
+    got = idx.cpu().numpy()
+    for r in range(n_rows):
+        ref = oracle.select_topk(x32[r].astype(np.float64), K)
+        assert np.array_equal(got[r], ref), (case, r, np.flatnonzero(got[r] != ref)[:5])
+
+
 FPS_CASES = {
     "tiny_f32": lambda: _synth().WORKLOADS["tiny"],
     "bf16_small": lambda: small(W=300, M=24, n_beacons_in=10),
