@@ -20,12 +20,14 @@
 //      that does not;
 //   4. writes the candidates' new distances back (exact, stamped) and, in an
 //      eager round, runs a distance pass that brings every point up to date.
-// Rounds are eager (with the pass) until one of them picks at least kSwitch
-// points: from then on only the candidates are refreshed (lazy rounds), which
-// avoids re-streaming the union; a lazy round that certifies no pick falls
-// back to an eager one.  On the clustered queries of the 14B-shaped workload
-// this takes ~5.5 passes over the union per head instead of ~9 (one per
-// round of the all-eager scheme).
+// A round that certifies fewer than kPassBelow picks is followed by a pass
+// (the next round starts from exact distances and certifies many); after a
+// round that certifies more, only the next round's candidates are refreshed
+// (a lazy round), which avoids re-streaming the union.  A pass costs about
+// as much as 1.8 rounds' select, gather and MMAs; on the clustered queries of
+// the 14B-shaped workload this policy takes ~8.4 rounds and ~5.8 passes per
+// head, against ~13.6 and ~4.6 for staying eager only until the first round
+// of 8 picks, and ~7.6 and ~6.6 for a pass after every round.
 //
 // The distance pass streams the union [beacons; window] of a query head by
 // TMA in tiles of 128 points (128-byte swizzle, no multicast) through a
@@ -72,7 +74,7 @@ constexpr int kPBlock = kPickRows * 128;          // one 64-element K block of t
 constexpr int kCBlock = kCand * 128;              // one 64-element K block of the candidates
 constexpr int kGramStride = kCand + 4;            // floats per Gram row (bank spread)
 constexpr int kListMax = 512;                     // threshold-bin keys ranked directly
-constexpr int kSwitch = 8;                        // picks that end the eager rounds
+constexpr int kPassBelow = 24;                    // a round with fewer picks is followed by a pass
 constexpr int kAhead = 4;                         // tiles prefetched into L2 beyond the ring
 constexpr int kSmallBytes = 4096;
 constexpr int kFixedBytes = kSmallBytes + 1024 + kStages * kTileBytes + 2 * kPBlock;
@@ -640,7 +642,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     int P = 1;          // picks so far
     int E = 1;          // every unselected point's stamp is at least E
-    bool eager = true;  // the next round runs a distance pass
+    bool eager = true;  // a pass preceded this round: every distance is exact
     float dmax = __uint_as_float(static_cast<uint32_t>(s.scal[kSKeyMax]) & 0x7fffffffu);
     while (P < m) {
       const int unsel = n - P;
@@ -907,8 +909,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncthreads();
         break;
       }
-      if (eager && np >= kSwitch) eager = false;
-      else if (!eager && np == 0) eager = true;
+      eager = np < kPassBelow;
       if (tid == 0) {  // the pass gathers the range of its new keys
         s.scal[kSKeyMin] = -1;
         s.scal[kSKeyMax] = 0;

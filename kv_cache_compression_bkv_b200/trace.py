@@ -15,10 +15,17 @@ device ring of ring_cap slots (query t in slot t % ring_cap), and the step
 reads the recent queries and the window in place from that ring (the window
 wraps around the ring's end whenever ring_cap is not a multiple of the
 interval); no window or recent-query buffer is assembled.
+
+Checkpoint and resume: between two compression events the whole state of the
+run is the current cache rows, the current beacons, the query ring (if any),
+the event log and a few counters; `checkpoint(path)` writes them with
+torch.save and `TraceRun.resume(path, device)` rebuilds the run (the trace's
+keys, values and queries are regenerated from its seed) and continues with
+the next event, with results identical to an uninterrupted run.
 """
 from __future__ import annotations
 
-from dataclasses import dataclass, field
+from dataclasses import asdict, dataclass, field
 
 import torch
 
@@ -86,13 +93,62 @@ class TraceRun:
         self.cur = 0            # which cache / beacon buffer holds the state
         self.L = 0              # cache rows
         self.n_beacons = 0
+        self.next_event = 0     # the event the next run() starts with
 
-    def run(self, on_event=None):
-        """Run the whole trace; on_event(run, event) sees the state after each
+    CHECKPOINT_VERSION = 1
+
+    def checkpoint(self, path) -> None:
+        """Write the state between two events (call it between run() calls)."""
+        kc, vc = self.cache[self.cur]
+        state = {
+            "version": self.CHECKPOINT_VERSION,
+            "trace": asdict(self.tr),
+            "seed": self.seed,
+            "layers": self.Ly,
+            "in_place": self.in_place,
+            "ring_cap": self.ring_cap,
+            "next_event": self.next_event,
+            "L": self.L,
+            "n_beacons": self.n_beacons,
+            "k": kc[:, :, :self.L].cpu(),
+            "v": vc[:, :, :self.L].cpu(),
+            "beacons": self.beacons[self.cur][:, :, :self.n_beacons].cpu(),
+            "ring": None if self.ring is None else self.ring.cpu(),
+            "events": [asdict(e) for e in self.events],
+        }
+        torch.save(state, path)
+
+    @classmethod
+    def resume(cls, path, device: torch.device) -> "TraceRun":
+        """A run in the state `checkpoint` wrote, ready to continue."""
+        state = torch.load(path, map_location="cpu", weights_only=True)
+        if state.get("version") != cls.CHECKPOINT_VERSION:
+            raise ValueError(f"unsupported trace checkpoint version {state.get('version')}")
+        run = cls(synth.Trace(**state["trace"]), seed=state["seed"], device=device,
+                  layers=state["layers"], in_place=state["in_place"],
+                  ring_cap=state["ring_cap"])
+        L, nb = state["L"], state["n_beacons"]
+        kc, vc = run.cache[run.cur]
+        kc[:, :, :L].copy_(state["k"])
+        vc[:, :, :L].copy_(state["v"])
+        run.beacons[run.cur][:, :, :nb].copy_(state["beacons"])
+        if run.ring is not None:
+            run.ring.copy_(state["ring"])
+        run.L, run.n_beacons, run.next_event = L, nb, state["next_event"]
+        run.events = [TraceEvent(**e) for e in state["events"]]
+        return run
+
+    def run(self, on_event=None, stop_after: int | None = None):
+        """Run the trace from the next event to the end (or through event
+        stop_after); on_event(run, event) sees the state after each
         compression (the current buffers; run.last_idx = kept positions)."""
         tr = self.tr
         stream = torch.cuda.current_stream(self.device)
         for e, t0 in enumerate(range(0, tr.steps, tr.interval)):
+            if e < self.next_event:
+                continue
+            if stop_after is not None and e > stop_after:
+                break
             t1 = t0 + tr.interval
             kc, vc = self.cache[self.cur]
             kc[:, :, self.L:self.L + tr.interval].copy_(self.keys[:, :, t0:t1])
@@ -125,6 +181,7 @@ class TraceRun:
             self.cur = 1 - self.cur
             self.L, self.n_beacons = nl, nb
             self.last_idx = idx
+            self.next_event = e + 1
             if on_event is not None:
                 on_event(self, event)
         return self.events

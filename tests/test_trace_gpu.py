@@ -92,3 +92,42 @@ def test_qwen3_4b_trace_follows_the_oracle_trace(in_place, ring_cap):
     assert sum(counts.values()) == Hkv * len(events), counts
     print(f"trace ({'in place' if in_place else 'out of place'}"
           f"{', query ring' if ring_cap else ''}): {counts}")
+
+
+def test_trace_resumes_from_a_checkpoint_bit_exactly(tmp_path):
+    """Run the trace to its end; run it again to event 3, checkpoint, resume
+    in a fresh run and finish: every later event keeps the same positions and
+    the final cache and beacons are the same bytes."""
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from kv_cache_compression_bkv_b200 import synth
+    from kv_cache_compression_bkv_b200.trace import TraceRun
+
+    tr = synth.TRACES["qwen3_4b_trace"]
+    dev = torch.device("cuda:0")
+
+    def record(store):
+        def on_event(run, ev):
+            store[ev.index] = (ev.L, ev.new_len, ev.n_beacons_out, run.last_idx.cpu().clone())
+        return on_event
+
+    full = {}
+    ref = TraceRun(tr, seed=0, device=dev, layers=1, ring_cap=5000)
+    ref.run(record(full))
+    first = TraceRun(tr, seed=0, device=dev, layers=1, ring_cap=5000)
+    first.run(stop_after=3)
+    path = tmp_path / "trace.pt"
+    first.checkpoint(path)
+    rest = {}
+    resumed = TraceRun.resume(path, dev)
+    assert resumed.next_event == 4 and len(resumed.events) == 4
+    resumed.run(record(rest))
+    assert sorted(rest) == [e for e in sorted(full) if e >= 4]
+    for e, (L, n, nb, idx) in rest.items():
+        fL, fn, fnb, fidx = full[e]
+        assert (L, n, nb) == (fL, fn, fnb), e
+        assert torch.equal(idx, fidx), e
+    for a, b in zip(ref.cache[ref.cur], resumed.cache[resumed.cur]):
+        assert torch.equal(a[:, :, :ref.L].view(torch.int16), b[:, :, :resumed.L].view(torch.int16))
+    assert torch.equal(ref.beacons[ref.cur][:, :, :ref.n_beacons].view(torch.int16),
+                       resumed.beacons[resumed.cur][:, :, :resumed.n_beacons].view(torch.int16))
