@@ -31,7 +31,8 @@
 //
 // The distance pass streams the union [beacons; window] of a query head by
 // TMA in tiles of 128 points (128-byte swizzle, no multicast) through a
-// 4-stage ring and forms D[128 points][N] = tile . picks^T (M = 128, K = 128,
+// 4-stage ring (each row fetched into L2 by its epilogue thread kAhead tiles
+// earlier) and forms D[128 points][N] = tile . picks^T (M = 128, K = 128,
 // N = the picks the points have not seen, rounded up to 16) in one of two
 // TMEM accumulators.  Two threads issue the MMAs (warp 1 the even tiles of
 // the sequence, warp 2 the odd ones) so their instruction latencies overlap;
@@ -75,7 +76,7 @@ constexpr int kCBlock = kCand * 128;              // one 64-element K block of t
 constexpr int kGramStride = kCand + 4;            // floats per Gram row (bank spread)
 constexpr int kListMax = 512;                     // threshold-bin keys ranked directly
 constexpr int kPassBelow = 24;                    // a round with fewer picks is followed by a pass
-constexpr int kAhead = 4;                         // tiles prefetched into L2 beyond the ring
+constexpr int kAhead = 12;                        // L2 prefetch distance of a pass, in tiles
 constexpr int kSmallBytes = 4096;
 constexpr int kFixedBytes = kSmallBytes + 1024 + kStages * kTileBytes + 2 * kPBlock;
 constexpr int kSmemLimit = 232448;
@@ -177,6 +178,34 @@ __device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Row r of tile j of a pass into L2 (its 256 bytes), if the row belongs
+// to the head: a beacon slot below nb, or a ring slot below w_cap.  The
+// pass's tiles are prefetched this way, by the epilogue thread of the row,
+// kAhead tiles ahead of the tile it has just finished, so that the TMA unit
+// moves only the ring's loads (an L2 prefetch by TMA costs the unit as much
+// time as the load itself).
+__device__ __forceinline__ void prefetch_row(const Head &h, const FpsGeom &g, int n_btiles,
+                                             int w_first, int j, int r) {
+  const __nv_bfloat16 *p = nullptr;
+  if (j < n_btiles) {
+    const int i = j * kTileRows + r;
+    if (i < h.nb) p = h.B + static_cast<size_t>(i) * kDim;
+  } else {
+    const long long slot = static_cast<long long>(w_first + j - n_btiles) * kTileRows + r;
+    if (slot < g.w_cap) p = h.Wp + static_cast<size_t>(slot) * kDim;
+  }
+  if (p != nullptr) {
+    // a 16-byte load that promotes the whole 256-byte row into L2.  Nothing
+    // reads its value, so the thread does not wait for it.  Measured a
+    // little ahead of prefetch instructions and of a bulk prefetch of the
+    // tile.
+    [[maybe_unused]] uint32_t a, b, c, d;
+    asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(a), "=r"(b), "=r"(c), "=r"(d)
+                 : "l"(p));
+  }
+}
+
 // Issue the TMA loads of tiles [0, n_tiles) of the pass that starts at
 // sequence number `seq` (producer thread only).  Returns false after a timeout.
 __device__ bool issue_tiles(const Layout &s, const CUtensorMap *bmap, const CUtensorMap *wmap,
@@ -188,15 +217,6 @@ __device__ bool issue_tiles(const Layout &s, const CUtensorMap *bmap, const CUte
     return j < n_btiles ? qh * g.M + j * kTileRows
                         : static_cast<int>(qh * g.w_cap) + (w_first + j - n_btiles) * kTileRows;
   };
-  // Tiles past the ring's depth are prefetched into L2 kAhead tiles before
-  // their stage frees, so that their loads are L2 hits: the ring holds
-  // kStages tiles, and a load from HBM takes about as long as kStages tiles'
-  // MMAs and epilogues.
-  auto prefetch = [&](int j) {
-    tma_prefetch_2d(map_of(j), 0, row_of(j));
-    tma_prefetch_2d(map_of(j), 64, row_of(j));
-  };
-  for (int j = kStages; j < min(n_tiles, kStages + kAhead); ++j) prefetch(j);
   for (int j = 0; j < n_tiles; ++j) {
     const uint32_t q = seq + j, st = q % kStages;
     if (!mbar_wait(empty0 + 8 * st, ((q / kStages) & 1) ^ 1, kWhereProd)) return false;
@@ -206,7 +226,6 @@ __device__ bool issue_tiles(const Layout &s, const CUtensorMap *bmap, const CUte
     const int y = row_of(j);
     tma_load_2d(dst, map, full0 + 8 * st, 0, y);
     tma_load_2d(dst + kTileRows * 128, map, full0 + 8 * st, 64, y);
-    if (j + kStages + kAhead < n_tiles) prefetch(j + kStages + kAhead);
   }
   return true;
 }
@@ -237,8 +256,9 @@ __device__ __forceinline__ float chunk_min(const float (&v)[32], const float *pi
 // so far have moved through the ring, so every role derives the same stage,
 // accumulator and barrier phase for each tile.
 __device__ void distance_pass(const Layout &s, const CUtensorMap *bmap, const CUtensorMap *wmap,
-                              uint32_t tmem, int qh, const FpsGeom &g, int n_btiles, int w_first,
-                              int n_tiles, uint32_t seq, int s0, int P, bool first) {
+                              uint32_t tmem, int qh, const Head &h, const FpsGeom &g,
+                              int n_btiles, int w_first, int n_tiles, uint32_t seq, int s0, int P,
+                              bool first) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t full0 = smem_u32(&s.bars[kBarFull]), empty0 = smem_u32(&s.bars[kBarEmpty]);
   const uint32_t tfull0 = smem_u32(&s.bars[kBarTfull]), tempty0 = smem_u32(&s.bars[kBarTempty]);
@@ -288,6 +308,10 @@ __device__ void distance_pass(const Layout &s, const CUtensorMap *bmap, const CU
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     bool ok = true;  // warp-uniform; after a timeout the warp keeps only the barriers
+    // the first kAhead tiles past the ring, split between the warpgroups like
+    // the tiles themselves
+    for (int j = kStages; j < min(n_tiles, kAhead); ++j)
+      if (static_cast<int>((seq + j) & 1u) == wg) prefetch_row(h, g, n_btiles, w_first, j, r);
     for (int j = 0; j < n_tiles; ++j) {
       const uint32_t q = seq + j, a = q % kAcc;
       if (static_cast<int>(a & 1u) != wg) continue;
@@ -373,6 +397,7 @@ __device__ void distance_pass(const Layout &s, const CUtensorMap *bmap, const CU
         atomicMin(reinterpret_cast<unsigned int *>(&s.scal[kSKeyMin]), kmn);
         atomicMax(reinterpret_cast<unsigned int *>(&s.scal[kSKeyMax]), kmx);
       }
+      if (j + kAhead < n_tiles) prefetch_row(h, g, n_btiles, w_first, j + kAhead, r);
     }
   }
 }
@@ -633,7 +658,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (m <= 1) continue;  // nothing past the seed (every thread sees the same m)
     fence_proxy_async_smem();
     __syncthreads();
-    distance_pass(s, &bmap, &wmap, tmem, qh, g, n_btiles, wt.first, n_tiles, seq, 0, 1, true);
+    distance_pass(s, &bmap, &wmap, tmem, qh, h, g, n_btiles, wt.first, n_tiles, seq, 0, 1, true);
     seq += n_tiles;
     __syncthreads();
     if (s.scal[kAbort]) break;
@@ -917,7 +942,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       __syncthreads();
       if (eager) {
-        distance_pass(s, &bmap, &wmap, tmem, qh, g, n_btiles, wt.first, n_tiles, seq, E & ~7, P,
+        distance_pass(s, &bmap, &wmap, tmem, qh, h, g, n_btiles, wt.first, n_tiles, seq, E & ~7, P,
                       false);
         seq += n_tiles;
         __syncthreads();
