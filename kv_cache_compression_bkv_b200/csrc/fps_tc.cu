@@ -77,7 +77,11 @@ constexpr int kGramStride = kCand + 4;            // floats per Gram row (bank s
 constexpr int kListMax = 512;                     // threshold-bin keys ranked directly
 constexpr int kPassBelow = 24;                    // a round with fewer picks is followed by a pass
 constexpr int kAhead = 12;                        // L2 prefetch distance of a pass, in tiles
-constexpr int kSmallBytes = 4096;
+constexpr int kSmallBytes = 8192;  // barriers, scalars, lists; the u histogram at 4096
+// The persistent histogram of the live points' u over [0, 2] (the range of a
+// cosine distance): bin = floor(u * 512), clamped to the last bin.
+constexpr int kUBins = 1024;
+constexpr float kUScale = 512.f;
 constexpr int kFixedBytes = kSmallBytes + 1024 + kStages * kTileBytes + 2 * kPBlock;
 constexpr int kSmemLimit = 232448;
 // TMEM: two pass accumulators of up to 128 columns, the Gram and refresh blocks
@@ -110,6 +114,8 @@ enum {
   kSDmax = 14,     // upper bound of every live distance (float bits)
   kAbort = 15,
   kSLive = 16,     // live keys counted by the histogram
+  kSPlaced = 17,   // points placed above the threshold bin (fixed-range select)
+  kSListed = 18,   // points listed from the threshold bin (fixed-range select)
   kScalWords = 32
 };
 
@@ -129,6 +135,7 @@ struct Layout {
   float *cdist;     // [kCand + 1]
   int *pick;        // [kCand] candidate slots picked this round, in order
   float *pinv;      // [kPickRows] inverse norm of pick k (NaN past the last pick)
+  uint32_t *uhist;  // [kUBins] live points per bin of u, kept up to date over a head
   uint8_t *ring;    // [kStages][kTileBytes]
   uint8_t *pop;     // picks, K-major 128-byte swizzle: [2][kPickRows][128 B]
   float *gram;      // (ring) [kCand][kGramStride]
@@ -176,6 +183,12 @@ struct WindowTiles {
 
 __device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// The u-histogram bin of a live point's distance (-1 for a selected point,
+// u = -1, or a distance that is not a number).  Monotonic in u.
+__device__ __forceinline__ int ubin(float u) {
+  return u >= 0.f ? min(kUBins - 1, static_cast<int>(u * kUScale)) : -1;
 }
 
 // Row r of tile j of a pass into L2 (its 256 bytes), if the row belongs
@@ -389,6 +402,7 @@ __device__ void distance_pass(const Layout &s, const CUtensorMap *bmap, const CU
         const float nd = fmaxf(fminf(di, mn), 0.f);
         s.dist[i] = nd;
         s.stamp[i] = static_cast<uint8_t>(P);
+        atomicAdd(&s.uhist[ubin(nd)], 1u);  // the pass rebuilds the histogram
         kmn = kmx = dist_key(nd);
       }
       kmn = __reduce_min_sync(0xffffffffu, kmn);
@@ -565,6 +579,123 @@ __device__ bool select_hist(const Layout &s, int n, int want, bool bounded, floa
   return true;
 }
 
+// Step 1 of a round from the persistent histogram (s.uhist, one count per
+// live point in bin ubin(u)): warp 0 finds the bin holding the want-th key,
+// every point above it is placed by a block-wide prefix sum, and the keys of
+// that bin are ranked against each other (key desc, index asc), the
+// (kCand+1)-th going to slot kCand when `bounded`.  The counts the placement
+// finds must equal the histogram's; if they do not (or the threshold bin
+// holds more than kListMax keys, or fewer than `want` keys are live), nothing
+// is kept and the caller uses the other selects.
+__device__ bool select_fixed(const Layout &s, int n, int want, bool bounded) {
+  if (n > kPerThread * kThreads) return false;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (warp == 0) {
+    // lane l sums bins 1023 - 32l - 31 .. 1023 - 32l (each lane reads a
+    // different bank at every step)
+    uint32_t sum = 0;
+#pragma unroll 8
+    for (int k = 0; k < 32; ++k) sum += s.uhist[kUBins - 1 - 32 * lane - ((k + lane) & 31)];
+    uint32_t incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    const uint32_t excl = incl - sum;
+    const uint32_t total = __shfl_sync(0xffffffffu, incl, 31);
+    const uint32_t w = static_cast<uint32_t>(want);
+    const uint32_t hold = __ballot_sync(0xffffffffu, excl < w && w <= incl);
+    int fallback = total < w || hold == 0u ? 1 : 0;
+    const int L = hold ? __ffs(hold) - 1 : 0;
+    // lane k takes the k-th highest bin of lane L's run
+    const uint32_t exL = __shfl_sync(0xffffffffu, excl, L);
+    const uint32_t c = s.uhist[kUBins - 1 - 32 * L - lane];
+    uint32_t inc2 = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t t = __shfl_up_sync(0xffffffffu, inc2, o);
+      if (lane >= o) inc2 += t;
+    }
+    const uint32_t reach = __ballot_sync(0xffffffffu, exL + inc2 >= w);
+    const int k = reach ? __ffs(reach) - 1 : 0;
+    if (!reach) fallback = 1;
+    const uint32_t ck = __shfl_sync(0xffffffffu, c, k);
+    const uint32_t above = exL + __shfl_sync(0xffffffffu, inc2, k) - ck;
+    if (lane == 0) {
+      s.scal[kSBin] = kUBins - 1 - 32 * L - k;
+      s.scal[kSAbove] = static_cast<int>(above);
+      s.scal[kSNeed] = want - static_cast<int>(above);
+      s.scal[kSFallback] = fallback || ck > static_cast<uint32_t>(kListMax) ? 1 : 0;
+      s.scal[kSListed] = static_cast<int>(ck);
+    }
+  }
+  __syncthreads();
+  if (s.scal[kSFallback]) return false;
+  const int bstar = s.scal[kSBin], above = s.scal[kSAbove], need = s.scal[kSNeed];
+  const int in_bin = s.scal[kSListed];
+  float du[kPerThread];
+  int bins[kPerThread];
+  uint32_t na = 0, nl = 0;
+#pragma unroll
+  for (int k = 0; k < kPerThread; ++k) {
+    const int i = tid + k * kThreads;
+    du[k] = i < n ? s.dist[i] : -1.f;
+    bins[k] = ubin(du[k]);
+    na += bins[k] > bstar ? 1u : 0u;
+    nl += bins[k] == bstar ? 1u : 0u;
+  }
+  const uint32_t mine = (na << 16) | nl;
+  const uint32_t pre = block_exclusive_scan(mine, s.whist);
+  if (tid == kThreads - 1) {
+    s.scal[kSPlaced] = static_cast<int>((pre + mine) >> 16);
+    s.scal[kSLive] = static_cast<int>((pre + mine) & 0xffffu);
+  }
+  int pa = static_cast<int>(pre >> 16), pb = static_cast<int>(pre & 0xffffu);
+#pragma unroll
+  for (int k = 0; k < kPerThread; ++k) {
+    const int i = tid + k * kThreads;
+    if (bins[k] > bstar) {
+      if (pa <= kCand) {
+        s.cidx[pa] = i;
+        s.cdist[pa] = du[k];
+      }
+      ++pa;
+    } else if (bins[k] == bstar) {
+      if (pb < kListMax) {
+        s.lkey[pb] = dist_key(du[k]);
+        s.lidx[pb] = i;
+      }
+      ++pb;
+    }
+  }
+  __syncthreads();
+  if (s.scal[kSPlaced] != above || s.scal[kSLive] != in_bin) {
+    // the histogram disagrees with the distances: report, use another select
+    if (tid == 0) record_device_status(BKV_DEV_ASSERT, 406);
+    __syncthreads();  // every thread has read the counts
+    return false;
+  }
+  // rank the bin's keys (key desc, index asc): rank r < need is taken, the
+  // last taken one (rank need-1) is the bound when the selection is bounded
+  for (int e = tid; e < in_bin; e += kThreads) {
+    const uint32_t ke = s.lkey[e];
+    const int ie = s.lidx[e];
+    int rank = 0;
+    for (int f = 0; f < in_bin; ++f) {
+      const uint32_t kf = s.lkey[f];
+      rank += (kf > ke || (kf == ke && s.lidx[f] < ie)) ? 1 : 0;
+    }
+    if (rank < need) {
+      const int slot = bounded && rank == need - 1 ? kCand : above + rank;
+      s.cidx[slot] = ie;
+      s.cdist[slot] = __uint_as_float(ke & 0x7fffffffu);
+    }
+  }
+  __syncthreads();
+  return true;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     fps_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__ CUtensorMap wmap,
                   const FpsGeom g, const __nv_bfloat16 *__restrict__ beacons_in,
@@ -582,6 +713,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   s.cdist = reinterpret_cast<float *>(smem_raw + 1936);
   s.pick = reinterpret_cast<int *>(smem_raw + 2464);
   s.pinv = reinterpret_cast<float *>(smem_raw + 2976);   // .. 3552
+  s.uhist = reinterpret_cast<uint32_t *>(smem_raw + 4096);  // .. 8192
   const uint32_t raw_base = smem_u32(smem_raw);
   const uint32_t big = (raw_base + kSmallBytes + 1023u) & ~1023u;
   s.ring = smem_raw + (big - raw_base);
@@ -656,13 +788,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int k = 1 + tid; k < kPickRows; k += kThreads) s.pinv[k] = __int_as_float(0x7fc00000);
     if (m <= 1) continue;  // nothing past the seed (every thread sees the same m)
+    for (int b = tid; b < kUBins; b += kThreads) s.uhist[b] = 0u;
     fence_proxy_async_smem();
     __syncthreads();
     distance_pass(s, &bmap, &wmap, tmem, qh, h, g, n_btiles, wt.first, n_tiles, seq, 0, 1, true);
     seq += n_tiles;
     __syncthreads();
     if (s.scal[kAbort]) break;
-    if (tid == 0) s.dist[0] = -1.f;
+    if (tid == 0) {
+      const int b = ubin(s.dist[0]);  // the seed leaves the live set
+      if (b >= 0) s.uhist[b] -= 1u;
+      s.dist[0] = -1.f;
+    }
     __syncthreads();
 
     int P = 1;          // picks so far
@@ -675,7 +812,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool bounded = unsel > kCand;
       const int want = bounded ? kCand + 1 : nc;
       // ---- 1. candidates
-      if (!select_hist(s, n, want, bounded, dmax)) {
+      if (!select_fixed(s, n, want, bounded) && !select_hist(s, n, want, bounded, dmax)) {
         // a threshold bin too crowded to rank (or distances that are not
         // numbers): the radix select, then the bound moves to slot kCand
         select_best<kThreads>(s.dist, n, unsel, want, s.whist, s.hist, s.scal, s.cidx, s.cdist,
@@ -887,10 +1024,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         // the candidates not picked keep exact distances to all P + np picks;
-        // every other point's u is at most the bound
+        // every other point's u is at most the bound.  The histogram of u
+        // follows: a picked candidate leaves it, the others move bins.
         float dm = bounded ? bd : 0.f;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
+          if (lane + 32 * q >= nc) continue;
+          const int bo = ubin(s.dist[ix[q]]);
+          const int bn = taken[q] ? -1 : ubin(c[q]);
+          if (bn != bo) {
+            if (bo >= 0) atomicSub(&s.uhist[bo], 1u);
+            if (bn >= 0) atomicAdd(&s.uhist[bn], 1u);
+          }
           if (!taken[q]) {
             s.dist[ix[q]] = c[q];
             s.stamp[ix[q]] = static_cast<uint8_t>(P + np);
@@ -939,6 +1084,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         s.scal[kSKeyMin] = -1;
         s.scal[kSKeyMax] = 0;
       }
+      if (eager)  // and rebuilds the histogram of u
+        for (int b = tid; b < kUBins; b += kThreads) s.uhist[b] = 0u;
       fence_proxy_async_smem();
       __syncthreads();
       if (eager) {
