@@ -16,7 +16,10 @@ from dataclasses import dataclass
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libbkv.so")
+# BKV_LIBRARY=debug loads the bounds-checked build (libbkv_debug.so), whose
+# kernels report a data-dependent index out of range in the device status word
+LIB_PATH = os.path.join(_HERE, "libbkv_debug.so" if os.environ.get("BKV_LIBRARY") == "debug"
+                        else "libbkv.so")
 
 BKV_F32, BKV_BF16 = 0, 1
 AGGREGATE = {"max": 0, "mean": 1}   # bkv_aggregate

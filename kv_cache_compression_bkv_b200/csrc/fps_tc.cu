@@ -49,6 +49,7 @@
 
 #include <algorithm>
 
+#include "bkv_check.cuh"
 #include "bkv_internal.h"
 #include "fps_common.cuh"
 #include "sm100.cuh"
@@ -342,6 +343,7 @@ __device__ void distance_pass(const Layout &s, const CUtensorMap *bmap, const CU
         valid = slot < g.w_cap && w < g.W;
         i = valid ? g.nb_in + static_cast<int>(w) : 0;
       }
+      if (valid && !BKV_CHECK(i >= 0 && i < g.nb_in + g.W, 707)) valid = false;
       const uint32_t st = q % kStages;
       if (ok && !mbar_wait_warp(tfull0 + 8 * a, (q / kAcc) & 1, kWhereEpi)) {
         s.scal[kAbort] = 1;
@@ -861,7 +863,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int u = 0; u < kIters; ++u) {
           const int e = tid + u * kThreads;
           if (e < nc * 16)
-            v[u] = __ldg(reinterpret_cast<const uint4 *>(h.point(s.cidx[e >> 4]) + (e & 15) * 8));
+          {
+            const int ci = s.cidx[e >> 4];
+            if (BKV_CHECK(ci >= 0 && ci < n, 701))
+              v[u] = __ldg(reinterpret_cast<const uint4 *>(h.point(ci) + (e & 15) * 8));
+          }
         }
 #pragma unroll
         for (int u = 0; u < kIters; ++u) {
@@ -873,7 +879,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (tid < nc) {
-          const int t = s.stamp[s.cidx[tid]];
+          const int ci = s.cidx[tid];
+          const int t = BKV_CHECK(ci >= 0 && ci < n, 702) ? s.stamp[ci] : P;
           if (t < P) atomicMin(&s.scal[kSRef], t);
         }
       }
@@ -937,7 +944,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
           } else {
-            const int i = a < nc ? s.cidx[a] : 0;
+            int i = a < nc ? s.cidx[a] : 0;
+            if (!BKV_CHECK(i >= 0 && i < n, 703)) i = 0;
             const int t = a < nc ? static_cast<int>(s.stamp[i]) : P;
             const float inv_a = a < nc ? s.inv[i] : 0.f;
             float mn = INFINITY;
@@ -980,6 +988,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           taken[q] = a >= nc;
           c[q] = taken[q] ? 0.f : s.cdist[a];
           ix[q] = taken[q] ? 0x7fffffff : s.cidx[a];
+          if (!taken[q] && !BKV_CHECK(ix[q] >= 0 && ix[q] < n, 704)) {
+            taken[q] = true;  // skipped: its index is not a point of the union
+            ix[q] = 0x7fffffff;
+          }
           iv[q] = taken[q] ? 0.f : s.inv[ix[q]];
         }
         const float bd = bounded ? s.cdist[kCand] : -3.f;
@@ -1064,11 +1076,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int e = tid; e < np * 16; e += kThreads) {
         const int k = e >> 4, c16 = e & 15, kb = c16 >> 3, c = c16 & 7;
         const int a = s.pick[k];
+        if (!BKV_CHECK(a >= 0 && a < nc && P + k < kPickRows, 705)) continue;
         const uint4 v = *reinterpret_cast<const uint4 *>(s.cop + kb * kCBlock + sw128_offset(a, c));
         *reinterpret_cast<uint4 *>(s.pop + kb * kPBlock + sw128_offset(P + k, c)) = v;
         *reinterpret_cast<uint4 *>(out + static_cast<size_t>(P + k) * kDim + c16 * 8) = v;
         if (c16 == 0) {
           const int i = s.cidx[a];
+          if (!BKV_CHECK(i >= 0 && i < n, 706)) continue;
           s.pinv[P + k] = s.inv[i];
           s.dist[i] = -1.f;
         }

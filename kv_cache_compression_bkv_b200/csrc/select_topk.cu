@@ -30,6 +30,7 @@
 
 #include <algorithm>
 
+#include "bkv_check.cuh"
 #include "bkv_device_status.cuh"
 #include "bkv_internal.h"
 
@@ -491,6 +492,7 @@ __global__ void __launch_bounds__(kThreads, 3)
   // ---- listed keys above T are kept; those equal to T are marked
   for (int e = tid; e < listed; e += kThreads) {
     const uint32_t key = lkey[e], pos = lpos[e];
+    if (!BKV_CHECK(pos < static_cast<uint32_t>(L), 711)) continue;
     if (key > T) atomicOr(&mask[pos >> 5], 1u << (pos & 31));
     else if (key == T) atomicOr(&eqm[pos >> 5], 1u << (pos & 31));
   }

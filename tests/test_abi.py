@@ -35,6 +35,16 @@ def test_exports_every_declared_function():
     assert set(bkv.EXPORTS) >= set(names) - set(), (set(names) - set(bkv.EXPORTS))
 
 
+def test_debug_library_exports_every_declared_function():
+    """libbkv_debug.so (the bounds-checked build) has the same ABI."""
+    path = os.path.join(os.path.dirname(bkv.__file__), "libbkv_debug.so")
+    if not os.path.exists(path):
+        pytest.skip("libbkv_debug.so is not built")
+    dbg = ctypes.CDLL(path)
+    for name in declared_functions():
+        assert hasattr(dbg, name), name
+
+
 def test_status_strings():
     for code in range(7):
         assert LIB.bkv_status_string(code)
