@@ -233,7 +233,29 @@ FPS_CASES = {
     "large_union": lambda: small(n_q_heads=2, n_kv_heads=1, W=9000, M=32, n_beacons_in=32),
     # naive FPS (Fig. 7's baseline): the whole query history, no beacons
     "naive_history": lambda: small(n_q_heads=4, n_kv_heads=1, W=20000, M=48, n_beacons_in=0),
+    # 1500 copies of one window row: the candidate select's threshold bin
+    # holds them all, past what it ranks directly, so its fallbacks run
+    "duplicate_rows": lambda: small(n_q_heads=2, n_kv_heads=1, W=2000, M=64, n_beacons_in=16),
+    # a window of nearly parallel rows: every distance below 1e-3
+    "near_parallel": lambda: small(n_q_heads=2, n_kv_heads=1, W=600, M=32, n_beacons_in=8),
 }
+
+
+def _duplicate_rows(inp):
+    inp.window[:, :, 200:1700] = inp.window[:, :, 100:101]
+
+
+def _near_parallel(inp):
+    gen = torch.Generator().manual_seed(77)
+    base = torch.randn(inp.window.shape[:2] + (1, inp.window.shape[-1]), generator=gen)
+    noise = 0.02 * torch.randn(inp.window.shape, generator=gen)
+    inp.window.copy_((base + noise).to(inp.window.dtype))
+    nb = inp.beacons.shape[2]
+    bnoise = 0.02 * torch.randn(inp.beacons.shape, generator=gen)
+    inp.beacons.copy_((base.expand(-1, -1, nb, -1) + bnoise).to(inp.beacons.dtype))
+
+
+FPS_HOOKS = {"duplicate_rows": _duplicate_rows, "near_parallel": _near_parallel}
 
 
 @pytest.mark.parametrize("case", sorted(FPS_CASES))
@@ -241,6 +263,8 @@ def test_update_beacons(case, dev):
     bkv, synth = _lib(), _synth()
     wl = FPS_CASES[case]()
     inp = synth.make_step_inputs(wl, seed=5)
+    if case in FPS_HOOKS:
+        FPS_HOOKS[case](inp)
     g = bkv.geometry_of(inp.k, wl.n_q_heads)
     bin_, win = inp.beacons.to(dev), inp.window.to(dev)
     bout = torch.zeros_like(bin_)
@@ -249,6 +273,7 @@ def test_update_beacons(case, dev):
     n = bkv.bkv_update_beacons(g, bin_ if wl.beacons_in else None, wl.beacons_in, wl.M, win,
                                wl.W, bout, ws)
     torch.cuda.synchronize()
+    assert bkv.bkv_read_device_status()[0] == 0
     assert n == min(wl.M, wl.beacons_in + wl.W)
     out_raw = raw(bout)
     for l in range(wl.n_layers):
