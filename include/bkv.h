@@ -170,6 +170,11 @@ bkv_status bkv_compact_inplace(const bkv_cache_desc *desc, void *k, void *v,
  *   beacons_in  device, [Ly][Hq][M][d];  window device, [Ly][Hq][W][d]
  *   beacons_out device, [Ly][Hq][M][d]; must not overlap beacons_in or window
  *   n_beacons_out  host out (optional): min(M, n_beacons_in + W)
+ *   workspace   device, 16-byte aligned, at least
+ *               bkv_workspace_size(desc, 1, 0, M, W, 1) bytes: the counter that
+ *               hands out query heads to the GPU's CTAs (16 bytes, reset at the
+ *               start of every call on `stream`), plus the per-point distance
+ *               arrays of unions too large for shared memory
  * Requires M >= 1, 0 <= n_beacons_in <= M, W >= 0, n_beacons_in + W >= 1. */
 bkv_status bkv_update_beacons(const bkv_cache_desc *desc,
                               const void *beacons_in, int32_t n_beacons_in,

@@ -117,6 +117,7 @@ enum {
   kSLive = 16,     // live keys counted by the histogram
   kSPlaced = 17,   // points placed above the threshold bin (fixed-range select)
   kSListed = 18,   // points listed from the threshold bin (fixed-range select)
+  kSHead = 19,     // the next query head this CTA takes
   kScalWords = 32
 };
 
@@ -702,7 +703,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     fps_tc_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__ CUtensorMap wmap,
                   const FpsGeom g, const __nv_bfloat16 *__restrict__ beacons_in,
                   const __nv_bfloat16 *__restrict__ window, __nv_bfloat16 *__restrict__ beacons_out,
-                  int n_qheads, uint8_t *__restrict__ garrays, size_t slice_bytes) {
+                  int n_qheads, uint8_t *__restrict__ garrays, size_t slice_bytes,
+                  int *__restrict__ head_counter) {
   extern __shared__ uint8_t smem_raw[];
   const int n = g.nb_in + g.W;
   const int m = g.n_pick;
@@ -765,7 +767,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t gram_phase = 0;
   bool stuck = false;  // uniform: set by every thread from the same shared value
 
-  for (int qh = blockIdx.x; qh < n_qheads; qh += gridDim.x) {
+  // Query heads are handed out as CTAs become free: head blockIdx.x first,
+  // then the next unclaimed one (a head's cost varies with its rounds and
+  // passes by about +-20%, which static striding would leave to the slowest
+  // CTA).
+  auto next_head = [&]() {
+    __syncthreads();  // the slot's previous value has been read by every thread
+    if (tid == 0) s.scal[kSHead] = static_cast<int>(gridDim.x) + atomicAdd(head_counter, 1);
+    __syncthreads();
+    return s.scal[kSHead];
+  };
+  for (int qh = blockIdx.x; qh < n_qheads; qh = next_head()) {
     Head h{beacons_in + static_cast<size_t>(qh) * g.M * kDim,
            window + static_cast<size_t>(qh) * g.w_cap * kDim, g.nb_in,
            g.w_cap > 0 ? g.w_cap : 1, g.w_start};
@@ -1161,8 +1173,12 @@ int fps_tc_grid(const FpsGeom &g) { return std::min(g.n_layers * g.n_q_heads, kM
 
 }  // namespace
 
+// The head counter (16 bytes), then, for a union too large for shared
+// memory, one slice of the per-point arrays per CTA.
+constexpr size_t kCounterBytes = 16;
 size_t fps_tc_workspace_bytes(const FpsGeom &g) {
-  return arrays_in_smem(g) ? 0 : static_cast<size_t>(fps_tc_grid(g)) * union_array_bytes(g);
+  return kCounterBytes +
+         (arrays_in_smem(g) ? 0 : static_cast<size_t>(fps_tc_grid(g)) * union_array_bytes(g));
 }
 
 bool fps_tc_supported(const FpsGeom &g) {
@@ -1176,8 +1192,7 @@ bkv_status launch_fps_tc(const FpsGeom &g, const void *beacons_in, const void *w
                          void *beacons_out, void *ws, size_t ws_bytes, cudaStream_t stream) {
   if (injected_launch_failure()) return BKV_ERR_CUDA;
   const size_t ws_need = fps_tc_workspace_bytes(g);
-  if (ws_need > 0 && (ws == nullptr || ws_bytes < ws_need ||
-                      (reinterpret_cast<uintptr_t>(ws) & 15u) != 0))
+  if (ws == nullptr || ws_bytes < ws_need || (reinterpret_cast<uintptr_t>(ws) & 15u) != 0)
     return BKV_ERR_WORKSPACE;
   const int n_qheads = g.n_layers * g.n_q_heads;
   // Tensor maps over every head's beacon slots and window rows.  A map needs
@@ -1200,10 +1215,13 @@ bkv_status launch_fps_tc(const FpsGeom &g, const void *beacons_in, const void *w
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = std::max(1, std::min(fps_tc_grid(g), sms));
+  int *counter = static_cast<int *>(ws);
+  if (cudaMemsetAsync(counter, 0, sizeof(int), stream) != cudaSuccess) return BKV_ERR_CUDA;
+  uint8_t *arrays = ws_need > kCounterBytes ? static_cast<uint8_t *>(ws) + kCounterBytes : nullptr;
   fps_tc_kernel<<<grid, kThreads, smem, stream>>>(
       bmap, wmap, g, static_cast<const __nv_bfloat16 *>(beacons_in),
       static_cast<const __nv_bfloat16 *>(window), static_cast<__nv_bfloat16 *>(beacons_out),
-      n_qheads, ws_need > 0 ? static_cast<uint8_t *>(ws) : nullptr, union_array_bytes(g));
+      n_qheads, arrays, union_array_bytes(g), counter);
   return cudaGetLastError() == cudaSuccess ? BKV_OK : BKV_ERR_CUDA;
 }
 
