@@ -238,6 +238,9 @@ FPS_CASES = {
     "duplicate_rows": lambda: small(n_q_heads=2, n_kv_heads=1, W=2000, M=64, n_beacons_in=16),
     # a window of nearly parallel rows: every distance below 1e-3
     "near_parallel": lambda: small(n_q_heads=2, n_kv_heads=1, W=600, M=32, n_beacons_in=8),
+    # more than 128 beacons, and bf16 rows of 64 dimensions: the CUDA-core kernel
+    "many_beacons": lambda: small(n_q_heads=2, n_kv_heads=1, W=400, M=160, n_beacons_in=100),
+    "bf16_d64": lambda: small(head_dim=64, W=300, M=24, n_beacons_in=10),
 }
 
 
