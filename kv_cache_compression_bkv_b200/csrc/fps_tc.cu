@@ -7,9 +7,12 @@
 // upper bound u_i of its distance to the picked set and a stamp t_i: u_i is
 // the exact distance to the first t_i picks (distances only fall as picks are
 // added, so u_i bounds the true distance).  A round
-//   1. selects the T = 128 points with the largest u (histogram of u over
-//      [0, max u] in 256 bins, then the threshold bin ranked exactly), and
-//      the (T+1)-th, whose u bounds every other point's true distance;
+//   1. selects the T = 128 points with the largest u, and the (T+1)-th,
+//      whose u bounds every other point's true distance: from a 1024-bin
+//      histogram of u over [0, 2] that is kept up to date across rounds
+//      (rebuilt by each pass, moved by each round's write-back), the
+//      threshold bin's keys ranked exactly; when that bin is too full, from
+//      a two-level histogram built afresh, then a radix select;
 //   2. stages the candidates' rows in the MMA's swizzled layout and forms, in
 //      one tcgen05 commit, their Gram block (M = N = 128) and -- for
 //      candidates whose stamp is behind -- their dots with the picks they
@@ -33,16 +36,17 @@
 // TMA in tiles of 128 points (128-byte swizzle, no multicast) through a
 // 4-stage ring (each row fetched into L2 by its epilogue thread kAhead tiles
 // earlier) and forms D[128 points][N] = tile . picks^T (M = 128, K = 128,
-// N = the picks the points have not seen, rounded up to 16) in one of two
+// N = the picks the points have not seen, rounded up to 16) in one of four
 // TMEM accumulators.  Two threads issue the MMAs (warp 1 the even tiles of
 // the sequence, warp 2 the odd ones) so their instruction latencies overlap;
 // two epilogue warpgroups (TMEM lane = point) turn the dots into cosine
 // distances.  Between passes the ring's shared memory holds the round's
 // candidate rows, Gram block and selection scratch.
 //
-// The grid is persistent: one CTA per SM loops over the query heads.  The
-// distance, inverse-norm and stamp arrays live in shared memory, or for a
-// union too large for it in the caller's workspace (one slice per CTA).
+// The grid is persistent: one CTA per SM takes query heads from a counter in
+// the workspace as it becomes free.  The distance, inverse-norm and stamp
+// arrays live in shared memory, or for a union too large for it in the
+// caller's workspace (one slice per CTA).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
