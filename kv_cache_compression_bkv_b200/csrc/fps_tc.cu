@@ -35,9 +35,10 @@
 // The distance pass streams the union [beacons; window] of a query head by
 // TMA in tiles of 128 points (128-byte swizzle, no multicast) through a
 // 4-stage ring (each row fetched into L2 by its epilogue thread kAhead tiles
-// earlier) and forms D[128 points][N] = tile . picks^T (M = 128, K = 128,
-// N = the picks the points have not seen, rounded up to 16) in one of four
-// TMEM accumulators.  Two threads issue the MMAs (warp 1 the even tiles of
+// earlier; a fixed share of each union's tiles stays in L2 across passes,
+// evict-last, and the rest streams evict-first) and forms D[128 points][N] =
+// tile . picks^T (M = 128, K = 128, N = the picks the points have not seen,
+// rounded up to 16) in one of four TMEM accumulators.  Two threads issue the MMAs (warp 1 the even tiles of
 // the sequence, warp 2 the odd ones) so their instruction latencies overlap;
 // two epilogue warpgroups (TMEM lane = point) turn the dots into cosine
 // distances.  Between passes the ring's shared memory holds the round's
@@ -78,7 +79,9 @@ constexpr int kMaxPick = 128;                     // beacons per head on this pa
 constexpr int kPickRows = kMaxPick + 16;          // picks operand rows (N padding)
 constexpr int kPBlock = kPickRows * 128;          // one 64-element K block of the picks
 constexpr int kCBlock = kCand * 128;              // one 64-element K block of the candidates
-constexpr int kGramStride = kCand + 4;            // floats per Gram row (bank spread)
+// floats per Gram row: an odd stride keeps both the row-per-lane copy and
+// the replay's column reads (lane = candidate) free of bank conflicts
+constexpr int kGramStride = kCand + 1;
 constexpr int kListMax = 512;                     // threshold-bin keys ranked directly
 constexpr int kPassBelow = 24;                    // a round with fewer picks is followed by a pass
 constexpr int kAhead = 12;                        // L2 prefetch distance of a pass, in tiles
@@ -187,6 +190,37 @@ struct WindowTiles {
   }
 };
 
+// ---- loads under an L2 cache policy
+// A 2-D tiled TMA load (as tma_load_2d) under an L2 cache policy.
+__device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const CUtensorMap *map,
+                                                 uint32_t bar, int32_t x, int32_t y,
+                                                 uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "l"(policy)
+      : "memory");
+}
+
+// Policies for tma_load_2d_hint: lines kept in L2 with evict-last priority,
+// or evicted first.
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t policy;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(policy));
+  return policy;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t policy;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(policy));
+  return policy;
+}
+// Return the 128-byte L2 line holding `p` to normal eviction priority.
+__device__ __forceinline__ void l2_demote_line(const void *p) {
+  asm volatile("applypriority.global.L2::evict_normal [%0], 128;" ::"l"(
+                   reinterpret_cast<uint64_t>(p) & ~static_cast<uint64_t>(127))
+               : "memory");
+}
+
 __device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
@@ -226,11 +260,14 @@ __device__ __forceinline__ void prefetch_row(const Head &h, const FpsGeom &g, in
 }
 
 // Issue the TMA loads of tiles [0, n_tiles) of the pass that starts at
-// sequence number `seq` (producer thread only).  Returns false after a timeout.
+// sequence number `seq` (producer thread only): tiles below n_keep stay in
+// L2 (evict-last), the rest stream through it (evict-first).  Returns false
+// after a timeout.
 __device__ bool issue_tiles(const Layout &s, const CUtensorMap *bmap, const CUtensorMap *wmap,
                             int qh, const FpsGeom &g, int n_btiles, int w_first, uint32_t seq,
-                            int n_tiles) {
+                            int n_tiles, int n_keep) {
   const uint32_t full0 = smem_u32(&s.bars[kBarFull]), empty0 = smem_u32(&s.bars[kBarEmpty]);
+  const uint64_t keep = l2_policy_evict_last(), stream = l2_policy_evict_first();
   auto map_of = [&](int j) { return j < n_btiles ? bmap : wmap; };
   auto row_of = [&](int j) {
     return j < n_btiles ? qh * g.M + j * kTileRows
@@ -243,8 +280,9 @@ __device__ bool issue_tiles(const Layout &s, const CUtensorMap *bmap, const CUte
     const uint32_t dst = smem_u32(s.ring + st * kTileBytes);
     const CUtensorMap *map = map_of(j);
     const int y = row_of(j);
-    tma_load_2d(dst, map, full0 + 8 * st, 0, y);
-    tma_load_2d(dst + kTileRows * 128, map, full0 + 8 * st, 64, y);
+    const uint64_t policy = j < n_keep ? keep : stream;
+    tma_load_2d_hint(dst, map, full0 + 8 * st, 0, y, policy);
+    tma_load_2d_hint(dst + kTileRows * 128, map, full0 + 8 * st, 64, y, policy);
   }
   return true;
 }
@@ -277,13 +315,14 @@ __device__ __forceinline__ float chunk_min(const float (&v)[32], const float *pi
 __device__ void distance_pass(const Layout &s, const CUtensorMap *bmap, const CUtensorMap *wmap,
                               uint32_t tmem, int qh, const Head &h, const FpsGeom &g,
                               int n_btiles, int w_first, int n_tiles, uint32_t seq, int s0, int P,
-                              bool first) {
+                              bool first, int n_keep) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t full0 = smem_u32(&s.bars[kBarFull]), empty0 = smem_u32(&s.bars[kBarEmpty]);
   const uint32_t tfull0 = smem_u32(&s.bars[kBarTfull]), tempty0 = smem_u32(&s.bars[kBarTempty]);
   const int N = (P - s0 + 15) & ~15;  // 16 .. 128
   if (warp == 0) {
-    if (lane == 0 && !issue_tiles(s, bmap, wmap, qh, g, n_btiles, w_first, seq, n_tiles))
+    if (lane == 0 &&
+        !issue_tiles(s, bmap, wmap, qh, g, n_btiles, w_first, seq, n_tiles, n_keep))
       s.scal[kAbort] = 1;
   } else if (warp == 1 || warp == 2) {
     if (lane == 0) {
@@ -708,7 +747,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   const FpsGeom g, const __nv_bfloat16 *__restrict__ beacons_in,
                   const __nv_bfloat16 *__restrict__ window, __nv_bfloat16 *__restrict__ beacons_out,
                   int n_qheads, uint8_t *__restrict__ garrays, size_t slice_bytes,
-                  int *__restrict__ head_counter) {
+                  int *__restrict__ head_counter, float l2_keep) {
   extern __shared__ uint8_t smem_raw[];
   const int n = g.nb_in + g.W;
   const int m = g.n_pick;
@@ -743,6 +782,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_btiles = (g.nb_in + kTileRows - 1) / kTileRows;
   const WindowTiles wt(g);
   const int n_tiles = n_btiles + wt.count;
+  // the passes keep the union's first n_keep tiles in L2 (l2_keep: the share
+  // of each union the launch can keep, from launch_fps_tc)
+  const int n_keep = min(n_tiles, static_cast<int>(l2_keep * n_tiles + 0.5f));
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) {
       mbar_init(smem_u32(&s.bars[kBarFull + i]), 1);
@@ -809,7 +851,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int b = tid; b < kUBins; b += kThreads) s.uhist[b] = 0u;
     fence_proxy_async_smem();
     __syncthreads();
-    distance_pass(s, &bmap, &wmap, tmem, qh, h, g, n_btiles, wt.first, n_tiles, seq, 0, 1, true);
+    distance_pass(s, &bmap, &wmap, tmem, qh, h, g, n_btiles, wt.first, n_tiles, seq, 0, 1, true,
+                  n_keep);
     seq += n_tiles;
     __syncthreads();
     if (s.scal[kAbort]) break;
@@ -954,9 +997,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               tmem_ld_wait_regs(x);
               if (a < nc) {
 #pragma unroll
-                for (int b = 0; b < 32; b += 4)
-                  *reinterpret_cast<float4 *>(row + c0 + b) =
-                      make_float4(x[b], x[b + 1], x[b + 2], x[b + 3]);
+                for (int b = 0; b < 32; ++b) row[c0 + b] = x[b];
               }
             }
           } else {
@@ -1120,13 +1161,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncthreads();
       if (eager) {
         distance_pass(s, &bmap, &wmap, tmem, qh, h, g, n_btiles, wt.first, n_tiles, seq, E & ~7, P,
-                      false);
+                      false, n_keep);
         seq += n_tiles;
         __syncthreads();
         if (s.scal[kAbort]) break;
         E = P;
         dmax = __uint_as_float(static_cast<uint32_t>(s.scal[kSKeyMax]) & 0x7fffffffu);
       }
+    }
+    // the kept tiles' lines return to normal priority, so that a finished
+    // union does not hold L2 against the next heads or kernels (a hint only:
+    // rows of a tile past the head's own are left as they are)
+    for (int t = tid; t < 2 * n_keep * kTileRows; t += kThreads) {
+      const int j = t / (2 * kTileRows), r = (t >> 1) % kTileRows;
+      const __nv_bfloat16 *row = nullptr;
+      if (j < n_btiles) {
+        if (j * kTileRows + r < h.nb) row = h.B + static_cast<size_t>(j * kTileRows + r) * kDim;
+      } else {
+        const long long slot = static_cast<long long>(wt.first + j - n_btiles) * kTileRows + r;
+        if (slot < h.w_cap) row = h.Wp + static_cast<size_t>(slot) * kDim;
+      }
+      if (row != nullptr) l2_demote_line(reinterpret_cast<const uint8_t *>(row) + (t & 1) * 128);
     }
     if (s.scal[kAbort] || stuck) break;
   }
@@ -1174,6 +1229,21 @@ size_t smem_bytes(const FpsGeom &g) {
 }
 
 int fps_tc_grid(const FpsGeom &g) { return std::min(g.n_layers * g.n_q_heads, kMaxCtas); }
+
+// L2 held by the unions of the heads in flight: each CTA keeps its share of
+// it (the first tiles of its union) across the passes and streams the rest.
+// With 148 unions of 1.08 MB (128 beacons + a 4096-query window) a cyclic
+// stream through L2 under the default policy keeps little between passes;
+// keeping a fixed ~40% of each union (64 MB in all) measured 2.36 ms
+// against 2.455 ms for the 40-layer launch, and larger shares less (0.55:
+// 2.37, 0.7: 2.43, all: 2.455 ms), as the kept lines push each other out.
+constexpr double kL2KeepBytes = 64.0 * (1 << 20);
+float l2_keep_fraction(const FpsGeom &g, int grid) {
+  const double union_bytes = (static_cast<double>(g.nb_in) + g.W) * kDim * 2;
+  if (union_bytes <= 0) return 1.f;
+  const double f = kL2KeepBytes / (grid * union_bytes);
+  return static_cast<float>(std::min(1.0, std::max(1.0 / 64, f)));
+}
 
 }  // namespace
 
@@ -1225,7 +1295,7 @@ bkv_status launch_fps_tc(const FpsGeom &g, const void *beacons_in, const void *w
   fps_tc_kernel<<<grid, kThreads, smem, stream>>>(
       bmap, wmap, g, static_cast<const __nv_bfloat16 *>(beacons_in),
       static_cast<const __nv_bfloat16 *>(window), static_cast<__nv_bfloat16 *>(beacons_out),
-      n_qheads, arrays, union_array_bytes(g), counter);
+      n_qheads, arrays, union_array_bytes(g), counter, l2_keep_fraction(g, grid));
   return cudaGetLastError() == cudaSuccess ? BKV_OK : BKV_ERR_CUDA;
 }
 
