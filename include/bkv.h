@@ -156,7 +156,8 @@ bkv_status bkv_compact(const bkv_cache_desc *src, const void *k_src,
  *        positions does (bkv_select_topk's output, for one).  A row breaking
  *        this is skipped and reported as BKV_ERR_DEVICE_ASSERT by
  *        bkv_read_device_status; rows already in place are not copied.
- *   v may be NULL to compact only the keys.  Rows are at most 32 KB.
+ *   v may be NULL to compact only the keys.  Rows are at most 16 KB
+ *   (BKV_ERR_UNSUPPORTED past that).
  * Requires 0 <= n_keep <= capacity. */
 bkv_status bkv_compact_inplace(const bkv_cache_desc *desc, void *k, void *v,
                                const int32_t *idx, int64_t n_keep, void *stream);

@@ -11,13 +11,13 @@
 //
 // In place (the destination is the source cache): row i takes row idx_i with
 // idx_i >= i, which holds for any ascending list of kept positions.  One CTA
-// per (head, K or V) walks its rows in chunks in increasing i; a chunk
-// is read whole into registers, the CTA synchronises, then it is written.
-// A row read by chunk c lies at or past the chunk's first row, so it is
-// either in chunk c (written only after the barrier) or in a later chunk
-// (written only after chunk c's reads have returned); rows written by chunk c
-// lie before every row a later chunk reads.  Rows already in place are
-// skipped.  A chunk is at most 32 KB (128 rows of 256 bytes).
+// per (head, K or V) walks its rows in chunks in increasing i; a chunk is
+// read whole into registers, the CTA synchronises, then it is written.  A
+// row read by chunk c lies at or past the chunk's
+// first row, so it is either in chunk c (written only after the barrier) or
+// in a later chunk (written only after chunk c's reads have returned); rows
+// written by chunk c lie before every row a later chunk reads.  Rows already
+// in place are skipped.  A chunk is at most 32 KB (128 rows of 256 bytes).
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -88,40 +88,91 @@ __global__ void __launch_bounds__(kThreads) compact_kernel(const CompactArgs a) 
 }
 
 constexpr int kInplaceThreads = 256;
-constexpr int kInplacePer = 8;  // 16-byte pieces per thread and chunk
+constexpr int kInplacePer = 8;  // 16-byte pieces per thread and chunk (32 KB chunks)
+constexpr int kInplaceMaxRows = kInplacePer * kInplaceThreads;  // rows per chunk, 16-byte rows
+// CTAs resident per SM: every (head, K or V) of a step runs at once up to
+// 5 x 148 = 740 of them (640 at the 14B shape).  A CTA walks its head's
+// chunks in order, so a CTA left for a second wave would take the whole
+// head's time again; at 4 per SM (62 registers) the 14B shape's 640 CTAs
+// took 0.59 ms against 0.33 ms for the out-of-place copy.
+constexpr int kInplaceCtasPerSm = 5;
 
-__global__ void __launch_bounds__(kInplaceThreads) compact_inplace_kernel(const CompactArgs a) {
+// Each chunk is read whole into registers, the CTA synchronises, and the
+// chunk is written.  The kept positions of the next chunk are fetched into
+// shared memory while the chunk's rows are in flight, so a chunk waits for
+// one load latency rather than two (position, then row).  kChunks: the
+// number of 16-byte pieces per row when the kernel is built for it (it
+// divides the CTA's threads, so each thread keeps one piece column and its
+// rows are a fixed stride apart, and a head's slice is below 4 GB, so byte
+// offsets within it take 32 bits); 0 for any row size.
+template <int kChunks>
+__global__ void __launch_bounds__(kInplaceThreads, kInplaceCtasPerSm)
+    compact_inplace_kernel(const CompactArgs a) {
+  constexpr bool kEven = kChunks > 0;
+  static_assert(!kEven || kInplaceThreads % kChunks == 0, "pieces must divide the threads");
+  __shared__ int32_t s_idx[2][kInplaceMaxRows];
   const int head = blockIdx.x;
   uint8_t *base = (blockIdx.y == 0 ? a.k_dst : a.v_dst) + static_cast<size_t>(head) * a.dst_cap * a.row_bytes;
   const int32_t *idx = a.idx + static_cast<size_t>(head) * a.n_keep;
-  const int chunks = a.row_bytes >> 4;  // 16-byte pieces per row
+  // kept positions are int32, so every row index fits in 32 bits (the
+  // launcher checks n_keep and the capacity)
+  const int n_keep = static_cast<int>(a.n_keep), cap = static_cast<int>(a.dst_cap);
+  const int chunks = kEven ? kChunks : a.row_bytes >> 4;  // 16-byte pieces per row
   const int rows = kInplacePer * kInplaceThreads / chunks;  // rows per chunk
   const int per_chunk = rows * chunks;
-  for (long long i0 = 0; i0 < a.n_keep; i0 += rows) {
+  // piece u of this thread: row ri(u) of the chunk, 16-byte column col(u)
+  auto ri = [&](int u) {
+    return kEven ? static_cast<int>(threadIdx.x) / kChunks + u * (kInplaceThreads / kChunks)
+                 : (static_cast<int>(threadIdx.x) + u * kInplaceThreads) / chunks;
+  };
+  auto col = [&](int u) {
+    return kEven ? static_cast<int>(threadIdx.x) % kChunks
+                 : (static_cast<int>(threadIdx.x) + u * kInplaceThreads) % chunks;
+  };
+  for (int r = threadIdx.x; r < rows; r += kInplaceThreads)
+    if (r < n_keep) s_idx[0][r] = idx[r];
+  __syncthreads();
+  int buf = 0;
+  for (int i0 = 0; i0 < n_keep; i0 += rows, buf ^= 1) {
     uint4 v[kInplacePer];
-    long long dst[kInplacePer];
+    uint32_t moved = 0u;  // bit u: piece u is read here and written below
+    bool bad = false;     // a kept position below its slot or past the cache
 #pragma unroll
     for (int u = 0; u < kInplacePer; ++u) {
-      const int e = threadIdx.x + u * kInplaceThreads;
-      dst[u] = -1;
-      if (e >= per_chunk) continue;
-      const long long i = i0 + e / chunks;
-      if (i >= a.n_keep) continue;
-      const int c = e % chunks;
-      const long long src = idx[i];
-      if (src < i || src >= a.dst_cap) {
-        if (c == 0) record_device_status(BKV_DEV_ASSERT, 501);
+      if (!kEven && static_cast<int>(threadIdx.x) + u * kInplaceThreads >= per_chunk) continue;
+      const int i = i0 + ri(u);
+      if (i >= n_keep) continue;
+      const int src = s_idx[buf][ri(u)];
+      if (src < i || src >= cap) {
+        bad = true;
         continue;
       }
       if (src == i) continue;  // already in place
       // L2-coherent load: this kernel writes the same buffer
-      v[u] = __ldcg(reinterpret_cast<const uint4 *>(base + src * a.row_bytes + c * 16));
-      dst[u] = i * a.row_bytes + c * 16;
+      const size_t off =
+          kEven ? static_cast<size_t>(static_cast<uint32_t>(src) * (kChunks * 16u) +
+                                      static_cast<uint32_t>(col(u) * 16))
+                : static_cast<size_t>(src) * a.row_bytes + col(u) * 16;
+      v[u] = __ldcg(reinterpret_cast<const uint4 *>(base + off));
+      moved |= 1u << u;
     }
+    // the next chunk's positions (the other buffer was last read before the
+    // previous barrier)
+    for (int r = threadIdx.x; r < rows; r += kInplaceThreads)
+      if (i0 + rows + r < n_keep) s_idx[buf ^ 1][r] = idx[i0 + rows + r];
     __syncthreads();
 #pragma unroll
-    for (int u = 0; u < kInplacePer; ++u)
-      if (dst[u] >= 0) __stcg(reinterpret_cast<uint4 *>(base + dst[u]), v[u]);
+    for (int u = 0; u < kInplacePer; ++u) {
+      if (!((moved >> u) & 1u)) continue;
+      const int i = i0 + ri(u);
+      const size_t off =
+          kEven ? static_cast<size_t>(static_cast<uint32_t>(i) * (kChunks * 16u) +
+                                      static_cast<uint32_t>(col(u) * 16))
+                : static_cast<size_t>(i) * a.row_bytes + col(u) * 16;
+      __stcg(reinterpret_cast<uint4 *>(base + off), v[u]);
+    }
+    // reported once the chunk's data is out of registers
+    if (bad) record_device_status(BKV_DEV_ASSERT, 501);
   }
 }
 
@@ -131,9 +182,17 @@ bkv_status launch_compact_inplace(const CompactArgs &a, cudaStream_t stream) {
   if (injected_launch_failure()) return BKV_ERR_CUDA;
   if (a.n_keep == 0 || a.n_heads == 0) return BKV_OK;
   if (a.row_bytes < 16 || a.row_bytes > 16 * kInplacePer * kInplaceThreads) return BKV_ERR_UNSUPPORTED;
+  if (a.dst_cap > INT32_MAX || a.n_keep > a.dst_cap) return BKV_ERR_INVALID_ARG;
   dim3 grid(static_cast<unsigned>(a.n_heads), a.v_dst != nullptr ? 2u : 1u);
   if (a.k_dst == nullptr) return BKV_ERR_INVALID_ARG;
-  compact_inplace_kernel<<<grid, kInplaceThreads, 0, stream>>>(a);
+  const bool off32 = static_cast<unsigned long long>(a.dst_cap) * a.row_bytes <= 0xffffffffull;
+  switch (off32 ? a.row_bytes : 0) {
+    case 128: compact_inplace_kernel<8><<<grid, kInplaceThreads, 0, stream>>>(a); break;
+    case 256: compact_inplace_kernel<16><<<grid, kInplaceThreads, 0, stream>>>(a); break;
+    case 512: compact_inplace_kernel<32><<<grid, kInplaceThreads, 0, stream>>>(a); break;
+    case 1024: compact_inplace_kernel<64><<<grid, kInplaceThreads, 0, stream>>>(a); break;
+    default: compact_inplace_kernel<0><<<grid, kInplaceThreads, 0, stream>>>(a); break;
+  }
   return cudaGetLastError() == cudaSuccess ? BKV_OK : BKV_ERR_CUDA;
 }
 

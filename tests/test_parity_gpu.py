@@ -455,8 +455,8 @@ def _ascending_positions(rng, cap, n_keep, mode):
     ("bf16", 128, 4096, 1537, "prefix_kept"),
     ("bf16", 128, 777, 777, "random"),        # every row kept: nothing moves
     ("bf16", 128, 5000, 129, "tail"),
-    ("f32", 128, 2000, 1000, "random"),       # 512-byte rows: 64-row chunks
-    ("f32", 24, 999, 400, "prefix_kept"),     # 96-byte rows: chunks of 341 rows
+    ("f32", 128, 2000, 1000, "random"),       # 512-byte rows: 32-row chunks
+    ("f32", 24, 999, 400, "prefix_kept"),     # 96-byte rows: chunks of 170 rows
 ])
 def test_compact_inplace(dtype, d, cap, n_keep, mode, dev):
     """In-place compaction equals the out-of-place gather, byte for byte."""
