@@ -168,7 +168,9 @@ SelectInput score_select_input(const ScoreGeom &g, int dtype, const ScoreWorkspa
                                bool mean) {
   SelectInput in;
   in.src = w.ypart;
-  in.n_parts = mean && dtype == BKV_BF16 ? mean_grouping(g).n_groups : g.n_groups;
+  // the tensor-core max aggregation leaves its groups merged, as order keys
+  in.keys = !mean && dtype == BKV_BF16 ? 1 : 0;
+  in.n_parts = in.keys ? 1 : mean && dtype == BKV_BF16 ? mean_grouping(g).n_groups : g.n_groups;
   in.part_stride = static_cast<size_t>(g.n_heads()) * static_cast<size_t>(g.L);
   in.mean = mean ? 1 : 0;
   in.inv_count = 1.0f / static_cast<float>(g.n_obs);

@@ -51,8 +51,9 @@ inline ScoreGeom mean_grouping(const ScoreGeom &g) {
 // Workspace sections of the scoring passes.
 struct ScoreWorkspace {
   float *c;      // [n_heads][n_obs_pad]  row normalisers (natural log units)
-  float *ypart;  // [groups][n_heads][L] per group of rows: max of (x - c)
-                 // (max aggregation) or sum of exp(x - c) (mean aggregation);
+  float *ypart;  // max aggregation (tensor cores): [n_heads][L] order keys of
+                 // max_o (x - c), every group merged; otherwise [groups][n_heads][L]
+                 // per group of rows: max of (x - c) or sum of exp(x - c) (mean);
                  // sized for the mean's (finer) grouping
 };
 size_t score_workspace_bytes(const ScoreGeom &g);
@@ -86,6 +87,7 @@ struct SelectInput {
   size_t part_stride;
   int mean;
   float inv_count;
+  int keys = 0;  // src holds one part of order keys (order_key.cuh) as 32-bit words
 };
 size_t select_workspace_bytes(int n_rows, long long L);
 bkv_status launch_select_topk(const SelectInput &in, int n_rows, long long L, long long K,

@@ -17,9 +17,12 @@
 //     K=16 step of the same MMA: every key carries a block (1, 1, 1, 0, ...)
 //     and every observation row (-c_hi, -c_mid, -c_lo, 0, ...), the three
 //     bf16 parts of c_o / scale.  TMEM lane = key, so each epilogue thread owns
-//     one key and takes the max over its columns in registers.  The mean
-//     variant sums exp(scale * acc) over the columns instead (s_j is that sum
-//     over all rows divided by their count).
+//     one key and takes the max over its columns in registers.  The groups of
+//     rows (CTAs) of a head meet in one row of order keys (order_key.cuh): an
+//     unsigned max in L2, so the top-K select reads one word per key instead
+//     of one per group.  The mean variant sums exp(scale * acc) over the
+//     columns instead (s_j is that sum over all rows divided by their count),
+//     one partial row per group.
 //
 // Both passes: warp 0 issues TMA loads of the key tiles (128-byte swizzle, no
 // multicast) into a ring of shared-memory stages; warp 1 allocates TMEM and
@@ -37,6 +40,7 @@
 #include <mutex>
 
 #include "bkv_internal.h"
+#include "order_key.cuh"
 #include "sm100.cuh"
 #include "tma_host.h"
 
@@ -658,7 +662,9 @@ __global__ void __launch_bounds__(p2_threads(kMean), 1)
     const int row = quarter * 32 + lane;  // key within the tile
     const int n_active = n_sub * kSplit;  // warpgroups with columns to read
     const float kz = g.scale * kLog2e;
-    float *yout = ypart + (static_cast<size_t>(gi) * g.n_heads() + head) * static_cast<size_t>(L);
+    // the head's merged maxima, as order keys: stored by a single group, else
+    // combined by an unsigned max in L2 over a row of zeros (below every key)
+    uint32_t *ykey = reinterpret_cast<uint32_t *>(ypart) + static_cast<size_t>(head) * static_cast<size_t>(L);
     if (u < n_sub) {
       const int Nu = u == 0 ? N0 : N1;
       const int n32 = Nu >> 5;
@@ -666,7 +672,7 @@ __global__ void __launch_bounds__(p2_threads(kMean), 1)
       const bool tail16 = (Nu & 16) && (n32 % kSplit) == h;  // Nu is a multiple of 16
       bool ok = true;  // warp-uniform; after a timeout only the barriers remain
       for (int it = 0; it < n_tiles; ++it) {
-        float y0 = kMean ? 0.f : -INFINITY, y1 = y0;
+        float y0 = -INFINITY, y1 = y0;
         if (ok && !mbar_wait_warp(tfull0 + 8 * u, it & 1, kWhereP2Epi)) ok = false;
         if (ok) {
           tc_fence_after();
@@ -732,7 +738,13 @@ __global__ void __launch_bounds__(p2_threads(kMean), 1)
         }
         if (e == 0 && ok) {
           const long long j = static_cast<long long>(t0 + it) * kP2Keys + row;
-          if (j < L) yout[j] = kMean ? y : y * g.scale;
+          const float v = y * g.scale;
+          if (j < L) {
+            if (g.n_groups == 1)
+              ykey[j] = order_key(v);
+            else if (!(v != v))  // a NaN group maximum is ignored, as fmaxf would
+              atomicMax(ykey + j, order_key(v));
+          }
         }
       }
     }
@@ -831,6 +843,12 @@ bkv_status launch_score_colmax_tc(const ScoreGeom &g, const void *k, const void 
   const long long grid = units * n_chunks;
   const auto *rq = static_cast<const uint16_t *>(recent);
   const auto *bq = static_cast<const uint16_t *>(beacons);
+  // the max form's groups meet in one row of keys per head, zero to start
+  if (!mean && g.n_groups > 1 &&
+      cudaMemsetAsync(ypart + static_cast<size_t>(head0) * static_cast<size_t>(g.L), 0,
+                      static_cast<size_t>(head_count) * static_cast<size_t>(g.L) * sizeof(float),
+                      stream) != cudaSuccess)
+    return BKV_ERR_CUDA;
   if (mean)
     score_colmax_kernel<true><<<static_cast<unsigned>(grid), p2_threads(true), smem, stream>>>(
         map, g, rq, bq, c, ypart, n_chunks, chunk_tiles, stages, head0);

@@ -4,8 +4,9 @@
 // One CTA per row (a (layer, KV head)); scores become order-preserving
 // unsigned keys (larger score -> larger key; -0 and +0 map to one key).  The
 // row is never staged whole: each pass re-reads it (from HBM the first time,
-// L2 after) and rebuilds the keys -- for the step's max form that also
-// merges the observation groups' partial maxima.
+// L2 after) and rebuilds the keys -- for a mean, or for partials of several
+// observation groups, that also merges the groups.  The tensor-core max
+// aggregation hands over the keys already merged (one word per position).
 //
 // The common path (rows of a multiple of 4 keys, 16-byte aligned, at most
 // 65536 of them) reads the row twice and does the rest in shared memory:
@@ -33,6 +34,7 @@
 #include "bkv_check.cuh"
 #include "bkv_device_status.cuh"
 #include "bkv_internal.h"
+#include "order_key.cuh"
 
 BKV_DEFINE_STATUS_ACCESSOR(take_status_select)
 
@@ -50,15 +52,8 @@ constexpr int mask_smem_bytes(long long L) {
   return static_cast<int>((kTopBins + 2 * kListCap + 2 * ((L + 127) / 128 * 4)) * 4);
 }
 
-__device__ __forceinline__ uint32_t order_key(float f) {
-  // f + 0 is +0 for f = -0 (round to nearest) and f otherwise; then the
-  // sign's arithmetic shift flips all bits of a negative and only the sign
-  // bit of a positive
-  const uint32_t u = __float_as_uint(f + 0.f);
-  return u ^ (static_cast<uint32_t>(static_cast<int32_t>(u) >> 31) | 0x80000000u);
-}
-
 __device__ __forceinline__ float load_key_value(const SelectInput &in, size_t off) {
+  if (in.keys) return key_value(reinterpret_cast<const uint32_t *>(in.src)[off]);
   float v = in.src[off];
   if (in.mean) {
     for (int p = 1; p < in.n_parts; ++p) v += in.src[p * in.part_stride + off];
@@ -76,6 +71,10 @@ __device__ __forceinline__ float score_of_key(const SelectInput &in, float v) {
 // Four consecutive values of a row (off a multiple of 4, the row 16-byte
 // aligned), merged over the parts like load_key_value.
 __device__ __forceinline__ float4 load_key_value4(const SelectInput &in, size_t off) {
+  if (in.keys) {
+    const uint4 k = *reinterpret_cast<const uint4 *>(in.src + off);
+    return make_float4(key_value(k.x), key_value(k.y), key_value(k.z), key_value(k.w));
+  }
   float4 v = *reinterpret_cast<const float4 *>(in.src + off);
   for (int p = 1; p < in.n_parts; ++p) {
     const float4 w = *reinterpret_cast<const float4 *>(in.src + p * in.part_stride + off);
@@ -324,25 +323,31 @@ __global__ void __launch_bounds__(kThreads)
 }
 
 // Four consecutive merged values at p (16-byte aligned), with the part count
-// fixed at compile time (kP > 0) or read from the input (kP == 0).
+// fixed at compile time (kP > 0) or read from the input (kP == 0); kP < 0:
+// the row holds the merged order keys themselves.
 template <int kP, bool kMean>
 __device__ __forceinline__ float4 merged4(const SelectInput &in, const float *p) {
-  float4 v = *reinterpret_cast<const float4 *>(p);
-  const int np = kP > 0 ? kP : in.n_parts;
+  if constexpr (kP < 0) {
+    const uint4 k = *reinterpret_cast<const uint4 *>(p);
+    return make_float4(key_value(k.x), key_value(k.y), key_value(k.z), key_value(k.w));
+  } else {
+    float4 v = *reinterpret_cast<const float4 *>(p);
+    const int np = kP > 0 ? kP : in.n_parts;
 #pragma unroll
-  for (int q = 1; q < (kP > 0 ? kP : 64); ++q) {
-    if (kP == 0 && q >= np) break;
-    const float4 w = *reinterpret_cast<const float4 *>(p + q * in.part_stride);
-    if constexpr (kMean) {
-      v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
-    } else {
-      v.x = fmaxf(v.x, w.x); v.y = fmaxf(v.y, w.y); v.z = fmaxf(v.z, w.z); v.w = fmaxf(v.w, w.w);
+    for (int q = 1; q < (kP > 0 ? kP : 64); ++q) {
+      if (kP == 0 && q >= np) break;
+      const float4 w = *reinterpret_cast<const float4 *>(p + q * in.part_stride);
+      if constexpr (kMean) {
+        v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
+      } else {
+        v.x = fmaxf(v.x, w.x); v.y = fmaxf(v.y, w.y); v.z = fmaxf(v.z, w.z); v.w = fmaxf(v.w, w.w);
+      }
     }
+    if constexpr (kMean) {
+      v.x *= in.inv_count; v.y *= in.inv_count; v.z *= in.inv_count; v.w *= in.inv_count;
+    }
+    return v;
   }
-  if constexpr (kMean) {
-    v.x *= in.inv_count; v.y *= in.inv_count; v.z *= in.inv_count; v.w *= in.inv_count;
-  }
-  return v;
 }
 
 // The common path: two streaming passes, then shared memory only (see the
@@ -423,35 +428,21 @@ __global__ void __launch_bounds__(kThreads, 3)
       const int q = base + u * kThreads + lane;
       if (q < L4) a[u] = merged4<kP, kMean>(in, src + 4 * q);
     }
+    // the mask words of all U steps first (no branch between them, so their
+    // shuffles overlap), then one vote for the rare listing of the bin's keys
+    uint32_t kq[U][4];
+    uint32_t inb = 0u;  // bit 4u + e: key e of step u lies in the threshold bin
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int q = base + u * kThreads + lane;
+      const uint4 k4 = q < L4 ? keys_of(a[u]) : make_uint4(0u, 0u, 0u, 0u);
+      kq[u][0] = k4.x; kq[u][1] = k4.y; kq[u][2] = k4.z; kq[u][3] = k4.w;
       uint32_t nib = 0u;
-      uint32_t k[4] = {0u, 0u, 0u, 0u};
-      bool in_bin_any = false;
-      if (q < L4) {
-        const uint4 k4 = keys_of(a[u]);
-        k[0] = k4.x; k[1] = k4.y; k[2] = k4.z; k[3] = k4.w;
-        // above the bin: key > key_top; in it: key - key_lo < bin width
+      // above the bin: key > key_top; in it: key - key_lo < bin width
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          nib |= (k[e] > key_top ? 1u : 0u) << e;
-          in_bin_any |= k[e] - key_lo < (1u << (32 - kTopBits));
-        }
-      }
-      if (__any_sync(0xffffffffu, in_bin_any)) {  // about 2% of keys: rare per warp step
-        if (in_bin_any) {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            if (k[e] - key_lo < (1u << (32 - kTopBits))) {
-              const int p = atomicAdd(&n_list, 1);
-              if (p < kListCap) {
-                lkey[p] = k[e];
-                lpos[p] = static_cast<uint32_t>(4 * q + e);
-              }
-            }
-          }
-        }
+      for (int e = 0; e < 4; ++e) {
+        nib |= (kq[u][e] > key_top ? 1u : 0u) << e;
+        if (q < L4 && kq[u][e] - key_lo < (1u << (32 - kTopBits))) inb |= 1u << (4 * u + e);
       }
       uint32_t word = nib << (4 * (lane & 7));
       word |= __shfl_xor_sync(0xffffffffu, word, 1);
@@ -459,6 +450,21 @@ __global__ void __launch_bounds__(kThreads, 3)
       word |= __shfl_xor_sync(0xffffffffu, word, 4);
       const int wi = (base + u * kThreads + lane) >> 3;
       if ((lane & 7) == 0 && wi < n_words) mask[wi] = word;
+    }
+    if (inb != 0u) {  // the threshold bin's keys: a few percent of a row, up to ~11%
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if ((inb >> (4 * u + e)) & 1u) {
+            const int p = atomicAdd(&n_list, 1);
+            if (p < kListCap) {
+              lkey[p] = kq[u][e];
+              lpos[p] = static_cast<uint32_t>(4 * (base + u * kThreads + lane) + e);
+            }
+          }
+        }
+      }
     }
   }
   __syncthreads();
@@ -571,7 +577,7 @@ bkv_status launch_select_topk(const SelectInput &in, int n_rows, long long L, lo
                    (reinterpret_cast<uintptr_t>(s_out) & 15u) == 0;
   if (vec && L <= kMaskMaxL) {
     const int smem = mask_smem_bytes(L);
-    const int parts = in.n_parts >= 1 && in.n_parts <= 4 ? in.n_parts : 0;
+    const int parts = in.keys ? -1 : in.n_parts >= 1 && in.n_parts <= 4 ? in.n_parts : 0;
     bkv_status st = BKV_OK;
     auto run = [&](auto kernel, int *attr_done) {
       if (!ensure_smem_limit(kernel, mask_smem_bytes(kMaskMaxL), attr_done)) {
@@ -581,7 +587,7 @@ bkv_status launch_select_topk(const SelectInput &in, int n_rows, long long L, lo
       kernel<<<n_rows, kThreads, smem, stream>>>(in, static_cast<int>(L), static_cast<int>(K),
                                                  idx, s_out);
     };
-    static int done[10][64];
+    static int done[11][64];
     if (in.mean) {
       switch (parts) {
         case 1: run(select_topk_mask_kernel<1, true>, done[0]); break;
@@ -592,6 +598,7 @@ bkv_status launch_select_topk(const SelectInput &in, int n_rows, long long L, lo
       }
     } else {
       switch (parts) {
+        case -1: run(select_topk_mask_kernel<-1, false>, done[10]); break;
         case 1: run(select_topk_mask_kernel<1, false>, done[5]); break;
         case 2: run(select_topk_mask_kernel<2, false>, done[6]); break;
         case 3: run(select_topk_mask_kernel<3, false>, done[7]); break;
