@@ -82,14 +82,17 @@ def load_traffic():
 # ----------------------------------------------------------------------------
 # algorithmic work per phase (per step, one rank)
 # ----------------------------------------------------------------------------
-def work_model(wl):
+def work_model(wl, aggregate="max"):
     H = wl.n_layers * wl.n_kv_heads
     Hq = wl.n_layers * wl.n_q_heads
     nb = min(wl.M, wl.beacons_in + wl.W) if wl.W else wl.beacons_in
     n_obs = wl.group * (wl.R + nb)
     d, L, K = wl.head_dim, wl.L, min(wl.K, wl.L)
     es = 2 if wl.dtype == "bf16" else 4
-    n_groups = (n_obs + 511) // 512
+    # the words the select streams per key: one (the max form's merged order
+    # key, or the CUDA-core path's single partial), else one partial per
+    # group of at most 256 observation rows (the tensor-core mean)
+    n_parts = (n_obs + 255) // 256 if aggregate == "mean" and wl.dtype == "bf16" else 1
     contraction = 2.0 * n_obs * L * d * H
     fps_fma = float(Hq) * wl.M * (wl.beacons_in + wl.W) * d
     return {
@@ -100,7 +103,7 @@ def work_model(wl):
         "fps_fma": fps_fma,
         "row_stats": {"bound": "tensor", "work": contraction, "unit": "FLOP"},
         "aggregate": {"bound": "tensor", "work": contraction, "unit": "FLOP"},
-        "select": {"bound": "hbm", "work": float(H) * (n_groups * 4 * L + 4 * K), "unit": "B"},
+        "select": {"bound": "hbm", "work": float(H) * (n_parts * 4 * L + 4 * K), "unit": "B"},
         "compact": {"bound": "hbm", "work": float(H) * 4 * K * d * es, "unit": "B"},
         # the step: one contraction + the algorithmic bytes of the whole step
         "step_flop": contraction,
@@ -674,7 +677,7 @@ def main():
         return
 
     peaks = load_peaks()
-    wm = work_model(wl)
+    wm = work_model(wl, args.aggregate)
     # the captured counters are those of the default configuration
     traffic = (load_traffic() if args.workload == "qwen3_14b" and not args.layers
                and args.aggregate == "max" and not args.in_place else {})
