@@ -51,6 +51,8 @@ SCORE_CASES = {
     "ragged_bf16": lambda: small(n_layers=2),
     "row_blocks": lambda: small(n_q_heads=16, R=24, M=20, n_beacons_in=20, L=777, K=100),
     "two_groups": lambda: small(n_q_heads=16, R=40, M=40, n_beacons_in=40, L=513, K=64),
+    # 1152 observation rows: three groups meet in the max aggregation's row of keys
+    "three_groups": lambda: small(n_q_heads=16, R=64, M=80, n_beacons_in=80, L=700, K=150),
     "one_key": lambda: small(L=1, K=1, capacity=16),
     "short": lambda: small(L=129, K=5),
     "recent_only": lambda: small(n_beacons_in=0, L=300),
@@ -457,6 +459,8 @@ def _ascending_positions(rng, cap, n_keep, mode):
     ("bf16", 128, 5000, 129, "tail"),
     ("f32", 128, 2000, 1000, "random"),       # 512-byte rows: 32-row chunks
     ("f32", 24, 999, 400, "prefix_kept"),     # 96-byte rows: chunks of 170 rows
+    ("bf16", 64, 3000, 1000, "random"),       # 128-byte rows: 256-row chunks
+    ("f32", 256, 600, 250, "prefix_kept"),    # 1024-byte rows: 32-row chunks
 ])
 def test_compact_inplace(dtype, d, cap, n_keep, mode, dev):
     """In-place compaction equals the out-of-place gather, byte for byte."""
