@@ -156,21 +156,27 @@ __device__ __forceinline__ uint4 ldg_nc_v4(const void *p) {
   return v;
 }
 
-// Pointer to observation row o of KV head (layer, kvh): query head g of the
-// group, row i of [recent (R rows); beacons (nb rows)].  The recent rows are
-// read where they are: a dense [R][d] block per query head, or the newest R
-// rows of a decode-side query ring (ScoreGeom::recent_cap / recent_start).
+// Pointer to observation row o of KV head (layer, kvh).  The group's beacon
+// rows come first (query head by query head, nb each), then its recent rows
+// (R each), so that a row block holds one query head's consecutive beacons
+// or recent rows; measured a little ahead of interleaving the two per query
+// head.  The recent rows are read where they are: a dense [R][d] block per
+// query head, or the newest R rows of a decode-side query ring
+// (ScoreGeom::recent_cap / recent_start).
 __device__ __forceinline__ const uint16_t *obs_row(const ScoreGeom &g, const uint16_t *recent,
                                                    const uint16_t *beacons, int layer, int kvh,
                                                    int o) {
-  const int per = g.R + g.nb;
-  const int gq = o / per;
-  const int i = o - gq * per;
-  const long long qh = static_cast<long long>(layer) * g.n_q_heads +
-                       static_cast<long long>(kvh) * g.group + gq;
-  if (i < g.R)  // row (recent_start + i) mod recent_cap of the head's block (a ring or dense)
-    return recent + (qh * g.recent_cap + (g.recent_start + i) % g.recent_cap) * kDim;
-  return beacons + (qh * g.M + (i - g.R)) * kDim;
+  const int n_bcn = g.group * g.nb;
+  const long long qh0 = static_cast<long long>(layer) * g.n_q_heads +
+                        static_cast<long long>(kvh) * g.group;
+  if (o < n_bcn) {
+    const int gq = o / g.nb;
+    return beacons + ((qh0 + gq) * g.M + (o - gq * g.nb)) * kDim;
+  }
+  const int gq = (o - n_bcn) / g.R;
+  const int i = o - n_bcn - gq * g.R;
+  // row (recent_start + i) mod recent_cap of the head's block (a ring or dense)
+  return recent + ((qh0 + gq) * g.recent_cap + (g.recent_start + i) % g.recent_cap) * kDim;
 }
 
 // Gather observation rows [row0, row0 + nrows) into shared memory as a
