@@ -26,6 +26,18 @@ def test_work_model_14b():
     assert wm["fps"]["bound"] == "tensor" and wm["fps"]["unit"] == "FLOP"
 
 
+def test_select_bytes_14b():
+    """The select streams one word per key and writes K positions per head:
+    the max form's merged order key, or one partial per group of at most 256
+    observation rows for the mean (960 rows: 4 groups)."""
+    wl = synth.WORKLOADS["qwen3_14b"]
+    H, L, K = 320, 32768, 6144
+    assert bench.work_model(wl, "max")["select"]["work"] == pytest.approx((4 * L + 4 * K) * H)
+    assert bench.work_model(wl, "max")["select"]["work"] == pytest.approx(49_807_360)
+    assert bench.work_model(wl, "mean")["select"]["work"] == pytest.approx((4 * 4 * L + 4 * K) * H)
+    assert bench.work_model(wl, "mean")["select"]["work"] == pytest.approx(175_636_480)
+
+
 def test_mufu_bound_14b():
     wm = bench.work_model(synth.WORKLOADS["qwen3_14b"])
     t = bench.mufu_bound_s(wm, {"sm_max_mhz": 1965.0})
