@@ -30,7 +30,8 @@
 // as much as 1.8 rounds' select, gather and MMAs; on the clustered queries of
 // the 14B-shaped workload this policy takes ~8.4 rounds and ~5.8 passes per
 // head, against ~13.6 and ~4.6 for staying eager only until the first round
-// of 8 picks, and ~7.6 and ~6.6 for a pass after every round.
+// of 8 picks, and ~7.6 and ~6.6 for a pass after every round.  The
+// threshold was measured: 20 picks ahead of 8, 12, 16, 24, 32 and 48.
 //
 // The distance pass streams the union [beacons; window] of a query head by
 // TMA in tiles of 128 points (128-byte swizzle, no multicast) through a
@@ -83,7 +84,7 @@ constexpr int kCBlock = kCand * 128;              // one 64-element K block of t
 // the replay's column reads (lane = candidate) free of bank conflicts
 constexpr int kGramStride = kCand + 1;
 constexpr int kListMax = 512;                     // threshold-bin keys ranked directly
-constexpr int kPassBelow = 24;                    // a round with fewer picks is followed by a pass
+constexpr int kPassBelow = 20;                    // a round with fewer picks is followed by a pass
 constexpr int kAhead = 12;                        // L2 prefetch distance of a pass, in tiles
 constexpr int kSmallBytes = 8192;  // barriers, scalars, lists; the u histogram at 4096
 // The persistent histogram of the live points' u over [0, 2] (the range of a
