@@ -1035,7 +1035,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- 3. replay the greedy choice among the candidates (warp 0, four
       // per lane: slots lane, lane+32, lane+64, lane+96).  The argmax in
       // (distance desc, index asc) order takes two warp reductions: the
-      // largest distance key, then the lowest index holding it.
+      // largest distance key, then the lowest index holding it (with the
+      // slot).
       if (warp == 0) {
         float c[4], iv[4];
         int ix[4];
@@ -1066,26 +1067,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const uint32_t kbest = __reduce_max_sync(0xffffffffu, kmax);
           if (kbest == 0u) break;  // no candidate left
+          // the lowest point index holding it, with its slot in the low 7
+          // bits (the union has fewer than 2^24 points), so one reduction
+          // names both the point and its candidate slot
           uint32_t mine = 0xffffffffu;
 #pragma unroll
           for (int q = 0; q < 4; ++q)
-            if (kq[q] == kbest) mine = min(mine, static_cast<uint32_t>(ix[q]));
-          const int best_i = static_cast<int>(__reduce_min_sync(0xffffffffu, mine));
+            if (kq[q] == kbest)
+              mine = min(mine, (static_cast<uint32_t>(ix[q]) << 7) |
+                                   static_cast<uint32_t>(lane + 32 * q));
+          const uint32_t best = __reduce_min_sync(0xffffffffu, mine);
+          const int best_i = static_cast<int>(best >> 7);
+          const int best_a = static_cast<int>(best & 127u);
           const float best_d = __uint_as_float(kbest - 1u);
           if (bounded && !before(best_d, best_i, bd, bi)) break;
-          int own = -1;
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            if (kq[q] == kbest && ix[q] == best_i) own = q;
-          const uint32_t owners = __ballot_sync(0xffffffffu, own >= 0);
-          const int src = __ffs(owners) - 1;
-          const int best_a = __shfl_sync(0xffffffffu, lane + 32 * max(own, 0), src);
-          const float inv_b = __shfl_sync(0xffffffffu, own >= 0 ? iv[own] : 0.f, src);
+          const float inv_b = s.inv[best_i];
           if (lane == 0) s.pick[np] = best_a;
           ++np;
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            if (q == own) taken[q] = true;
+            if (lane + 32 * q == best_a) taken[q] = true;
             if (!taken[q]) {
               // D[a][best] has the candidate as operand A, like the pass
               const float dot = s.gram[(lane + 32 * q) * kGramStride + best_a];
@@ -1257,7 +1258,10 @@ size_t fps_tc_workspace_bytes(const FpsGeom &g) {
 }
 
 bool fps_tc_supported(const FpsGeom &g) {
+  // a union of fewer than 2^24 points: the replay packs a point index and a
+  // 7-bit candidate slot into one 32-bit word
   return g.dtype == BKV_BF16 && g.head_dim == kDim && g.M <= kMaxPick &&
+         static_cast<long long>(g.nb_in) + g.W < (1LL << 24) &&
          static_cast<long long>(g.n_layers) * g.n_q_heads *
                  std::max<long long>(g.M, std::max<long long>(g.W, g.w_cap)) <
              (1LL << 31) - 256;
